@@ -1,0 +1,207 @@
+"""Pins for the oracle's 1x128 activation and 128x128 weight quantizers (CPU).
+
+What fixes the answer:
+* hand-computed worked examples (tests/golden/quant_worked_examples.txt);
+* the grouping geometry of Figure 7 (a) in "The Insider Secrets Of Deepseek
+  Discovered" (one scale per token per 128 channels; one per 128x128 weight
+  block): a single outlier changes exactly its own group;
+* the scaling rule of the same passage (largest magnitude -> FP8 maximum):
+  the amax element encodes to +-448, every code decodes to |v| <= 448, s > 0,
+  an all-zero group gets s = 1, a group whose amax is already 448 gets s = 1
+  and q equal to PyTorch's own E4M3 cast of x.
+"""
+import numpy as np
+import pytest
+import torch
+
+from conftest import golden_lines, hexfloat
+from workloads import bf16_bits, bf16_to_f32, tiny_dense
+
+TILE = 128
+
+
+def _bits(values):
+    return bf16_bits(np.asarray(values, dtype=np.float32))
+
+
+def _parse_worked():
+    ex = {"act": {}, "act2": {}, "w": {}}
+    for tok in golden_lines("quant_worked_examples.txt"):
+        kind = tok[0]
+        if kind in ("act", "act2") and tok[1] == "K":
+            ex[kind]["K"] = int(tok[2])
+            ex[kind]["scales"], ex[kind]["elems"] = {}, []
+        elif kind in ("act_scale", "act2_scale"):
+            ex[kind[:-6]]["scales"][int(tok[1])] = hexfloat(tok[2])
+        elif kind in ("act", "act2"):
+            ex[kind]["elems"].append((int(tok[1]), hexfloat(tok[2]), int(tok[3], 16)))
+        elif kind == "w" and tok[1] == "N":
+            ex["w"].update(N=int(tok[2]), K=int(tok[4]), scales={}, elems=[])
+        elif kind == "w_scale":
+            ex["w"]["scales"][(int(tok[1]), int(tok[2]))] = hexfloat(tok[3])
+        elif kind == "w":
+            ex["w"]["elems"].append((int(tok[1]), int(tok[2]), hexfloat(tok[3]), int(tok[4], 16)))
+    return ex
+
+
+@pytest.mark.parametrize("which", ["act", "act2"])
+def test_worked_activation_examples(orc, which):
+    ex = _parse_worked()[which]
+    K = ex["K"]
+    x = np.zeros((1, K), dtype=np.float32)
+    for k, v, _ in ex["elems"]:
+        x[0, k] = v
+    xb = _bits(x)
+    assert np.array_equal(bf16_to_f32(xb), x), "worked-example inputs must be bf16-exact"
+    q, s = orc.quant_act_1x128(xb)
+    assert s.shape == (1, K // TILE)
+    for kb, sv in ex["scales"].items():
+        assert s[0, kb] == np.float32(sv), (kb, float(s[0, kb]).hex(), sv)
+    expect = np.zeros(K, dtype=np.uint8)
+    for k, _, code in ex["elems"]:
+        expect[k] = code
+    assert np.array_equal(q[0], expect), np.nonzero(q[0] != expect)
+
+
+def test_worked_weight_example(orc):
+    ex = _parse_worked()["w"]
+    N, K = ex["N"], ex["K"]
+    w = np.zeros((N, K), dtype=np.float32)
+    for r, c, v, _ in ex["elems"]:
+        w[r, c] = v
+    q, s = orc.quant_w_128x128(_bits(w))
+    assert s.shape == (N // TILE, K // TILE)
+    for (nb, kb), sv in ex["scales"].items():
+        assert s[nb, kb] == np.float32(sv)
+    expect = np.zeros((N, K), dtype=np.uint8)
+    for r, c, _, code in ex["elems"]:
+        expect[r, c] = code
+    assert np.array_equal(q, expect)
+
+
+def test_zero_groups_get_unit_scale(orc):
+    q, s = orc.quant_act_1x128(np.zeros((3, 256), dtype=np.uint16))
+    assert np.all(s == 1.0) and np.all(q == 0)
+    q, s = orc.quant_w_128x128(np.zeros((2, 128, 256), dtype=np.uint16))
+    assert np.all(s == 1.0) and np.all(q == 0)
+    # -0.0 inputs keep their sign through the unit scale
+    q, s = orc.quant_act_1x128(np.full((1, 128), 0x8000, dtype=np.uint16))
+    assert np.all(s == 1.0) and np.all(q == 0x80)
+
+
+def test_amax_448_groups_reduce_to_plain_cast(orc):
+    """amax == 448 gives s == 1, so q must equal PyTorch's RNE E4M3 cast of x."""
+    rng = np.random.default_rng(11)
+    x = rng.uniform(-447.0, 447.0, size=(4, 512)).astype(np.float32)
+    x[:, ::TILE] = 448.0
+    xb = _bits(x)
+    q, s = orc.quant_act_1x128(xb)
+    assert np.all(s == 1.0)
+    ref = torch.from_numpy(bf16_to_f32(xb)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(q, ref)
+    w = rng.uniform(-447.0, 447.0, size=(256, 256)).astype(np.float32)
+    w[::TILE, ::TILE] = -448.0
+    wb = _bits(w)
+    q, s = orc.quant_w_128x128(wb)
+    assert np.all(s == 1.0)
+    ref = torch.from_numpy(bf16_to_f32(wb)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(q, ref)
+
+
+def test_invariants_on_outlier_workload(orc):
+    d = tiny_dense()
+    table = orc.e4m3_decode_table()
+    for q, s, x, groups in (
+        (*orc.quant_act_1x128(d.a), d.a, "act"),
+        (*orc.quant_w_128x128(d.b), d.b, "w"),
+    ):
+        xf = bf16_to_f32(x)
+        v = table[q]
+        assert np.all(np.isfinite(v)) and np.all(np.abs(v) <= 448.0)
+        assert np.all(s > 0)
+        if groups == "act":
+            g = np.abs(xf).reshape(xf.shape[0], -1, TILE)
+            amax = g.max(axis=2)
+            qa = q.reshape(g.shape)
+            hit = g == amax[..., None]
+            assert np.all((qa[hit] & 0x7F) == 0x7E), "amax element must encode to +-448"
+            assert np.array_equal(s, (amax / np.float32(448.0)).astype(np.float32))
+            # sign preserved
+            xs = xf.reshape(g.shape)
+            nz = xs != 0
+            assert np.all((qa[nz & (xs < 0)] & 0x80) == 0x80)
+        else:
+            N, K = xf.shape
+            g = np.abs(xf).reshape(N // TILE, TILE, K // TILE, TILE)
+            amax = g.max(axis=(1, 3))
+            assert np.array_equal(s, (amax / np.float32(448.0)).astype(np.float32))
+            qb = q.reshape(g.shape)
+            hit = g == amax[:, None, :, None]
+            assert np.all((qb[hit] & 0x7F) == 0x7E)
+
+
+def test_dequantized_error_bound(orc):
+    """|decode(q)*s - x| is at most half an E4M3 step of x/s (plus the f32
+    rounding of the quotient): relative 2^-4 for normals, 2^-10*s absolute
+    in the subnormal range."""
+    d = tiny_dense(seed=5)
+    q, s = orc.quant_act_1x128(d.a)
+    table = orc.e4m3_decode_table()
+    x = bf16_to_f32(d.a).astype(np.float64)
+    sv = np.repeat(s.astype(np.float64), TILE, axis=1)
+    y = x / sv
+    deq = table[q]
+    err = np.abs(deq - y)
+    bound = np.maximum(np.abs(y) * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(err <= bound)
+
+
+def test_single_outlier_changes_only_its_group_act(orc):
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((4, 640)).astype(np.float32)
+    base_q, base_s = orc.quant_act_1x128(_bits(x))
+    m, k = 2, 300
+    x2 = x.copy()
+    x2[m, k] = 1000.0
+    q, s = orc.quant_act_1x128(_bits(x2))
+    ds = np.argwhere(s != base_s)
+    assert ds.tolist() == [[m, k // TILE]]
+    dq = np.argwhere(q != base_q)
+    assert np.all(dq[:, 0] == m) and np.all(dq[:, 1] // TILE == k // TILE)
+    assert len(dq) > 64  # the whole tile is rescaled, not just the outlier
+
+
+def test_single_outlier_changes_only_its_group_w(orc):
+    rng = np.random.default_rng(4)
+    w = (0.02 * rng.standard_normal((384, 512))).astype(np.float32)
+    base_q, base_s = orc.quant_w_128x128(_bits(w))
+    r, c = 200, 77
+    w2 = w.copy()
+    w2[r, c] = 5.0
+    q, s = orc.quant_w_128x128(_bits(w2))
+    assert np.argwhere(s != base_s).tolist() == [[r // TILE, c // TILE]]
+    dq = np.argwhere(q != base_q)
+    assert np.all(dq[:, 0] // TILE == r // TILE) and np.all(dq[:, 1] // TILE == c // TILE)
+    assert len(dq) > 8000
+
+
+def test_weight_batch_matches_per_matrix(orc):
+    rng = np.random.default_rng(8)
+    w = _bits(rng.standard_normal((3, 256, 384)).astype(np.float32))
+    q, s = orc.quant_w_128x128(w)
+    for g in range(3):
+        qg, sg = orc.quant_w_128x128(np.ascontiguousarray(w[g]))
+        assert np.array_equal(q[g], qg) and np.array_equal(s[g], sg)
+
+
+def test_bf16_generator_rounding_matches_torch():
+    """The input generator's float32 -> bf16 conversion is torch's RNE cast."""
+    rng = np.random.default_rng(1)
+    x = (rng.standard_normal(1 << 16) * np.exp(rng.uniform(-20, 20, 1 << 16))).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bf16_bits(x), ref)
+
+
+def test_rejects_bad_shapes(orc):
+    with pytest.raises(ValueError):
+        orc.quant_w_128x128(np.zeros((100, 128), dtype=np.uint16))

@@ -1,0 +1,247 @@
+"""Seeded synthetic inputs for the fine-grained FP8 quantization + GEMM path.
+
+This module holds random draws and input layout only -- none of the method's
+arithmetic (no scaling, no E4M3 encoding, no products).  It is the one module
+that both the CPU oracle side and the CUDA side of the tests and the benchmark
+take their inputs from.  Every tensor is produced as bf16 *bit patterns*
+(``numpy.uint16``) so the same bytes go to the oracle and to the GPU.
+
+Workloads (shapes and distributions of the MoE/dense Linear layers the pages
+discuss; all seeds are numpy PCG64):
+
+* ``tiny_dense``      A 128x512 N(0,1) with 0.1% of entries scaled x100, B 256x512 N(0,1); seed 0.
+* ``dense_fprop``     A 4096x7168 z[m,k]*exp(g[k]) (per-channel log-normal, sigma 1) plus 0.01%
+                      entries set to +-200; B 7168x7168 N(0, 0.02^2); seed 1.
+* ``long_k``          A 2048x16384, B 2048x16384, both U[-1,1] + 0.5; seed 2.
+* ``moe_contiguous``  4096 tokens, top-8 of 32 experts with Zipf(1.1) expert popularity, rows of each
+                      expert padded to a multiple of 128 (pad rows zero); A N(0,1) [M_tot,7168];
+                      B [32,4096,7168] N(0,0.02^2); m_indices = expert of each 128-row block; seed 3.
+* ``moe_masked``      32 experts x capacity 256, valid counts uniform on {0..256}; A [32,256,7168]
+                      N(0,1), B1 [32,4096,7168]; second GEMM A2 [32,256,2048] N(0,1), B2
+                      [32,7168,2048]; weights N(0,0.02^2); seed 4.
+
+Every generator takes size overrides so the tests can draw the same
+distributions at sizes the oracle finishes in seconds.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+TILE = 128
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float32 array -> bf16 bit patterns (uint16), round-to-nearest-even.
+
+    Input preparation only: the generators draw in float32 and store bf16.
+    Non-finite values are not produced by any generator here."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return rounded.astype(np.uint16)
+
+
+def bf16_to_f32(b: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float32 (exact widening)."""
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _normal_bf16(rng: np.random.Generator, shape, std: float = 1.0, chunk_rows: int = 4096) -> np.ndarray:
+    """N(0, std^2) bf16 bits, drawn in row chunks to bound host memory."""
+    shape = tuple(int(s) for s in shape)
+    out = np.empty(shape, dtype=np.uint16)
+    flat = out.reshape(-1, shape[-1]) if len(shape) > 1 else out.reshape(1, -1)
+    for r0 in range(0, flat.shape[0], chunk_rows):
+        r1 = min(flat.shape[0], r0 + chunk_rows)
+        z = rng.standard_normal((r1 - r0, flat.shape[1]), dtype=np.float32)
+        if std != 1.0:
+            z *= np.float32(std)
+        flat[r0:r1] = bf16_bits(z)
+    return out
+
+
+@dataclass
+class Dense:
+    name: str
+    a: np.ndarray  # [M,K] bf16 bits
+    b: np.ndarray  # [N,K] bf16 bits
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def M(self):
+        return self.a.shape[0]
+
+    @property
+    def N(self):
+        return self.b.shape[0]
+
+    @property
+    def K(self):
+        return self.a.shape[1]
+
+    @property
+    def flops(self):
+        return 2.0 * self.M * self.N * self.K
+
+
+def tiny_dense(seed: int = 0, M: int = 128, N: int = 256, K: int = 512, outlier_frac: float = 1e-3,
+               outlier_mult: float = 100.0) -> Dense:
+    rng = np.random.default_rng(seed)
+    a = rng.standard_normal((M, K), dtype=np.float32)
+    n_out = int(round(outlier_frac * M * K))
+    idx = rng.choice(M * K, size=n_out, replace=False)
+    a.reshape(-1)[idx] *= np.float32(outlier_mult)
+    b = rng.standard_normal((N, K), dtype=np.float32)
+    return Dense("tiny_dense", bf16_bits(a), bf16_bits(b), {"seed": seed, "outliers": n_out})
+
+
+def dense_fprop(seed: int = 1, M: int = 4096, N: int = 7168, K: int = 7168, outlier_frac: float = 1e-4,
+                outlier_value: float = 200.0, w_std: float = 0.02) -> Dense:
+    rng = np.random.default_rng(seed)
+    g = rng.standard_normal(K, dtype=np.float32)
+    chan = np.exp(g).astype(np.float32)  # per-channel log-normal magnitude, sigma = 1
+    a = rng.standard_normal((M, K), dtype=np.float32)
+    a *= chan[None, :]
+    n_out = int(round(outlier_frac * M * K))
+    idx = rng.choice(M * K, size=n_out, replace=False)
+    signs = np.where(rng.random(n_out) < 0.5, -1.0, 1.0).astype(np.float32)
+    a.reshape(-1)[idx] = np.float32(outlier_value) * signs
+    a_bits = bf16_bits(a)
+    del a
+    b_bits = _normal_bf16(rng, (N, K), w_std)
+    return Dense("dense_fprop", a_bits, b_bits, {"seed": seed, "outliers": n_out})
+
+
+def long_k(seed: int = 2, M: int = 2048, N: int = 2048, K: int = 16384, shift: float = 0.5) -> Dense:
+    rng = np.random.default_rng(seed)
+    a = rng.uniform(-1.0, 1.0, size=(M, K)).astype(np.float32) + np.float32(shift)
+    b = rng.uniform(-1.0, 1.0, size=(N, K)).astype(np.float32) + np.float32(shift)
+    return Dense("long_k", bf16_bits(a), bf16_bits(b), {"seed": seed})
+
+
+@dataclass
+class Contiguous:
+    name: str
+    a: np.ndarray          # [M_tot,K] bf16 bits (pad rows zero)
+    b: np.ndarray          # [E,N,K] bf16 bits
+    m_indices: np.ndarray  # [M_tot/128] int32
+    counts: np.ndarray     # [E] valid rows per expert
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def M_tot(self):
+        return self.a.shape[0]
+
+    @property
+    def E(self):
+        return self.b.shape[0]
+
+    @property
+    def N(self):
+        return self.b.shape[1]
+
+    @property
+    def K(self):
+        return self.a.shape[1]
+
+    @property
+    def flops(self):
+        """Algorithmic FLOPs: valid (unpadded) rows only."""
+        return 2.0 * float(self.counts.sum()) * self.N * self.K
+
+    @property
+    def flops_padded(self):
+        return 2.0 * self.M_tot * self.N * self.K
+
+
+def zipf_topk_counts(rng: np.random.Generator, tokens: int, E: int, topk: int, alpha: float) -> np.ndarray:
+    """Rows per expert for ``tokens`` tokens each routed to ``topk`` distinct
+    experts.  Expert popularity p_e ~ rank_e^-alpha over a random permutation of
+    ranks; each token samples ``topk`` experts without replacement
+    (Gumbel-top-k on log p)."""
+    ranks = rng.permutation(E) + 1
+    logp = -alpha * np.log(ranks.astype(np.float64))
+    g = rng.gumbel(size=(tokens, E))
+    chosen = np.argsort(-(logp[None, :] + g), axis=1)[:, :topk]
+    return np.bincount(chosen.reshape(-1), minlength=E).astype(np.int64)
+
+
+def moe_contiguous(seed: int = 3, tokens: int = 4096, topk: int = 8, E: int = 32, N: int = 4096, K: int = 7168,
+                   alpha: float = 1.1, w_std: float = 0.02) -> Contiguous:
+    rng = np.random.default_rng(seed)
+    counts = zipf_topk_counts(rng, tokens, E, topk, alpha)
+    padded = (counts + TILE - 1) // TILE * TILE
+    M_tot = int(padded.sum())
+    a = np.zeros((M_tot, K), dtype=np.uint16)
+    m_indices = np.empty(M_tot // TILE, dtype=np.int32)
+    r = 0
+    for e in range(E):
+        c, p = int(counts[e]), int(padded[e])
+        if c:
+            a[r:r + c] = _normal_bf16(rng, (c, K))
+        m_indices[r // TILE:(r + p) // TILE] = e
+        r += p
+    b = _normal_bf16(rng, (E, N, K), w_std)
+    return Contiguous("moe_contiguous", a, b, m_indices, counts, {"seed": seed, "tokens": tokens, "topk": topk})
+
+
+@dataclass
+class Masked:
+    name: str
+    a: np.ndarray         # [E,cap,K] bf16 bits
+    b: np.ndarray         # [E,N,K] bf16 bits
+    masked_m: np.ndarray  # [E] int32
+    a2: np.ndarray | None = None  # second GEMM [E,cap,K2]
+    b2: np.ndarray | None = None  # [E,N2,K2]
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def E(self):
+        return self.a.shape[0]
+
+    @property
+    def cap(self):
+        return self.a.shape[1]
+
+    def flops(self, second: bool = False):
+        b = self.b2 if second else self.b
+        return 2.0 * float(self.masked_m.sum()) * b.shape[1] * b.shape[2]
+
+
+def moe_masked(seed: int = 4, E: int = 32, cap: int = 256, N: int = 4096, K: int = 7168, N2: int = 7168,
+               K2: int = 2048, w_std: float = 0.02, second: bool = True) -> Masked:
+    rng = np.random.default_rng(seed)
+    masked_m = rng.integers(0, cap, size=E, endpoint=True).astype(np.int32)
+    a = _normal_bf16(rng, (E, cap, K))
+    b = _normal_bf16(rng, (E, N, K), w_std)
+    a2 = b2 = None
+    if second:
+        a2 = _normal_bf16(rng, (E, cap, K2))
+        b2 = _normal_bf16(rng, (E, N2, K2), w_std)
+    return Masked("moe_masked", a, b, masked_m, a2, b2, {"seed": seed})
+
+
+def parity_rows(rng: np.random.Generator, M: int, per_tile: int = 2, tile: int = TILE) -> np.ndarray:
+    """Seeded sample of row indices: ``per_tile`` rows from every 128-row tile
+    (first and last row of the tile always included, so ragged tails count)."""
+    rows = []
+    for t0 in range(0, M, tile):
+        t1 = min(M, t0 + tile)
+        pick = {t0, t1 - 1}
+        extra = max(0, per_tile - len(pick))
+        if extra and t1 - t0 > 2:
+            pick.update(int(v) for v in rng.choice(np.arange(t0 + 1, t1 - 1), size=min(extra, t1 - t0 - 2),
+                                                     replace=False))
+        rows.extend(sorted(pick))
+    return np.asarray(rows, dtype=np.int64)
+
+
+CONFIGS = {
+    "tiny_dense": tiny_dense,
+    "dense_fprop": dense_fprop,
+    "long_k": long_k,
+    "moe_contiguous": moe_contiguous,
+    "moe_masked": moe_masked,
+}
