@@ -1,0 +1,369 @@
+// fp8q_api.cu -- the C ABI declared in include/fp8q.h: argument validation,
+// TMA descriptor encoding, tile-shape choice and launches on the caller's
+// stream.  One translation unit holds every kernel so the device status word
+// is a single symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fp8q.h"
+#include "fp8q_gemm.cuh"
+#include "fp8q_ptx.cuh"
+#include "fp8q_quant.cuh"
+
+namespace fp8q {
+
+__device__ uint32_t g_device_status;
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;
+constexpr int kMaxDevices = 64;
+
+std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<uint64_t> g_launches{0};
+
+struct DeviceInfo {
+  bool ready = false;
+  bool supported = false;
+  int num_sms = 0;
+  uint32_t* status = nullptr;  // device address of g_device_status
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Per-device set-up, done once: SM count, arch check, status-word address,
+// and the dynamic shared-memory opt-in of every GEMM instantiation.
+template <int BN, int STAGES, Sched S>
+cudaError_t opt_in_smem() {
+  return cudaFuncSetAttribute(gemm_blockscaled_kernel<BN, STAGES, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              GemmSmem<BN, STAGES>::kDynamicBytes);
+}
+
+constexpr int kStages256 = 4;
+constexpr int kStages128 = 6;
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8Q_ERR_CUDA;
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (!d.ready) {
+      int major = 0, minor = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return FP8Q_ERR_CUDA;
+      d.supported = (major == 10 && minor == 0);
+      d.num_sms = sms;
+      if (d.supported) {
+        if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_device_status) != cudaSuccess)
+          return FP8Q_ERR_CUDA;
+        cudaError_t e = cudaSuccess;
+        if (e == cudaSuccess) e = opt_in_smem<256, kStages256, Sched::kDense>();
+        if (e == cudaSuccess) e = opt_in_smem<256, kStages256, Sched::kContiguous>();
+        if (e == cudaSuccess) e = opt_in_smem<256, kStages256, Sched::kMasked>();
+        if (e == cudaSuccess) e = opt_in_smem<128, kStages128, Sched::kDense>();
+        if (e == cudaSuccess) e = opt_in_smem<128, kStages128, Sched::kContiguous>();
+        if (e == cudaSuccess) e = opt_in_smem<128, kStages128, Sched::kMasked>();
+        if (e != cudaSuccess) return FP8Q_ERR_CUDA;
+      }
+      d.ready = true;
+    }
+  }
+  if (!d.supported) return FP8Q_ERR_UNSUPPORTED;
+  *out = &d;
+  return FP8Q_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// ---------------------------------------------------------------- TMA maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// [rows, K] bytes, row stride K, box = 128 bytes x box_rows, 128-byte swizzle.
+// Rows past `rows` read as zero.
+int make_operand_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FP8Q_ERR_CUDA;
+  const cuuint64_t dims[2] = {K, rows};
+  const cuuint64_t strides[1] = {K};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kSlabK), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- GEMM launch
+struct GemmCall {
+  const uint8_t* qa;
+  const float* sa;
+  const uint8_t* qb;
+  const float* sb;
+  void* c;
+  const int32_t* m_indices;
+  const int32_t* masked_m;
+  int64_t a_rows;   // rows of A's 2-D view
+  int64_t M;        // dense M, M_tot, or cap
+  int64_t N, K, E;
+  int64_t m_tiles;  // per expert for masked
+  int64_t expected_m;
+  int promote;
+};
+
+// Tile width: the candidate whose last wave is fullest, preferring the wide
+// tile (half the shared-memory traffic per FLOP) unless it wastes > 15% more.
+int choose_bn(const GemmCall& g, Sched s, int num_sms) {
+  if (g.N <= 128) return 128;
+  auto eff = [&](int bn) {
+    const double n_tiles = static_cast<double>((g.N + bn - 1) / bn);
+    double m_tiles = static_cast<double>(g.m_tiles) * (s == Sched::kMasked ? g.E : 1);
+    if (s == Sched::kMasked && g.expected_m > 0)
+      m_tiles = static_cast<double>(g.E) * ((g.expected_m + kBlockM - 1) / kBlockM);
+    const double tiles = m_tiles * n_tiles;
+    const double waves = std::ceil(tiles / num_sms);
+    const double work = tiles * bn;                     // useful work in units of 128 x 1 columns
+    const double cost = waves * bn * (bn == 128 ? 1.15 : 1.0);  // narrow tiles run below peak
+    return work / cost;
+  };
+  return eff(128) > eff(256) * 1.0 ? 128 : 256;
+}
+
+template <int BN, int STAGES, Sched S>
+int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
+  CUtensorMap ma, mb;
+  int rc = make_operand_map(&ma, g.qa, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K), kBlockM);
+  if (rc) return rc;
+  rc = make_operand_map(&mb, g.qb, static_cast<uint64_t>(g.E * g.N), static_cast<uint64_t>(g.K), BN);
+  if (rc) return rc;
+  GemmArgs a;
+  a.sa = g.sa;
+  a.sb = g.sb;
+  a.c = static_cast<__nv_bfloat16*>(g.c);
+  a.m_indices = g.m_indices;
+  a.masked_m = g.masked_m;
+  a.status = dev.status;
+  a.timeout_ns = g_timeout_ns.load();
+  a.M = static_cast<int32_t>(g.M);
+  a.N = static_cast<int32_t>(g.N);
+  a.nkb = static_cast<int32_t>(g.K / kSlabK);
+  a.E = static_cast<int32_t>(g.E);
+  a.m_tiles = static_cast<int32_t>(g.m_tiles);
+  a.n_tiles = static_cast<int32_t>((g.N + BN - 1) / BN);
+  a.promote = g.promote;
+  int64_t max_tiles = g.m_tiles * a.n_tiles * (S == Sched::kMasked ? g.E : 1);
+  const int grid = static_cast<int>(max_tiles < dev.num_sms ? max_tiles : dev.num_sms);
+  if (grid <= 0) return FP8Q_OK;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = GemmSmem<BN, STAGES>::kDynamicBytes;
+  cfg.stream = stream;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<BN, STAGES, S>, ma, mb, a);
+  if (e != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
+template <Sched S>
+int run_gemm(const GemmCall& g, cudaStream_t stream) {
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  const int bn = choose_bn(g, S, dev->num_sms);
+  if (bn == 128) return launch_gemm<128, kStages128, S>(g, *dev, stream);
+  return launch_gemm<256, kStages256, S>(g, *dev, stream);
+}
+
+int check_operands(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, const void* c) {
+  if (!qa || !sa || !qb || !sb || !c) return FP8Q_ERR_NULL;
+  if (!aligned(qa, 16) || !aligned(qb, 16) || !aligned(c, 16) || !aligned(sa, 4) || !aligned(sb, 4))
+    return FP8Q_ERR_ALIGN;
+  return FP8Q_OK;
+}
+
+constexpr int64_t kMaxRows = int64_t(1) << 31;
+
+}  // namespace
+
+// Bounded-wait self-test kernel: waits on a barrier nobody completes.
+__global__ void wait_selftest_kernel(uint32_t* status, uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    WaitCtl w{timeout_ns, status, &abort_flag};
+    mbar_wait(smem_u32(&bar), 0, w, 0x7F);
+  }
+}
+
+}  // namespace fp8q
+
+using namespace fp8q;
+
+extern "C" {
+
+int fp8_quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
+  if (M < 0 || K < 0 || K % 128) return FP8Q_ERR_SHAPE;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (!x_bf16 || !q || !s) return FP8Q_ERR_NULL;
+  if (!aligned(x_bf16, 16) || !aligned(q, 16) || !aligned(s, 4)) return FP8Q_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  const int64_t tiles = M * (K / 128);
+  constexpr int kUnroll = 4;
+  const int64_t per_cta = (256 / 16) * kUnroll;
+  int64_t grid = (tiles + per_cta - 1) / per_cta;
+  const int64_t cap = static_cast<int64_t>(dev->num_sms) * 8;
+  if (grid > cap) grid = cap;
+  quant_act_1x128_kernel<kUnroll><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+      static_cast<const uint4*>(x_bf16), reinterpret_cast<uint2*>(q), s, tiles);
+  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
+int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, uint8_t* q, float* s,
+                        cudaStream_t stream) {
+  if (G < 0 || N < 0 || K < 0 || N % 128 || K % 128) return FP8Q_ERR_SHAPE;
+  if (G == 0 || N == 0 || K == 0) return FP8Q_OK;
+  if (!w_bf16 || !q || !s) return FP8Q_ERR_NULL;
+  if (!aligned(w_bf16, 16) || !aligned(q, 16) || !aligned(s, 4)) return FP8Q_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  const int64_t blocks = G * (N / 128) * (K / 128);
+  const int64_t cap = static_cast<int64_t>(dev->num_sms) * 64;
+  const int64_t grid = blocks < cap ? blocks : cap;
+  quant_w_128x128_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(static_cast<const uint8_t*>(w_bf16), q, s,
+                                                                           N, K, blocks);
+  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
+static int dense_common(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, void* c, int64_t M,
+                        int64_t N, int64_t K, int promote, cudaStream_t stream) {
+  if (M < 0 || N < 0 || K < 128 || K % 128 || N % 128 || M >= kMaxRows || N >= kMaxRows || K >= kMaxRows)
+    return FP8Q_ERR_SHAPE;
+  if (M == 0 || N == 0) return FP8Q_OK;
+  int rc = check_operands(qa, sa, qb, sb, c);
+  if (rc) return rc;
+  GemmCall g{qa, sa, qb, sb, c, nullptr, nullptr, M, M, N, K, 1, (M + kBlockM - 1) / kBlockM, 0, promote};
+  return run_gemm<Sched::kDense>(g, stream);
+}
+
+int fp8_gemm_blockscaled(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, void* c_bf16,
+                         int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+  return dense_common(qa, sa, qb, sb, c_bf16, M, N, K, 1, stream);
+}
+
+int fp8_gemm_unpromoted_diag(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, void* c_bf16,
+                             int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+  return dense_common(qa, sa, qb, sb, c_bf16, M, N, K, 0, stream);
+}
+
+int fp8_grouped_gemm_contiguous(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb,
+                                const int32_t* m_indices, void* c_bf16, int64_t M_tot, int64_t N, int64_t K,
+                                int64_t E, cudaStream_t stream) {
+  if (M_tot < 0 || N < 0 || E < 0 || K < 128 || K % 128 || N % 128 || M_tot % 128 || M_tot >= kMaxRows ||
+      K >= kMaxRows || E * N >= kMaxRows)
+    return FP8Q_ERR_SHAPE;
+  if (M_tot == 0 || N == 0) return FP8Q_OK;
+  if (E == 0) return FP8Q_OK;  // every block index is out of range: nothing is written
+  int rc = check_operands(qa, sa, qb, sb, c_bf16);
+  if (rc) return rc;
+  if (!m_indices) return FP8Q_ERR_NULL;
+  if (!aligned(m_indices, 4)) return FP8Q_ERR_ALIGN;
+  GemmCall g{qa, sa, qb, sb, c_bf16, m_indices, nullptr, M_tot, M_tot, N, K, E, M_tot / kBlockM, 0, 1};
+  return run_gemm<Sched::kContiguous>(g, stream);
+}
+
+int fp8_grouped_gemm_masked(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb,
+                            const int32_t* masked_m, void* c_bf16, int64_t E, int64_t cap, int64_t N, int64_t K,
+                            int64_t expected_m, cudaStream_t stream) {
+  if (E < 0 || cap < 0 || N < 0 || K < 128 || K % 128 || N % 128 || cap % 128 || E > kMaxMaskedExperts ||
+      E * cap >= kMaxRows || E * N >= kMaxRows || K >= kMaxRows || expected_m < 0)
+    return FP8Q_ERR_SHAPE;
+  if (E == 0 || cap == 0 || N == 0) return FP8Q_OK;
+  int rc = check_operands(qa, sa, qb, sb, c_bf16);
+  if (rc) return rc;
+  if (!masked_m) return FP8Q_ERR_NULL;
+  if (!aligned(masked_m, 4)) return FP8Q_ERR_ALIGN;
+  GemmCall g{qa, sa, qb, sb, c_bf16, nullptr, masked_m, E * cap, cap, N, K, E, cap / kBlockM, expected_m, 1};
+  return run_gemm<Sched::kMasked>(g, stream);
+}
+
+const char* fp8q_status_string(int status) {
+  switch (status) {
+    case FP8Q_OK: return "ok";
+    case FP8Q_ERR_NULL: return "null pointer";
+    case FP8Q_ERR_SHAPE: return "invalid shape";
+    case FP8Q_ERR_ALIGN: return "misaligned pointer";
+    case FP8Q_ERR_CUDA: return "CUDA error";
+    case FP8Q_ERR_TIMEOUT: return "device wait timed out";
+    case FP8Q_ERR_UNSUPPORTED: return "unsupported device or limit";
+    default: return "unknown status";
+  }
+}
+
+int fp8q_get_device_error(cudaStream_t stream) {
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FP8Q_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof v) != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (v == 0) return FP8Q_OK;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero) != cudaSuccess) return FP8Q_ERR_CUDA;
+  return (v & kDevErrTimeout) ? FP8Q_ERR_TIMEOUT : FP8Q_ERR_CUDA;
+}
+
+int fp8q_set_wait_timeout_ns(uint64_t timeout_ns) {
+  g_timeout_ns.store(timeout_ns ? timeout_ns : kDefaultTimeoutNs);
+  return FP8Q_OK;
+}
+
+int fp8q_selftest_wait_timeout(uint64_t timeout_ns, cudaStream_t stream) {
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(dev->status, timeout_ns);
+  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
+uint64_t fp8q_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

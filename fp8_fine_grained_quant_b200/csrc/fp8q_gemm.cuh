@@ -1,0 +1,397 @@
+// fp8q_gemm.cuh -- block-scaled FP8 GEMM for sm_100a with per-slab promotion.
+//
+// Method ("The Insider Secrets Of Deepseek Discovered", Figure 7 (b); the
+// codingmall DeepSeek-V3 FP8 page, increased accumulation precision): the
+// tensor cores produce one 128-deep K slab's partial sum at a time; each
+// partial is moved to FP32 registers on the CUDA cores, multiplied by the two
+// dequantization scales of that slab (the activation tile's and the weight
+// block's) and added to the running FP32 sum.  The output is rounded to bf16
+// once at the end.  Dense and the two MoE grouped layouts of the DeepGEMM
+// announcement ("Deepgemm lancado ...", contiguous and masked) share one
+// kernel; only the tile scheduler differs.
+//
+// Design (B200):
+//   * persistent CTAs, one per SM, walking a static tile sequence;
+//   * warp 0: TMA producer (one 128-deep K slab of A [128 x 128 B] and
+//     B [BN x 128 B] per pipeline stage, 128-byte swizzle, mbarrier tx count);
+//   * warp 1: allocates TMEM and issues tcgen05.mma.kind::f8f6f4 (M = 128,
+//     N = BN, K = 32, four per slab) into one of two TMEM slab buffers; the
+//     first MMA of every slab overwrites, so each buffer holds exactly one
+//     slab's partial;
+//   * warp 2 builds the masked-layout tile table; warp 3 idles;
+//   * warps 4-11: epilogue; warp w reads TMEM lanes 32*(w%4)..+31 (the rows the
+//     hardware lets it access) and half of the BN columns, applies
+//     acc += (sa * sb) * partial with packed FP32 FMAs, releases the buffer,
+//     and after the last slab stores bf16.  The MMA of slab k+1 runs while
+//     slab k is being promoted.
+//   * every mbarrier wait is bounded; a wait that runs out records a timeout
+//     in the device status word and all roles drain and return.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "fp8q_ptx.cuh"
+
+namespace fp8q {
+
+enum class Sched : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+
+constexpr int kBlockM = 128;
+constexpr int kSlabK = 128;  // promotion interval = scale slab
+constexpr int kGemmThreads = 384;  // warpgroup 0: TMA + MMA (+ scheduler set-up); 1-2: epilogue
+constexpr int kMaxMaskedExperts = 1024;
+
+struct GemmArgs {
+  const float* sa;           // [rows of A][nkb]
+  const float* sb;           // [E][N/128][nkb]
+  __nv_bfloat16* c;          // [rows of A][N]: C row r belongs to A row r in every layout
+  const int32_t* m_indices;  // contiguous: expert of each 128-row block
+  const int32_t* masked_m;   // masked: valid rows per expert
+  uint32_t* status;          // device status word
+  uint64_t timeout_ns;
+  int32_t M;                 // dense: rows of A; contiguous: M_tot; masked: cap
+  int32_t N;
+  int32_t nkb;               // K / 128
+  int32_t E;
+  int32_t m_tiles;           // dense: ceil(M/128); contiguous: M_tot/128; masked: cap/128
+  int32_t n_tiles;           // ceil(N / BN)
+  int32_t promote;           // 1: per-slab promotion; 0: accumulate all of K in TMEM (diagnostic)
+};
+
+struct Tile {
+  int32_t a_row;  // first row in A's [rows, K] view (and in C)
+  int32_t b_row;  // first row in B's [E*N, K] view
+  int32_t n0;     // first output column
+  int32_t e;      // expert (0 for dense)
+  int32_t rows;   // valid rows in this tile (<= 128)
+};
+
+template <int BN, int STAGES>
+struct GemmSmem {
+  static constexpr uint32_t kABytes = kBlockM * kSlabK;  // 16 KB
+  static constexpr uint32_t kBBytes = BN * kSlabK;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr uint32_t kTmemStride = BN <= 128 ? 128 : 256;  // columns between the two slab buffers
+  static constexpr uint32_t kTmemCols = 2 * kTmemStride;          // power of two >= 32
+  static constexpr uint32_t kOffA = 0;
+  static constexpr uint32_t kOffB = STAGES * kABytes;
+  static constexpr uint32_t kOffBars = STAGES * kStageBytes;  // full[S], empty[S], tfull[2], tempty[2], drain
+  static constexpr uint32_t kNumBars = 2 * STAGES + 5;
+  static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;     // tmem slot, abort flag, total tiles
+  static constexpr uint32_t kOffPrefix = (kOffMisc + 16 + 15) / 16 * 16;
+  static constexpr uint32_t kBytes = kOffPrefix + 4 * (kMaxMaskedExperts + 1);
+  static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack for 1024-byte alignment
+};
+
+// ----------------------------------------------------------------- scheduler
+// Masked layout: per-expert counts of 128-row tiles are turned into a prefix
+// over (expert, n-tile, m-tile) once per CTA, in shared memory.
+__device__ __forceinline__ int32_t masked_rows(const GemmArgs& a, int e) {
+  int32_t m = a.masked_m[e];
+  return m < 0 ? 0 : (m > a.M ? a.M : m);
+}
+
+__device__ void build_masked_prefix(const GemmArgs& a, int32_t* prefix, int lane) {
+  // one warp: lane l sums a contiguous chunk of experts, then a warp scan
+  const int chunk = (a.E + 31) / 32;
+  const int e0 = lane * chunk, e1 = min(a.E, e0 + chunk);
+  int32_t local = 0;
+  for (int e = e0; e < e1; ++e) local += ((masked_rows(a, e) + kBlockM - 1) / kBlockM) * a.n_tiles;
+  int32_t incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    int32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  int32_t run = incl - local;
+  for (int e = e0; e < e1; ++e) {
+    prefix[e] = run;
+    run += ((masked_rows(a, e) + kBlockM - 1) / kBlockM) * a.n_tiles;
+  }
+  if (lane == 31) prefix[a.E] = incl;
+}
+
+template <Sched S, int BN>
+__device__ __forceinline__ bool get_tile(const GemmArgs& a, const int32_t* prefix, int32_t t, Tile& tile) {
+  if constexpr (S == Sched::kMasked) {
+    int lo = 0, hi = a.E;  // largest e with prefix[e] <= t
+    while (hi - lo > 1) {
+      int mid = (lo + hi) >> 1;
+      if (prefix[mid] <= t) lo = mid; else hi = mid;
+    }
+    const int e = lo;
+    const int32_t rows_e = masked_rows(a, e);
+    const int32_t mt_count = (rows_e + kBlockM - 1) / kBlockM;
+    const int32_t local = t - prefix[e];
+    const int32_t nt = local / mt_count, mt = local - nt * mt_count;  // m-tile fastest: siblings share B
+    tile.e = e;
+    tile.a_row = e * a.M + mt * kBlockM;
+    tile.rows = min(kBlockM, rows_e - mt * kBlockM);
+    tile.n0 = nt * BN;
+    tile.b_row = e * a.N + tile.n0;
+    return true;
+  } else {
+    const int32_t mt = t / a.n_tiles, nt = t - mt * a.n_tiles;
+    tile.a_row = mt * kBlockM;
+    tile.n0 = nt * BN;
+    if constexpr (S == Sched::kContiguous) {
+      const int32_t e = a.m_indices[mt];
+      if (e < 0 || e >= a.E) return false;
+      tile.e = e;
+      tile.rows = kBlockM;
+    } else {
+      tile.e = 0;
+      tile.rows = min(kBlockM, a.M - tile.a_row);
+    }
+    tile.b_row = tile.e * a.N + tile.n0;
+    return true;
+  }
+}
+
+// ----------------------------------------------------------------- roles
+// Shared-memory barrier addresses (mbarrier objects, 8 bytes each).
+template <int STAGES>
+struct Bars {
+  uint32_t base;
+  __device__ uint32_t full(int s) const { return base + 8u * s; }
+  __device__ uint32_t empty(int s) const { return base + 8u * (STAGES + s); }
+  __device__ uint32_t tfull(int b) const { return base + 8u * (2 * STAGES + b); }
+  __device__ uint32_t tempty(int b) const { return base + 8u * (2 * STAGES + 2 + b); }
+  __device__ uint32_t drain() const { return base + 8u * (2 * STAGES + 4); }
+};
+
+// TMA producer (one thread): one pipeline stage per 128-deep K slab.
+template <int BN, int STAGES, Sched S>
+__device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensorMap* tma_b, const GemmArgs& args,
+                                     const int32_t* prefix, uint32_t s_base, Bars<STAGES> bars, WaitCtl wc,
+                                     int32_t total) {
+  using L = GemmSmem<BN, STAGES>;
+  int stage = 0;
+  uint32_t phase = 0;
+  uint32_t armed = 0, armed_parity = 0;  // per stage: ever armed / parity of its last phase
+  for (int32_t t = blockIdx.x; t < total && !*wc.abort; t += gridDim.x) {
+    Tile tile;
+    if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
+    for (int kb = 0; kb < args.nkb; ++kb) {
+      if (!mbar_wait(bars.empty(stage), phase ^ 1u, wc, 1)) break;
+      mbar_arrive_expect_tx(bars.full(stage), L::kStageBytes);
+      tma_load_2d(s_base + L::kOffA + stage * L::kABytes, tma_a, bars.full(stage), kb * kSlabK, tile.a_row);
+      tma_load_2d(s_base + L::kOffB + stage * L::kBBytes, tma_b, bars.full(stage), kb * kSlabK, tile.b_row);
+      armed |= 1u << stage;
+      armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+      if (++stage == STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+  if (*wc.abort) {
+    // let copies still in flight land before the CTA exits (bounded, 1 ms each)
+    for (int s = 0; s < STAGES; ++s)
+      if (armed & (1u << s)) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(bars.full(s), (armed_parity >> s) & 1u) && globaltimer_ns() - t0 < 1000000ull) {
+        }
+      }
+  }
+}
+
+// MMA issuer (one thread): four K = 32 MMAs per slab into a TMEM slab buffer.
+template <int BN, int STAGES, Sched S>
+__device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* prefix, uint32_t s_base,
+                                       Bars<STAGES> bars, WaitCtl wc, int32_t total, uint32_t tmem_base) {
+  using L = GemmSmem<BN, STAGES>;
+  constexpr uint32_t kIdesc = idesc_e4m3_f32(kBlockM, BN);
+  int stage = 0, buf = 0;
+  uint32_t phase = 0, tphase = 0;
+  bool ok = true;
+  for (int32_t t = blockIdx.x; ok && t < total && !*wc.abort; t += gridDim.x) {
+    Tile tile;
+    if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
+    for (int kb = 0; kb < args.nkb; ++kb) {
+      const bool new_acc = args.promote || kb == 0;
+      if (new_acc) {
+        if (!mbar_wait(bars.tempty(buf), tphase ^ 1u, wc, 2)) { ok = false; break; }
+        tc_fence_after();
+      }
+      if (!mbar_wait(bars.full(stage), phase, wc, 3)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + buf * L::kTmemStride;
+      const uint64_t adesc = smem_desc_k_sw128(s_base + L::kOffA + stage * L::kABytes);
+      const uint64_t bdesc = smem_desc_k_sw128(s_base + L::kOffB + stage * L::kBBytes);
+#pragma unroll
+      for (int k = 0; k < kSlabK / 32; ++k)
+        mma_e4m3(d_tmem, adesc + 2u * k, bdesc + 2u * k, kIdesc, (new_acc && k == 0) ? 0u : 1u);
+      mma_commit(bars.empty(stage));
+      if (++stage == STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+      if (args.promote || kb == args.nkb - 1) {
+        mma_commit(bars.tfull(buf));
+        buf ^= 1;
+        if (buf == 0) tphase ^= 1u;
+      }
+    }
+  }
+  // every issued MMA completes before TMEM is released
+  mma_commit(bars.drain());
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bars.drain(), 0) && globaltimer_ns() - t0 < args.timeout_ns) {
+  }
+}
+
+// Epilogue warp: promotion of every slab partial into FP32 registers, then the
+// bf16 store of the finished tile.  Warp w owns TMEM lanes 32*(w%4)..+31 (tile
+// rows) and columns [half*BN/2, (half+1)*BN/2).  For BN in {128, 256} each
+// half lies inside one 128-column weight block, so one sb value per slab.
+template <int BN, int STAGES, Sched S>
+__device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* prefix, Bars<STAGES> bars, WaitCtl wc,
+                                         int32_t total, uint32_t tmem_base, int warp, int lane) {
+  using L = GemmSmem<BN, STAGES>;
+  constexpr int kHalf = BN / 2;
+  constexpr int kChunk = 32;
+  constexpr int kChunks = kHalf / kChunk;
+  static_assert(kHalf <= 128 && 128 % kHalf == 0, "each half must sit inside one 128-column scale block");
+  const int quad = warp & 3;
+  const int half = (warp - 4) >> 2;
+  const int r = quad * 32 + lane;
+  const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+  const int nkb = args.nkb;
+  const int nnb = args.N / 128;
+  int buf = 0;
+  uint32_t tphase = 0;
+  for (int32_t t = blockIdx.x; t < total && !*wc.abort; t += gridDim.x) {
+    Tile tile;
+    if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
+    const bool row_ok = r < tile.rows;
+    const int col0 = tile.n0 + half * kHalf;
+    const bool col_ok = col0 < args.N;
+    const float* sa_row = args.sa + static_cast<int64_t>(tile.a_row + (row_ok ? r : 0)) * nkb;
+    const float* sb_row = args.sb + (static_cast<int64_t>(tile.e) * nnb + (col_ok ? col0 / 128 : 0)) * nkb;
+    float acc[kHalf];
+#pragma unroll
+    for (int i = 0; i < kHalf; ++i) acc[i] = 0.0f;
+
+    const int n_reads = args.promote ? nkb : 1;
+    // the next slab's scales are fetched one slab ahead
+    float sa_next = row_ok ? __ldg(sa_row) : 0.0f;
+    float sb_next = col_ok ? __ldg(sb_row) : 0.0f;
+    bool ok = true;
+    for (int it = 0; it < n_reads; ++it) {
+      const float scale = sa_next * sb_next;
+      if (it + 1 < n_reads) {
+        sa_next = row_ok ? __ldg(sa_row + it + 1) : 0.0f;
+        sb_next = col_ok ? __ldg(sb_row + it + 1) : 0.0f;
+      }
+      // warp-uniform outcome: the tcgen05.ld below must be executed by all 32 lanes
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bars.tfull(buf), tphase, wc, 4))) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t t_buf = t_lane + buf * L::kTmemStride + half * kHalf;
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
+        uint32_t v[kChunk];
+        tmem_ld_32x32b_x32(t_buf + c * kChunk, v);
+        tmem_ld_wait(v);
+#pragma unroll
+        for (int j = 0; j < kChunk; j += 2)
+          ffma2(acc[c * kChunk + j], acc[c * kChunk + j + 1], __uint_as_float(v[j]), __uint_as_float(v[j + 1]), scale);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.tempty(buf));
+      buf ^= 1;
+      if (buf == 0) tphase ^= 1u;
+    }
+    if (!ok) break;
+    if (row_ok && col_ok) {
+      __nv_bfloat16* crow = args.c + static_cast<int64_t>(tile.a_row + r) * args.N + col0;
+#pragma unroll
+      for (int j = 0; j < kHalf; j += 8) {
+        __nv_bfloat162 p0 = __floats2bfloat162_rn(acc[j], acc[j + 1]);
+        __nv_bfloat162 p1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
+        __nv_bfloat162 p2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
+        __nv_bfloat162 p3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
+        uint4 o;
+        o.x = *reinterpret_cast<uint32_t*>(&p0);
+        o.y = *reinterpret_cast<uint32_t*>(&p1);
+        o.z = *reinterpret_cast<uint32_t*>(&p2);
+        o.w = *reinterpret_cast<uint32_t*>(&p3);
+        *reinterpret_cast<uint4*>(crow + j) = o;
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------------- kernel
+template <int BN, int STAGES, Sched S>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                            const GemmArgs args) {
+  using L = GemmSmem<BN, STAGES>;
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "UMMA N for M=128 must be a multiple of 16 in [16,256]");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const Bars<STAGES> bars{s_base + L::kOffBars};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
+  int32_t* total_slot = reinterpret_cast<int32_t*>(smem + L::kOffMisc + 8);
+  int32_t* prefix = reinterpret_cast<int32_t*>(smem + L::kOffPrefix);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const WaitCtl wc{args.timeout_ns, args.status, abort_flag};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bars.full(s), 1);
+      mbar_init(bars.empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bars.tfull(b), 1);
+      mbar_init(bars.tempty(b), 8);  // one arrival per epilogue warp
+    }
+    mbar_init(bars.drain(), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_map(&tma_a);
+    tma_prefetch_map(&tma_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  if constexpr (S == Sched::kMasked) {
+    if (warp == 2) build_masked_prefix(args, prefix, lane);
+  } else {
+    if (threadIdx.x == 64) *total_slot = args.m_tiles * args.n_tiles;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if constexpr (S == Sched::kMasked) {
+    if (threadIdx.x == 64) *total_slot = prefix[args.E];
+    __syncthreads();
+  }
+  const uint32_t tmem_base = *tmem_slot;
+  const int32_t total = *total_slot;
+
+  if (warp < 4) {
+    if (warp == 0 && lane == 0) produce<BN, STAGES, S>(&tma_a, &tma_b, args, prefix, s_base, bars, wc, total);
+    if (warp == 1 && lane == 0) issue_mma<BN, STAGES, S>(args, prefix, s_base, bars, wc, total, tmem_base);
+  } else {
+    epilogue<BN, STAGES, S>(args, prefix, bars, wc, total, tmem_base, warp, lane);
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+}  // namespace fp8q

@@ -1,0 +1,181 @@
+/*
+ * fp8q.h -- C ABI of the fine-grained FP8 quantization + block-scaled FP8 GEMM
+ * library for NVIDIA B200 (sm_100a).
+ *
+ * The method (sources cited by page title and passage):
+ *  - "The Insider Secrets Of Deepseek Discovered", FP8 mixed-precision passage:
+ *    activations are scaled per 1x128 tile (one scale per token per 128
+ *    channels) and weights per 128x128 block, Figure 7 (a); the group's largest
+ *    magnitude is mapped onto the largest FP8 value; tensor-core partial sums
+ *    are promoted to FP32 on CUDA cores at fixed K intervals, where the
+ *    dequantization scales are applied, Figure 7 (b).
+ *  - codingmall "DeepSeek-V3 FP8" page (Korean), sections on online
+ *    quantization (scales computed from the current tile), increased
+ *    accumulation precision, and the unified E4M3 format.
+ *  - "Deepgemm lancado no dia 4 da semana de codigo aberto Deepseek", sections
+ *    "O que e FP8?" (E4M3: 1 sign, 4 exponent, 3 mantissa bits) and
+ *    "Necessidade de DeepGemm" / "Principais caracteristicas" (dense GEMM plus
+ *    two MoE grouped layouts, contiguous and masked).
+ *
+ * Conventions shared by every entry point:
+ *  - All data pointers are DEVICE pointers on the current CUDA device; the
+ *    caller owns and allocates every buffer.  No call allocates memory.
+ *  - Every call is asynchronous on `stream` and never synchronizes the host.
+ *  - All tensors are dense and row-major (last index fastest).  FP8 tensors
+ *    hold E4M3FN codes (bias 7, largest finite 448 = 0x7E, NaN = 0x7F/0xFF, no
+ *    infinities; byte-compatible with torch.float8_e4m3fn).  bf16 tensors hold
+ *    IEEE bfloat16.  Scale tensors are float32.
+ *  - Quantization rule (per group): s = fl32(amax / 448) with IEEE division,
+ *    s = 1 when that is zero; q = E4M3(fl32(x / s)) rounded to nearest even,
+ *    saturating at +-448, subnormal E4M3 codes down to 2^-9, sign of zero kept.
+ *  - Argument errors return a non-zero status before anything is launched
+ *    (no side effects).  A failed launch returns FP8Q_ERR_CUDA.
+ *  - Pointer alignment: bf16 / FP8 / output pointers 16 bytes; scale and index
+ *    pointers 4 bytes.
+ *  - Non-finite inputs are outside the contract (results unspecified, no fault).
+ *  - Every on-device wait is bounded (default 4 s, see fp8q_set_wait_timeout_ns);
+ *    a wait that runs out records FP8Q_ERR_TIMEOUT in a device status word,
+ *    the kernel releases its resources and returns, and the host reads the
+ *    word with fp8q_get_device_error.
+ */
+#ifndef FP8Q_H_
+#define FP8Q_H_
+
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define FP8Q_API __attribute__((visibility("default")))
+#else
+#define FP8Q_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FP8Q_OK = 0,
+  FP8Q_ERR_NULL = 1,        /* a required pointer is NULL */
+  FP8Q_ERR_SHAPE = 2,       /* a size is negative, not a multiple of 128 where required, or too large */
+  FP8Q_ERR_ALIGN = 3,       /* a pointer is not aligned as required */
+  FP8Q_ERR_CUDA = 4,        /* the CUDA runtime/driver reported an error */
+  FP8Q_ERR_TIMEOUT = 5,     /* a bounded on-device wait ran out (read via fp8q_get_device_error) */
+  FP8Q_ERR_UNSUPPORTED = 6  /* device is not sm_100 or a limit of this build is exceeded */
+} fp8q_status;
+
+/*
+ * Activation quantization, 1x128 tiles ("The Insider Secrets Of Deepseek
+ * Discovered", Figure 7 (a), item 1; codingmall page, online quantization).
+ *   x_bf16 : [M, K] bf16, read only.
+ *   q      : [M, K] E4M3 codes, written.
+ *   s      : [M, K/128] float32, written; s[m, kb] is the scale of
+ *            x[m, 128*kb .. 128*kb+127].
+ * K must be a multiple of 128.  M == 0 or K == 0 is a no-op.
+ */
+FP8Q_API int fp8_quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream);
+
+/*
+ * Weight quantization, 128x128 blocks (same passage, item 2).
+ *   w_bf16 : [G, N, K] bf16 (G stacked [out_features, in_features] matrices;
+ *            G = 1 for one matrix), read only.
+ *   q      : [G, N, K] E4M3 codes, written.
+ *   s      : [G, N/128, K/128] float32, written; s[g, nb, kb] is the scale of
+ *            rows 128*nb..+127, columns 128*kb..+127 of matrix g.
+ * N and K must be multiples of 128.  Any zero size is a no-op.
+ */
+FP8Q_API int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, uint8_t* q, float* s,
+                        cudaStream_t stream);
+
+/*
+ * Dense block-scaled FP8 GEMM, C = A * B^T, with promotion at every 128-wide
+ * K slab ("The Insider Secrets Of Deepseek Discovered", Figure 7 (b); codingmall
+ * page, increased accumulation precision):
+ *   C[m,n] = bf16_rne( sum_kb sa[m,kb] * sb[n/128,kb] * sum_{k in slab kb} A[m,k] * B[n,k] )
+ * where each slab's partial sum comes from the tensor cores in FP32 and the
+ * scaled sum over slabs is kept in FP32 registers.
+ *   qa : [M, K] E4M3, sa : [M, K/128] f32   (from fp8_quant_act_1x128)
+ *   qb : [N, K] E4M3, sb : [N/128, K/128] f32 (from fp8_quant_w_128x128, G = 1)
+ *   c_bf16 : [M, N] bf16, written (every element).
+ * K >= 128 and K, N multiples of 128; any M >= 0 (M == 0 or N == 0: no-op).
+ */
+FP8Q_API int fp8_gemm_blockscaled(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, void* c_bf16,
+                         int64_t M, int64_t N, int64_t K, cudaStream_t stream);
+
+/*
+ * Grouped GEMM, contiguous layout ("Deepgemm lancado ...", MoE grouped GEMM
+ * kinds): the rows of all experts are concatenated, each expert's run padded
+ * to a multiple of 128 rows.
+ *   qa : [M_tot, K], sa : [M_tot, K/128]
+ *   qb : [E, N, K], sb : [E, N/128, K/128]
+ *   m_indices : [M_tot/128] int32 (device): expert of each 128-row block.
+ *   c_bf16 : [M_tot, N] bf16.  Rows of block b are A[b]*B[m_indices[b]]^T.
+ *   A block whose index is outside [0, E) is skipped and its C rows are left
+ *   unwritten.  Padding rows are computed like any row (zero rows give zero).
+ * M_tot, N, K multiples of 128, K >= 128.
+ */
+FP8Q_API int fp8_grouped_gemm_contiguous(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb,
+                                const int32_t* m_indices, void* c_bf16, int64_t M_tot, int64_t N, int64_t K,
+                                int64_t E, cudaStream_t stream);
+
+/*
+ * Grouped GEMM, masked layout (same page): expert e owns a fixed capacity of
+ * `cap` rows of which only the first masked_m[e] are valid; the counts stay on
+ * the device, so the call never synchronizes and can sit in a CUDA graph.
+ *   qa : [E, cap, K], sa : [E, cap, K/128]
+ *   qb : [E, N, K],   sb : [E, N/128, K/128]
+ *   masked_m : [E] int32 (device); values are clamped to [0, cap].
+ *   c_bf16 : [E, cap, N] bf16; rows m >= masked_m[e] are left unwritten.
+ *   expected_m : hint of the typical valid count (may be 0); results never
+ *   depend on it.
+ * cap, N, K multiples of 128, K >= 128, E <= 1024.
+ */
+FP8Q_API int fp8_grouped_gemm_masked(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb,
+                            const int32_t* masked_m, void* c_bf16, int64_t E, int64_t cap, int64_t N, int64_t K,
+                            int64_t expected_m, cudaStream_t stream);
+
+/*
+ * Accumulation diagnostic ("The Insider Secrets Of Deepseek Discovered": the
+ * drift of limited-precision tensor-core accumulation over long K, Figure 7 (b)
+ * is its remedy).  Same operands and layouts as fp8_gemm_blockscaled, but the
+ * whole K range is accumulated inside the tensor cores with no promotion; the
+ * result is scaled once by sa[m,0] * sb[n/128,0].  Only meaningful for
+ * per-tensor scales (every sa and sb entry equal); used to measure the
+ * tensor cores' own accumulation precision.  Not part of the quantized path.
+ */
+FP8Q_API int fp8_gemm_unpromoted_diag(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, void* c_bf16,
+                             int64_t M, int64_t N, int64_t K, cudaStream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+FP8Q_API const char* fp8q_status_string(int status);
+
+/*
+ * Synchronizes `stream`, then reads and clears the device status word that
+ * bounded waits write.  Returns FP8Q_OK, FP8Q_ERR_TIMEOUT, or FP8Q_ERR_CUDA if
+ * the synchronization itself failed.
+ */
+FP8Q_API int fp8q_get_device_error(cudaStream_t stream);
+
+/* Sets the limit of every later on-device wait, in nanoseconds (0 restores
+ * the 4 s default).  Host-side setting; affects launches made after it. */
+FP8Q_API int fp8q_set_wait_timeout_ns(uint64_t timeout_ns);
+
+/*
+ * Self-test of the bounded-wait path: launches one CTA that waits on an
+ * mbarrier nothing will ever complete, with the given limit, so the wait runs
+ * out, records FP8Q_ERR_TIMEOUT and the kernel returns normally.  Nothing
+ * faults or hangs.  Returns the launch status; read the recorded status with
+ * fp8q_get_device_error.
+ */
+FP8Q_API int fp8q_selftest_wait_timeout(uint64_t timeout_ns, cudaStream_t stream);
+
+/* Number of the library's kernels launched since load (host-side counter),
+ * for launch accounting in benchmarks. */
+FP8Q_API uint64_t fp8q_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H_ */

@@ -1,0 +1,135 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol the
+header declares, and rejects bad arguments before touching the device.
+
+No call here reaches CUDA: every argument set below fails host-side
+validation (shape, NULL or alignment), which the library checks first.
+"""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import fp8_fine_grained_quant_b200 as fq
+
+ROOT = Path(__file__).resolve().parents[1]
+HEADER = ROOT / "include" / "fp8q.h"
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    return re.findall(r"^FP8Q_API\s+[\w\s\*]+?\b(\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for required in ("fp8_quant_act_1x128", "fp8_quant_w_128x128", "fp8_gemm_blockscaled",
+                     "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked", "fp8q_status_string",
+                     "fp8q_get_device_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = fq.lib()
+    raw = ctypes.CDLL(str(fq.LIB_PATH))
+    for name in declared_functions():
+        assert hasattr(raw, name), name
+        assert name in fq.EXPORTS, "binding lacks %s" % name
+        assert hasattr(lib, name)
+    assert set(fq.EXPORTS) == set(declared_functions())
+
+
+def test_internal_symbols_hidden():
+    out = ctypes.CDLL(str(fq.LIB_PATH))
+    with pytest.raises(AttributeError):
+        out.make_operand_map  # noqa: B018  (C++ internals are not exported)
+
+
+def test_status_strings():
+    assert fq.status_string(0) == "ok"
+    for s in range(1, 7):
+        assert fq.status_string(s) not in ("ok", "unknown status")
+    assert fq.status_string(99) == "unknown status"
+
+
+A16 = 0x10000  # a 16-byte aligned fake address; never dereferenced
+A4 = 0x10004   # 4-byte aligned only
+A1 = 0x10001
+
+
+def _call(name, *args):
+    return getattr(fq.lib(), name)(*args)
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((A16, 4, 100, A16, A16, None), fq.ERR_SHAPE),     # K not a multiple of 128
+    ((A16, -1, 128, A16, A16, None), fq.ERR_SHAPE),
+    ((A16, 0, 128, A16, A16, None), fq.OK),            # empty: no-op
+    ((A16, 4, 0, A16, A16, None), fq.OK),
+    ((None, 4, 128, A16, A16, None), fq.ERR_NULL),
+    ((A16, 4, 128, None, A16, None), fq.ERR_NULL),
+    ((A4, 4, 128, A16, A16, None), fq.ERR_ALIGN),
+    ((A16, 4, 128, A4, A16, None), fq.ERR_ALIGN),
+    ((A16, 4, 128, A16, A1, None), fq.ERR_ALIGN),
+])
+def test_quant_act_validation(args, expect):
+    assert _call("fp8_quant_act_1x128", *args) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((A16, 1, 100, 128, A16, A16, None), fq.ERR_SHAPE),
+    ((A16, 1, 128, 129, A16, A16, None), fq.ERR_SHAPE),
+    ((A16, 0, 128, 128, A16, A16, None), fq.OK),
+    ((None, 1, 128, 128, A16, A16, None), fq.ERR_NULL),
+    ((A16, 2, 128, 128, A16, A1, None), fq.ERR_ALIGN),
+])
+def test_quant_w_validation(args, expect):
+    assert _call("fp8_quant_w_128x128", *args) == expect
+
+
+@pytest.mark.parametrize("name", ["fp8_gemm_blockscaled", "fp8_gemm_unpromoted_diag"])
+@pytest.mark.parametrize("mnk,ptrs,expect", [
+    ((128, 256, 100), (A16,) * 5, fq.ERR_SHAPE),
+    ((128, 200, 128), (A16,) * 5, fq.ERR_SHAPE),
+    ((128, 256, 0), (A16,) * 5, fq.ERR_SHAPE),   # K >= 128 required
+    ((-1, 256, 128), (A16,) * 5, fq.ERR_SHAPE),
+    ((0, 256, 128), (A16,) * 5, fq.OK),
+    ((128, 0, 128), (A16,) * 5, fq.OK),
+    ((128, 256, 128), (None, A16, A16, A16, A16), fq.ERR_NULL),
+    ((128, 256, 128), (A16, A16, A16, A16, None), fq.ERR_NULL),
+    ((128, 256, 128), (A4, A16, A16, A16, A16), fq.ERR_ALIGN),
+    ((128, 256, 128), (A16, A1, A16, A16, A16), fq.ERR_ALIGN),
+    ((128, 256, 128), (A16, A16, A16, A16, A4), fq.ERR_ALIGN),
+])
+def test_gemm_validation(name, mnk, ptrs, expect):
+    assert _call(name, *ptrs, *mnk, None) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((A16, A16, A16, A16, A16, A16, 200, 256, 128, 4), fq.ERR_SHAPE),   # M_tot % 128
+    ((A16, A16, A16, A16, A16, A16, 256, 256, 100, 4), fq.ERR_SHAPE),
+    ((A16, A16, A16, A16, A16, A16, 0, 256, 128, 4), fq.OK),
+    ((A16, A16, A16, A16, A16, A16, 256, 256, 128, 0), fq.OK),          # no expert: nothing written
+    ((A16, A16, A16, A16, None, A16, 256, 256, 128, 4), fq.ERR_NULL),
+    ((A16, A16, A16, A16, A1, A16, 256, 256, 128, 4), fq.ERR_ALIGN),
+])
+def test_contiguous_validation(args, expect):
+    assert _call("fp8_grouped_gemm_contiguous", *args, None) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((A16, A16, A16, A16, A16, A16, 4, 200, 256, 128, 0), fq.ERR_SHAPE),  # cap % 128
+    ((A16, A16, A16, A16, A16, A16, 2000, 128, 256, 128, 0), fq.ERR_SHAPE),  # E > 1024
+    ((A16, A16, A16, A16, A16, A16, 4, 128, 256, 128, -1), fq.ERR_SHAPE),
+    ((A16, A16, A16, A16, A16, A16, 0, 128, 256, 128, 0), fq.OK),
+    ((A16, A16, A16, A16, None, A16, 4, 128, 256, 128, 0), fq.ERR_NULL),
+    ((A16, A16, A16, A16, A1, A16, 4, 128, 256, 128, 0), fq.ERR_ALIGN),
+])
+def test_masked_validation(args, expect):
+    assert _call("fp8_grouped_gemm_masked", *args, None) == expect
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        fq.fp8_quant_act_1x128(torch.zeros(4, 128, dtype=torch.bfloat16))

@@ -1,0 +1,206 @@
+"""GPU block-scaled GEMMs vs the oracle's float64 dequantized-input product.
+
+Tolerance (written here, from the target): max |C - C_ref| <= 1e-2 * rms(C_ref)
+and max relative error <= 2e-3 over elements with |C_ref| >= 0.1 * rms(C_ref)
+(see parity.py).  The oracle quantizes the same bf16 inputs itself; nothing it
+compares against comes from the GPU.  Small shapes are compared in full
+(several tiles, ragged tails); full-size workloads on a seeded row sample that
+covers every 128-row tile (first and last row of each), every expert and all
+N columns.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import fp8_fine_grained_quant_b200 as fq
+import workloads as wl
+from parity import assert_gemm_close, bf16_bits_of, to_torch_bf16
+
+pytestmark = pytest.mark.gpu
+TILE = 128
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+def _quantize_both(a_bits, b_bits, dev):
+    """GPU quantization (for the GPU GEMM) and oracle quantization (for the
+    reference).  The quantizer tests establish that both are identical."""
+    a = to_torch_bf16(a_bits.reshape(-1, a_bits.shape[-1]), dev)
+    b = to_torch_bf16(b_bits, dev)
+    qa, sa = fq.fp8_quant_act_1x128(a)
+    qb, sb = fq.fp8_quant_w_128x128(b)
+    oqa, osa = oracle.quant_act_1x128(np.ascontiguousarray(a_bits.reshape(-1, a_bits.shape[-1])))
+    oqb, osb = oracle.quant_w_128x128(b_bits)
+    return (qa, sa, qb, sb), (oqa, osa, oqb, osb)
+
+
+def _finish(dev):
+    torch.cuda.synchronize(dev)
+    assert fq.get_device_error(device=dev) == fq.OK
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (128, 256, 512),    # one tile
+    (1, 128, 128),      # single row, single slab
+    (300, 384, 640),    # ragged M, N = 3 weight blocks
+    (257, 512, 1024),
+    (129, 2048, 256),
+    (64, 7168, 384),    # wide N
+    (640, 128, 2048),   # N = one block
+])
+def test_dense_small_full(dev, M, N, K):
+    rng = np.random.default_rng(M + 3 * N + 7 * K)
+    a = rng.standard_normal((M, K)).astype(np.float32) * np.exp(rng.standard_normal(K)).astype(np.float32)
+    b = (0.02 * rng.standard_normal((N, K))).astype(np.float32)
+    (qa, sa, qb, sb), (oqa, osa, oqb, osb) = _quantize_both(wl.bf16_bits(a), wl.bf16_bits(b), dev)
+    c = fq.fp8_gemm_blockscaled(qa, sa, qb, sb)
+    _finish(dev)
+    ref = oracle.gemm_blockscaled(oqa, osa, oqb, osb)
+    assert_gemm_close(bf16_bits_of(c), ref, "dense %dx%dx%d" % (M, N, K))
+
+
+def test_tiny_dense_workload(dev):
+    d = wl.tiny_dense()
+    (qa, sa, qb, sb), (oqa, osa, oqb, osb) = _quantize_both(d.a, d.b, dev)
+    c = fq.fp8_gemm_blockscaled(qa, sa, qb, sb)
+    _finish(dev)
+    assert_gemm_close(bf16_bits_of(c), oracle.gemm_blockscaled(oqa, osa, oqb, osb), "tiny_dense")
+
+
+@pytest.mark.parametrize("name", ["dense_fprop", "long_k"])
+def test_dense_workloads_sampled(dev, name):
+    d = wl.CONFIGS[name]()
+    (qa, sa, qb, sb), (oqa, osa, oqb, osb) = _quantize_both(d.a, d.b, dev)
+    c = fq.fp8_gemm_blockscaled(qa, sa, qb, sb)
+    _finish(dev)
+    rows = wl.parity_rows(np.random.default_rng(77), d.M, per_tile=2)
+    ref = oracle.gemm_blockscaled(oqa, osa, oqb, osb, rows=rows)
+    assert_gemm_close(bf16_bits_of(c)[rows], ref, name)
+
+
+def test_all_ones_closed_form(dev):
+    M, N, K = 256, 512, 1024
+    a = torch.ones((M, K), dtype=torch.bfloat16, device=dev)
+    b = torch.ones((N, K), dtype=torch.bfloat16, device=dev)
+    qa, sa = fq.fp8_quant_act_1x128(a)
+    qb, sb = fq.fp8_quant_w_128x128(b)
+    c = fq.fp8_gemm_blockscaled(qa, sa, qb, sb)
+    _finish(dev)
+    s = float(np.float32(1.0) / np.float32(448.0))
+    closed = K * (448.0 * s) ** 2
+    assert_gemm_close(bf16_bits_of(c), np.full((M, N), closed), "all-ones")
+
+
+def test_output_rows_beyond_m_untouched(dev):
+    """A ragged M writes exactly M rows of the caller's buffer."""
+    M, N, K = 130, 256, 256
+    rng = np.random.default_rng(5)
+    a = wl.bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    b = wl.bf16_bits(rng.standard_normal((N, K)).astype(np.float32))
+    (qa, sa, qb, sb), _ = _quantize_both(a, b, dev)
+    buf = torch.full((M + 126, N), 7.0, dtype=torch.bfloat16, device=dev)
+    fq.fp8_gemm_blockscaled(qa, sa, qb, sb, out=buf[:M])
+    _finish(dev)
+    assert torch.all(buf[M:] == 7.0)
+
+
+# ------------------------------------------------------------------ contiguous
+def _contiguous_case(dev, d, rows_per_block=2):
+    (qa, sa, qb, sb), (oqa, osa, oqb, osb) = _quantize_both(d.a, d.b, dev)
+    mi = torch.from_numpy(d.m_indices).to(dev)
+    c = fq.fp8_grouped_gemm_contiguous(qa, sa, qb.view(d.b.shape), sb, mi)
+    _finish(dev)
+    rows = wl.parity_rows(np.random.default_rng(3), d.M_tot, per_tile=rows_per_block)
+    ref = oracle.grouped_contiguous(oqa, osa, oqb, osb, d.m_indices, rows=rows)
+    assert_gemm_close(bf16_bits_of(c)[rows], ref, d.name)
+
+
+def test_contiguous_small(dev):
+    _contiguous_case(dev, wl.moe_contiguous(tokens=96, topk=4, E=6, N=384, K=512, seed=21), rows_per_block=128)
+
+
+def test_contiguous_full(dev):
+    _contiguous_case(dev, wl.moe_contiguous())
+
+
+def test_contiguous_skips_out_of_range_blocks(dev):
+    d = wl.moe_contiguous(tokens=64, topk=4, E=4, N=256, K=256, seed=8)
+    (qa, sa, qb, sb), (oqa, osa, oqb, osb) = _quantize_both(d.a, d.b, dev)
+    mi = d.m_indices.copy()
+    mi[0] = -1
+    mi[-1] = d.E  # out of range too
+    out = torch.full((d.M_tot, d.N), 3.0, dtype=torch.bfloat16, device=dev)
+    fq.fp8_grouped_gemm_contiguous(qa, sa, qb.view(d.b.shape), sb, torch.from_numpy(mi).to(dev), out=out)
+    _finish(dev)
+    got = bf16_bits_of(out)
+    assert np.all(got[:TILE] == 0x4040) and np.all(got[-TILE:] == 0x4040)  # bf16 3.0 untouched
+    ref = oracle.grouped_contiguous(oqa, osa, oqb, osb, mi)
+    assert_gemm_close(got[TILE:-TILE], ref[TILE:-TILE], "contiguous middle")
+
+
+# ------------------------------------------------------------------ masked
+def _masked_case(dev, a, b, masked_m, rows_per_expert=None):
+    E, cap, K = a.shape
+    N = b.shape[1]
+    (qa, sa, qb, sb), (oqa, osa, oqb, osb) = _quantize_both(a, b, dev)
+    qa = qa.view(E, cap, K)
+    sa = sa.view(E, cap, K // TILE)
+    mm = torch.from_numpy(np.asarray(masked_m, dtype=np.int32)).to(dev)
+    out = torch.full((E, cap, N), -5.0, dtype=torch.bfloat16, device=dev)
+    fq.fp8_grouped_gemm_masked(qa, sa, qb.view(b.shape), sb, mm, expected_m=int(np.mean(masked_m)), out=out)
+    _finish(dev)
+    got = bf16_bits_of(out).reshape(E * cap, N)
+    oqa3 = oqa.reshape(E, cap, K)
+    osa3 = osa.reshape(E, cap, K // TILE)
+    valid = np.concatenate([np.arange(e * cap, e * cap + min(cap, max(0, int(masked_m[e])))) for e in range(E)]
+                           + [np.zeros(0, np.int64)])
+    invalid = np.setdiff1d(np.arange(E * cap), valid)
+    assert np.all(got[invalid] == 0xC0A0), "rows at or past masked_m must stay untouched"  # bf16 -5.0
+    if rows_per_expert is None:
+        rows = valid
+    else:
+        rng = np.random.default_rng(11)
+        rows = []
+        for e in range(E):
+            m = min(cap, max(0, int(masked_m[e])))
+            if m:
+                pick = {0, m - 1} | set(rng.choice(m, size=min(m, rows_per_expert), replace=False).tolist())
+                rows.extend(e * cap + r for r in sorted(pick))
+        rows = np.asarray(rows, dtype=np.int64)
+    if rows.size:
+        ref = oracle.grouped_masked(oqa3, osa3, oqb, osb, np.asarray(masked_m, np.int32), rows=rows)
+        assert_gemm_close(got[rows], ref, "masked")
+
+
+def test_masked_small_edge_counts(dev):
+    rng = np.random.default_rng(31)
+    E, cap, N, K = 6, 256, 384, 512
+    a = wl.bf16_bits(rng.standard_normal((E, cap, K)).astype(np.float32))
+    b = wl.bf16_bits((0.02 * rng.standard_normal((E, N, K))).astype(np.float32))
+    _masked_case(dev, a, b, [0, 1, 128, 129, 256, 255])
+
+
+def test_masked_all_empty(dev):
+    rng = np.random.default_rng(32)
+    a = wl.bf16_bits(rng.standard_normal((3, 128, 256)).astype(np.float32))
+    b = wl.bf16_bits(rng.standard_normal((3, 256, 256)).astype(np.float32))
+    _masked_case(dev, a, b, [0, 0, 0])
+
+
+def test_masked_out_of_range_counts_clamped(dev):
+    rng = np.random.default_rng(33)
+    a = wl.bf16_bits(rng.standard_normal((3, 128, 256)).astype(np.float32))
+    b = wl.bf16_bits(rng.standard_normal((3, 256, 256)).astype(np.float32))
+    _masked_case(dev, a, b, [-4, 500, 77])
+
+
+def test_masked_full_both_gemms(dev):
+    d = wl.moe_masked()
+    _masked_case(dev, d.a, d.b, d.masked_m, rows_per_expert=4)
+    _masked_case(dev, d.a2, d.b2, d.masked_m, rows_per_expert=4)

@@ -1,0 +1,145 @@
+"""GPU quantizers vs the oracle: E4M3 codes and scales must match bit for bit.
+
+Covers the hand-computed worked examples, edge tensors (zeros, -0, exact
+ties, E4M3 subnormals, bf16 subnormals, +-448 boundaries, huge values),
+ragged row counts, and every workload's full-size tensors.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import fp8_fine_grained_quant_b200 as fq
+import workloads as wl
+from conftest import golden_lines, hexfloat
+from parity import bytes_of, to_torch_bf16
+
+pytestmark = pytest.mark.gpu
+TILE = 128
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+def gpu_act(bits, dev):
+    x = to_torch_bf16(bits, dev)
+    q, s = fq.fp8_quant_act_1x128(x)
+    torch.cuda.synchronize(dev)
+    assert fq.get_device_error(device=dev) == fq.OK
+    return bytes_of(q), s.cpu().numpy()
+
+
+def gpu_w(bits, dev):
+    w = to_torch_bf16(bits, dev)
+    q, s = fq.fp8_quant_w_128x128(w)
+    torch.cuda.synchronize(dev)
+    return bytes_of(q).reshape(bits.shape), s.cpu().numpy()
+
+
+def assert_act_exact(bits, dev):
+    q, s = gpu_act(bits, dev)
+    oq, os_ = oracle.quant_act_1x128(bits)
+    assert np.array_equal(s.reshape(os_.shape).view(np.uint32), os_.view(np.uint32)), \
+        np.argwhere(s.reshape(os_.shape).view(np.uint32) != os_.view(np.uint32))[:5]
+    bad = np.argwhere(q.reshape(oq.shape) != oq)
+    assert bad.size == 0, (bad[:5], q.reshape(oq.shape)[tuple(bad[0])], oq[tuple(bad[0])])
+
+
+def assert_w_exact(bits, dev):
+    q, s = gpu_w(bits, dev)
+    oq, os_ = oracle.quant_w_128x128(bits)
+    assert np.array_equal(s.reshape(os_.shape).view(np.uint32), os_.view(np.uint32))
+    bad = np.argwhere(q.reshape(oq.shape) != oq)
+    assert bad.size == 0, bad[:5]
+
+
+def test_worked_examples(dev):
+    rows = {}
+    for tok in golden_lines("quant_worked_examples.txt"):
+        if tok[0] in ("act", "act2") and tok[1] != "K":
+            rows.setdefault(tok[0], []).append((int(tok[1]), hexfloat(tok[2]), int(tok[3], 16)))
+    for kind, K in (("act", 384), ("act2", 128)):
+        x = np.zeros((1, K), dtype=np.float32)
+        expect = np.zeros(K, dtype=np.uint8)
+        for k, v, code in rows[kind]:
+            x[0, k] = v
+            expect[k] = code
+        q, _ = gpu_act(wl.bf16_bits(x), dev)
+        assert np.array_equal(q.reshape(-1), expect), kind
+
+
+def _edge_tile_values():
+    """One 128-wide tile per row, each exercising a boundary of the encoder."""
+    v = []
+    ramp = np.arange(128, dtype=np.float32)
+    v.append(np.zeros(128, np.float32))                          # zero tile
+    v.append(-np.zeros(128, np.float32))                         # -0 tile
+    v.append(np.full(128, 448.0, np.float32) * np.where(ramp % 2, -1, 1))  # +-448, s = 1
+    t = (ramp - 64) * np.float32(3.5)                            # many exact ties after scaling
+    t[0] = 448.0
+    v.append(t)
+    v.append(np.float32(2.0) ** -(ramp % 30 + 1) * np.where(ramp % 3, 1, -1))  # wide dynamic range
+    v.append(np.full(128, np.float32(1e-38)) * (ramp + 1))       # near-subnormal scale
+    sub = np.full(128, np.float32(2.0 ** -133)) * (ramp % 7)     # bf16 subnormals
+    v.append(sub)
+    big = np.full(128, np.float32(3.0e38)) * np.where(ramp % 2, -1, 1)
+    big[5] = 1.0
+    v.append(big)
+    mix = np.float32(56.0) * np.float32(2.0) ** -(ramp % 20)     # s = 1/8, codes cover subnormals
+    v.append(mix)
+    return np.stack(v)
+
+
+def test_edge_tiles(dev):
+    bits = wl.bf16_bits(_edge_tile_values())
+    assert_act_exact(bits, dev)
+    # as weights: replicate the pattern into a 128 x (9*128) block row
+    w = np.repeat(bits.reshape(1, -1), 128, axis=0)
+    assert_w_exact(np.ascontiguousarray(w), dev)
+
+
+@pytest.mark.parametrize("M,K", [(1, 128), (3, 256), (129, 384), (300, 1024), (2048, 128), (7, 7168)])
+def test_act_random_shapes(dev, M, K):
+    rng = np.random.default_rng(M * 131 + K)
+    x = rng.standard_normal((M, K)).astype(np.float32) * np.exp(rng.uniform(-8, 8, size=(M, 1))).astype(np.float32)
+    x.reshape(-1)[rng.choice(M * K, size=max(1, M * K // 1000), replace=False)] *= 100
+    assert_act_exact(wl.bf16_bits(x), dev)
+
+
+@pytest.mark.parametrize("G,N,K", [(1, 128, 128), (1, 256, 640), (3, 384, 256), (2, 1024, 2048)])
+def test_w_random_shapes(dev, G, N, K):
+    rng = np.random.default_rng(G * 7 + N + K)
+    w = (0.02 * rng.standard_normal((G, N, K))).astype(np.float32)
+    w[:, ::97, ::89] *= 50
+    assert_w_exact(wl.bf16_bits(w), dev)
+
+
+def test_zero_sizes_are_noops(dev):
+    x = torch.zeros((0, 256), dtype=torch.bfloat16, device=dev)
+    q, s = fq.fp8_quant_act_1x128(x)
+    assert q.shape == (0, 256) and s.shape == (0, 2)
+
+
+@pytest.mark.parametrize("name", ["tiny_dense", "dense_fprop", "long_k"])
+def test_dense_workloads_full(dev, name):
+    d = wl.CONFIGS[name]()
+    assert_act_exact(d.a, dev)
+    assert_w_exact(d.b, dev)
+
+
+def test_moe_contiguous_full(dev):
+    d = wl.moe_contiguous()
+    assert_act_exact(d.a, dev)
+    assert_w_exact(d.b, dev)
+
+
+def test_moe_masked_full(dev):
+    d = wl.moe_masked()
+    assert_act_exact(d.a.reshape(-1, d.a.shape[-1]), dev)
+    assert_w_exact(d.b, dev)
+    assert_act_exact(d.a2.reshape(-1, d.a2.shape[-1]), dev)
+    assert_w_exact(d.b2, dev)
