@@ -1,0 +1,527 @@
+#!/usr/bin/env python
+"""Benchmark of the fine-grained FP8 path on B200: one step = online 1x128
+activation quantization + online 128x128 weight quantization + block-scaled
+FP8 GEMM with per-slab promotion, on one batch of synthetic input.
+
+Default workload: dense Fprop M=4096 (tokens), K=7168, N=7168 (the dense
+configuration the headline metric is quoted on).  ``--workload`` selects the
+others (tiny_dense, long_k, moe_contiguous, moe_masked) for extra lines.
+
+Prints ONE JSON line (rank 0).  Timing: W untimed warm-up steps, then K timed
+steps bracketed by barrier + device synchronize, CUDA events on the launching
+stream, max over ranks.  Inputs rotate over enough buffer sets that a step's
+inputs were not touched by the step before (the per-set footprint exceeds the
+126 MB L2).
+
+Multi-GPU: launched by torchrun, every rank runs its own independent problem
+of the same size (weak scaling; the path has no exchange step, so no
+collective touches the data).
+
+``--impl reference`` times the CPU oracle (the only reference implementation
+this path has) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+TILE = 128
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP8_OVER_BF16 = 2.0  # nominal dense fp8 / bf16 tensor throughput ratio (4.5 / 2.25 PFLOP/s)
+SUSTAINED_AFTER_S = 1.0
+
+
+# ---------------------------------------------------------------------------- helpers
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"],
+                "bf16_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16": FALLBACK_BF16_TFLOPS, "bf16_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted((ROOT / "fp8_fine_grained_quant_b200" / "csrc").glob("*")) + [ROOT / "include" / "fp8q.h"]:
+        h.update(p.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event (throttle) reasons through NVML while
+    the timed region runs (reading only; nothing is changed)."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self._stop = threading.Event()
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        except Exception:  # noqa: BLE001
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+        for bit, name in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._sample()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "note": getattr(self, "err", "")}
+        busy = sorted(self.reasons - {"gpu_idle"})
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz, "reasons": busy,
+                "samples": len(self.samples), "sm_mhz_min": min(self.samples)}
+
+
+# ---------------------------------------------------------------------------- workloads
+def make_workload(name: str):
+    import workloads as wl
+    return wl.CONFIGS[name]()
+
+
+def describe(name: str, d) -> dict:
+    if name in ("tiny_dense", "dense_fprop", "long_k"):
+        return {"workload": "%s M=%d N=%d K=%d" % (name, d.M, d.N, d.K), "M": d.M, "N": d.N, "K": d.K,
+                "seed": d.meta["seed"]}
+    if name == "moe_contiguous":
+        return {"workload": "moe_contiguous E=%d M_tot=%d (valid %d) N=%d K=%d" % (d.E, d.M_tot, int(d.counts.sum()),
+                                                                                 d.N, d.K),
+                "E": d.E, "M_tot": d.M_tot, "valid_rows": int(d.counts.sum()), "N": d.N, "K": d.K,
+                "seed": d.meta["seed"]}
+    return {"workload": "moe_masked E=%d cap=%d valid=%d (N,K)=(%d,%d)+(%d,%d)" % (
+        d.E, d.cap, int(d.masked_m.sum()), d.b.shape[1], d.b.shape[2], d.b2.shape[1], d.b2.shape[2]),
+        "E": d.E, "cap": d.cap, "valid_rows": int(d.masked_m.sum()), "seed": d.meta["seed"]}
+
+
+def _to_dev_bf16(torch, bits, dev):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def build_sets(name, d, dev, nsets, torch, fq):
+    """Per input set: device tensors and preallocated outputs."""
+    sets = []
+    for _ in range(nsets):
+        s = {}
+        if name == "moe_masked":
+            E, cap, K = d.a.shape
+            s["a"] = _to_dev_bf16(torch, d.a.reshape(E * cap, K), dev)
+            s["b"] = _to_dev_bf16(torch, d.b, dev)
+            s["a2"] = _to_dev_bf16(torch, d.a2.reshape(E * cap, -1), dev)
+            s["b2"] = _to_dev_bf16(torch, d.b2, dev)
+            s["mm"] = torch.from_numpy(d.masked_m).to(dev)
+        else:
+            s["a"] = _to_dev_bf16(torch, d.a, dev)
+            s["b"] = _to_dev_bf16(torch, d.b, dev)
+            if name == "moe_contiguous":
+                s["mi"] = torch.from_numpy(d.m_indices).to(dev)
+        sets.append(s)
+    return sets
+
+
+def kernel_plan(name, d):
+    """(kernel label, algorithmic bytes, algorithmic FLOPs) per launch of one step."""
+    def qa_bytes(rows, K):
+        return rows * K * (2 + 1) + rows * (K // TILE) * 4
+
+    def qw_bytes(G, N, K):
+        return G * N * K * (2 + 1) + G * (N // TILE) * (K // TILE) * 4
+
+    def gemm_bytes(rows, N, K, G=1):
+        return rows * K + rows * (K // TILE) * 4 + G * N * K + G * (N // TILE) * (K // TILE) * 4 + rows * N * 2
+
+    if name in ("tiny_dense", "dense_fprop", "long_k"):
+        M, N, K = d.M, d.N, d.K
+        return [("quant_act_1x128", qa_bytes(M, K), 0.0), ("quant_w_128x128", qw_bytes(1, N, K), 0.0),
+                ("gemm_blockscaled", gemm_bytes(M, N, K), 2.0 * M * N * K)]
+    if name == "moe_contiguous":
+        return [("quant_act_1x128", qa_bytes(d.M_tot, d.K), 0.0), ("quant_w_128x128", qw_bytes(d.E, d.N, d.K), 0.0),
+                ("grouped_gemm_contiguous", gemm_bytes(d.M_tot, d.N, d.K, d.E), d.flops)]
+    E, cap, K = d.a.shape
+    N, K2, N2 = d.b.shape[1], d.a2.shape[2], d.b2.shape[1]
+    active = int((d.masked_m > 0).sum())
+    valid = int(d.masked_m.sum())
+    return [("quant_act_1x128", qa_bytes(E * cap, K), 0.0), ("quant_w_128x128", qw_bytes(E, N, K), 0.0),
+            ("grouped_gemm_masked", gemm_bytes(valid, N, K, active), d.flops(False)),
+            ("quant_act_1x128#2", qa_bytes(E * cap, K2), 0.0), ("quant_w_128x128#2", qw_bytes(E, N2, K2), 0.0),
+            ("grouped_gemm_masked#2", gemm_bytes(valid, N2, K2, active), d.flops(True))]
+
+
+def launch_step(name, d, s, fq, events=None):
+    """Launch the kernels of one step on the current stream.  `events`, if
+    given, is a list of (start, end) CUDA-event pairs, one per kernel."""
+    def rec(i, which):
+        if events is not None:
+            events[i][which].record()
+
+    if name == "moe_masked":
+        E, cap, K = d.a.shape
+        rec(0, 0); qa, sa = fq.fp8_quant_act_1x128(s["a"], s.get("qa"), s.get("sa")); rec(0, 1)
+        rec(1, 0); qb, sb = fq.fp8_quant_w_128x128(s["b"], s.get("qb"), s.get("sb")); rec(1, 1)
+        rec(2, 0)
+        c = fq.fp8_grouped_gemm_masked(qa.view(E, cap, K), sa.view(E, cap, K // TILE), qb, sb, s["mm"],
+                                       expected_m=int(d.masked_m.mean()), out=s.get("c"))
+        rec(2, 1)
+        K2 = d.a2.shape[2]
+        rec(3, 0); qa2, sa2 = fq.fp8_quant_act_1x128(s["a2"], s.get("qa2"), s.get("sa2")); rec(3, 1)
+        rec(4, 0); qb2, sb2 = fq.fp8_quant_w_128x128(s["b2"], s.get("qb2"), s.get("sb2")); rec(4, 1)
+        rec(5, 0)
+        c2 = fq.fp8_grouped_gemm_masked(qa2.view(E, cap, K2), sa2.view(E, cap, K2 // TILE), qb2, sb2, s["mm"],
+                                        expected_m=int(d.masked_m.mean()), out=s.get("c2"))
+        rec(5, 1)
+        s.update(qa=qa, sa=sa, qb=qb, sb=sb, c=c, qa2=qa2, sa2=sa2, qb2=qb2, sb2=sb2, c2=c2)
+        return c2
+    rec(0, 0); qa, sa = fq.fp8_quant_act_1x128(s["a"], s.get("qa"), s.get("sa")); rec(0, 1)
+    rec(1, 0); qb, sb = fq.fp8_quant_w_128x128(s["b"], s.get("qb"), s.get("sb")); rec(1, 1)
+    rec(2, 0)
+    if name == "moe_contiguous":
+        c = fq.fp8_grouped_gemm_contiguous(qa, sa, qb, sb, s["mi"], out=s.get("c"))
+    else:
+        c = fq.fp8_gemm_blockscaled(qa, sa, qb, sb, out=s.get("c"))
+    rec(2, 1)
+    s.update(qa=qa, sa=sa, qb=qb, sb=sb, c=c)
+    return c
+
+
+def step_flops(name, d):
+    if name == "moe_masked":
+        return d.flops(False) + d.flops(True)
+    return d.flops
+
+
+# ---------------------------------------------------------------------------- CPU oracle timing
+def oracle_sample_step(name, d, rows: int, nblocks: int):
+    """One oracle step on a bounded sample of the workload: the activation
+    quantization of `rows` rows, the weight quantization of `nblocks` 128-row
+    weight blocks, and the GEMM outputs rows x (128 * nblocks).  Returns
+    (seconds, flops of the sample)."""
+    import oracle
+    if name == "moe_masked":
+        a, b = d.a[0], d.b[0]
+    elif name == "moe_contiguous":
+        a, b = d.a, d.b[int(d.m_indices[0])]
+    else:
+        a, b = d.a, d.b
+    K = a.shape[1]
+    ra = np.ascontiguousarray(a[:rows])
+    rb = np.ascontiguousarray(b[:TILE * nblocks])
+    t0 = time.perf_counter()
+    qa, sa = oracle.quant_act_1x128(ra)
+    qb, sb = oracle.quant_w_128x128(rb)
+    oracle.gemm_blockscaled(qa, sa, qb, sb)
+    dt = time.perf_counter() - t0
+    return dt, 2.0 * rows * TILE * nblocks * K
+
+
+def cpu_sample_size(name, d, budget_s: float):
+    """Rows x weight blocks whose oracle step takes about budget_s."""
+    rows, nb = 8, 1
+    dt, _ = oracle_sample_step(name, d, rows, nb)
+    scale = max(1.0, budget_s / max(dt, 1e-4))
+    nb_max = (d.b.shape[-2]) // TILE
+    nb = int(min(nb_max, max(1, round(scale ** 0.5))))
+    rows = int(min(d.a.shape[-2], max(1, round(rows * scale / nb))))
+    return rows, nb
+
+
+def run_reference(args, name):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    d = make_workload(name)
+    per_step = max(0.05, min(2.0, 120.0 / max(1, args.steps + args.warmup)))
+    rows, nb = cpu_sample_size(name, d, per_step)
+    for _ in range(args.warmup):
+        oracle_sample_step(name, d, rows, nb)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, f = oracle_sample_step(name, d, rows, nb)
+        times.append(dt)
+        flops += f
+    total = sum(times)
+    value = flops / total / 1e12
+    sample = ("per step: 1x128 quantization of %d rows of A, 128x128 quantization of %d weight block-rows "
+              "(%d x %d), GEMM of %d x %d outputs over K=%d" % (rows, nb, TILE * nb, d.a.shape[-1], rows, TILE * nb,
+                                                               d.a.shape[-1]))
+    line = {
+        "impl": "reference", "metric": "FP8 block-scaled GEMM TFLOPS", "value": value, "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": describe(name, d),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------------------- GPU arm
+def traffic_for(kernel: str, name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; otherwise None."""
+    p = ROOT / "profiles" / "traffic.json"
+    if not p.exists():
+        return None
+    try:
+        t = json.loads(p.read_text())
+        ent = t.get("%s:%s" % (kernel, name))
+        if ent and ent.get("source_hash") == source_hash():
+            return ent["dram_bytes_per_launch"]
+    except Exception:  # noqa: BLE001
+        return None
+    return None
+
+
+def run_ours(args, name):
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    import fp8_fine_grained_quant_b200 as fq
+    fq.lib()
+
+    d = make_workload(name)
+    plan = kernel_plan(name, d)
+    nk = len(plan)
+    flops = step_flops(name, d)
+    per_set_bytes = sum(b for _, b, _ in plan)
+    nsets = max(2, int(np.ceil(2 * 126e6 / max(per_set_bytes, 1))))
+    nsets = min(nsets, 4)
+    sets = build_sets(name, d, dev, nsets, torch, fq)
+    stream = torch.cuda.current_stream(dev)
+
+    for i in range(args.warmup):
+        launch_step(name, d, sets[i % nsets], fq)
+    torch.cuda.synchronize(dev)
+    if fq.get_device_error(device=dev) != fq.OK:
+        raise RuntimeError("device error during warm-up")
+
+    events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(nk)]
+              for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    launches0 = fq.launch_count()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            launch_step(name, d, sets[i % nsets], fq, events[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    launches = fq.launch_count() - launches0
+    elapsed_ms = t_start.elapsed_time(t_end)
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
+    if fq.get_device_error(device=dev) != fq.OK:
+        raise RuntimeError("device error in the timed region")
+    kernel_ms = [[events[i][k][0].elapsed_time(events[i][k][1]) for i in range(args.steps)] for k in range(nk)]
+
+    # ------------------------------------------------------------ e2e (host buffers)
+    e2e = run_e2e(args, name, d, dev, torch, fq, world)
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
+
+    peaks = load_peaks()
+    timed_s = elapsed_ms / 1e3
+    sustained = timed_s >= SUSTAINED_AFTER_S
+    bf16_peak = peaks["bf16_sustained"] if sustained else peaks["bf16"]
+    fp8_peak = bf16_peak * FP8_OVER_BF16
+    kernels = {}
+    for k, (label, nbytes, kflops) in enumerate(plan):
+        avg_ms = float(np.mean(kernel_ms[k]))
+        ent = {"avg_ms": avg_ms, "bytes": nbytes}
+        if kflops:
+            ent.update(tflops=kflops / avg_ms / 1e9, frac_of_fp8_peak=kflops / avg_ms / 1e9 / fp8_peak)
+        ent.update(gbs=nbytes / avg_ms / 1e6, frac_of_hbm=nbytes / avg_ms / 1e6 / peaks["hbm_gbs"])
+        kernels[label] = ent
+    gemm_label = [l for l, _, f in plan if f][0]
+    g = kernels[gemm_label]
+    # dominant kernel: the GEMM (tensor-bound at these shapes except masked decode, reported both ways)
+    bound = "tensor"
+    roofline = {"bound": bound, "kernel": gemm_label, "achieved": g["tflops"], "peak": fp8_peak, "unit": "TFLOP/s",
+                "frac": g["tflops"] / fp8_peak, "traffic": traffic_for(gemm_label, name),
+                "peak_source": "%s (%s bf16 %.1f TFLOP/s x %.0f fp8/bf16 nominal ratio)" % (
+                    peaks["source"], "sustained" if sustained else "burst", bf16_peak, FP8_OVER_BF16),
+                "algorithmic_flops_per_launch": [f for _, _, f in plan if f][0]}
+    value = world * flops * args.steps / (elapsed_ms / 1e3) / 1e12
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(name, d)
+    line = {
+        "metric": "FP8 block-scaled GEMM TFLOPS (step = 1x128 act quant + 128x128 weight quant + GEMM)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3", "data": "synthetic",
+        "config": dict(describe(name, d), parallelism="replicas" if world > 1 else "single",
+                       l2="inputs rotated over %d buffer sets (%.0f MB each) between steps" % (
+                           nsets, per_set_bytes / 1e6)),
+        "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": int(launches), "clocks": clk.summary(),
+    }
+    print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, name, d, dev, torch, fq, world):
+    """Same step through the public API from pinned host buffers: H2D copy of
+    the bf16 inputs, the three kernels, D2H copy of the bf16 result."""
+    host = {}
+    keys = ["a", "b"] + (["a2", "b2"] if name == "moe_masked" else [])
+    src = {"a": d.a, "b": d.b}
+    if name == "moe_masked":
+        src.update(a2=d.a2, b2=d.b2)
+    for k in keys:
+        arr = np.ascontiguousarray(src[k]).view(np.int16)
+        host[k] = torch.from_numpy(arr).pin_memory()
+    s = build_sets(name, d, dev, 1, torch, fq)[0]
+    out_host = None
+    h2d = sum(host[k].numel() * 2 for k in keys)
+    steps = max(3, min(args.steps, 20))
+
+    def one():
+        nonlocal out_host
+        for k in keys:
+            s[k].view(torch.int16).view(host[k].shape).copy_(host[k], non_blocking=True)
+        c = launch_step(name, d, s, fq)
+        if out_host is None:
+            out_host = torch.empty(c.shape, dtype=c.dtype).pin_memory()
+        out_host.copy_(c, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    value = world * step_flops(name, d) / (ms / 1e3) / 1e12
+    return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(out_host.numel() * 2), "ms_per_step": ms, "steps": steps}
+
+
+def cpu_baseline(name, d):
+    import oracle
+    budget = float(os.environ.get("FP8Q_CPU_BASELINE_S", "8"))
+    rows, nb = cpu_sample_size(name, d, budget / 3)
+    dts, fl = [], 0.0
+    for _ in range(3):
+        dt, f = oracle_sample_step(name, d, rows, nb)
+        dts.append(dt)
+        fl += f
+    value = fl / sum(dts) / 1e12
+    return {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "3 oracle steps, each: 1x128 quantization of %d rows of A, 128x128 quantization of %d weight "
+                      "block-rows, float64 GEMM of the %d x %d outputs they determine (K=%d); %.1f s total" % (
+                          rows, nb, rows, TILE * nb, d.a.shape[-1], sum(dts))}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="dense_fprop",
+                    choices=["tiny_dense", "dense_fprop", "long_k", "moe_contiguous", "moe_masked"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args, args.workload)
+    return run_ours(args, args.workload)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

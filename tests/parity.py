@@ -1,12 +1,23 @@
 """Comparison helpers shared by the GPU parity tests, smoke() and bench.py.
 
-GEMM tolerance (the target's own wording: max relative error 2e-3 and max
-absolute error <= 1e-2 * rms(C) against the oracle's dequantized-input
-product).  Read as two checks over the compared elements:
-  (1) max |C - C_ref| <= 1e-2 * rms(C_ref)
-  (2) max |C - C_ref| / |C_ref| <= 2e-3 over elements with |C_ref| >= 0.1 * rms(C_ref)
-(near-zero elements make a pure relative error meaningless).  bf16 rounding
-of the output alone spends up to 2^-9 / (1 + 2^-9) = 1.949e-3 of (2).
+GEMM tolerance.  The target bounds the GEMM's error against the oracle's
+dequantized-input product by a max relative error of 2e-3 and a max absolute
+error of 1e-2 * rms(C).  The GEMM's result is delivered in bf16, whose unit
+roundoff is 2^-8: rounding alone can move an element by up to
+2^-8 / (1 + 2^-8) = 3.89e-3 relative, so the bound, applied literally to the
+bf16 output, would reject even an exact computation.  The reading used here
+applies the bound to the product *before* its one rounding to bf16:
+
+  every output element C must be the round-to-nearest-even bf16 of some value
+  v with |v - C_ref| <= d, where
+      d = min(2e-3 * |C_ref|, 1e-2 * rms(C_ref))   if |C_ref| >= 0.1 * rms(C_ref)
+      d = 1e-2 * rms(C_ref)                          otherwise
+  (relative error is meaningless for near-zero elements, which cancellation
+  produces; they are held to the absolute bound).
+
+Equivalently the implied pre-rounding error e = distance from C_ref to the set
+of reals that round to C must satisfy e <= d.  The statistics also report the
+raw output error and how many elements are not the correctly rounded C_ref.
 """
 from __future__ import annotations
 
@@ -31,35 +42,61 @@ def bytes_of(t: torch.Tensor) -> np.ndarray:
 
 
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
-    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def bf16_rne_f64(x: np.ndarray) -> np.ndarray:
+    """float64 -> nearest bf16 value (ties to even), one rounding, as float64.
+    (Normal range only; the magnitudes compared here are far from bf16's
+    subnormals.)"""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)  # x = m * 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.rint(m * 256.0), e - 8)  # 8 significant bits, rint = half-to-even
+
+
+def _neighbours(bits: np.ndarray):
+    """bf16 values just above and just below each pattern (as float64)."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.int32)
+    mag = b & 0x7FFF
+    neg = (b & 0x8000) != 0
+    up_bits = np.where(neg, np.where(mag > 0, 0x8000 | (mag - 1), 0x0001), mag + 1)
+    dn_bits = np.where(neg, 0x8000 | (mag + 1), np.where(mag > 0, mag - 1, 0x8001))
+    return bf16_to_f64(up_bits.astype(np.uint16)), bf16_to_f64(dn_bits.astype(np.uint16))
 
 
 def gemm_errors(c_bits: np.ndarray, ref: np.ndarray) -> dict:
-    """Error statistics of a bf16 result (bit patterns) against float64 ref."""
     c = bf16_to_f64(c_bits)
     ref = np.asarray(ref, dtype=np.float64)
     assert c.shape == ref.shape, (c.shape, ref.shape)
-    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
-    err = np.abs(c - ref)
+    n = ref.size
+    rms = float(np.sqrt(np.mean(ref * ref))) if n else 0.0
     big = np.abs(ref) >= REL_FLOOR_RMS * rms
-    rel = err[big] / np.abs(ref[big]) if big.any() else np.zeros(1)
-    ref_bf16 = torch.from_numpy(ref).to(torch.bfloat16).to(torch.float64).numpy()
-    ulp = np.abs(ref_bf16) * 2.0 ** -7
-    beyond_1ulp = int(np.count_nonzero(np.abs(c - ref_bf16) > np.maximum(ulp, 1e-30) * 1.0001))
+    d = np.full(ref.shape, ABS_TOL_RMS * rms)
+    d[big] = np.minimum(d[big], REL_TOL * np.abs(ref[big]))
+    up, dn = _neighbours(c_bits)
+    half_up = (up - c) / 2.0
+    half_dn = (c - dn) / 2.0
+    implied = np.where(ref > c, np.maximum(0.0, ref - c - half_up), np.maximum(0.0, c - ref - half_dn))
+    err = np.abs(c - ref)
+    finite = np.isfinite(c)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        used = np.where(d > 0, implied / d, np.where(implied > 0, np.inf, 0.0))
     return {
         "rms": rms,
-        "max_abs": float(err.max()) if err.size else 0.0,
-        "max_abs_over_rms": float(err.max() / rms) if err.size and rms > 0 else 0.0,
-        "max_rel": float(rel.max()),
-        "n": int(ref.size),
+        "n": int(n),
         "n_rel": int(big.sum()),
-        "beyond_1ulp": beyond_1ulp,
-        "nonfinite": int(np.count_nonzero(~np.isfinite(c))),
+        "tol_used": float(used.max()) if n else 0.0,             # <= 1 passes
+        "implied_max_rel": float((implied[big] / np.abs(ref[big])).max()) if big.any() else 0.0,
+        "implied_max_abs_over_rms": float(implied.max() / rms) if n and rms > 0 else 0.0,
+        "out_max_rel": float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0,
+        "out_max_abs_over_rms": float(err.max() / rms) if n and rms > 0 else 0.0,
+        "not_correctly_rounded": int(np.count_nonzero(c != bf16_rne_f64(ref))),
+        "nonfinite": int(np.count_nonzero(~finite)),
     }
 
 
 def gemm_ok(stats: dict) -> bool:
-    return (stats["nonfinite"] == 0 and stats["max_abs_over_rms"] <= ABS_TOL_RMS and stats["max_rel"] <= REL_TOL)
+    return stats["nonfinite"] == 0 and stats["tol_used"] <= 1.0
 
 
 def assert_gemm_close(c_bits: np.ndarray, ref: np.ndarray, what: str = "gemm") -> dict:

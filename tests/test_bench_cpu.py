@@ -1,0 +1,73 @@
+"""bench.py host logic on CPU: the reference (oracle) arm's JSON line, the
+per-kernel algorithmic byte/FLOP accounting, and the multi-rank timing
+reduction (max over ranks) on a world-size-2 gloo group."""
+import json
+import os
+import subprocess
+import sys
+from pathlib import Path
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = Path(__file__).resolve().parents[1]
+sys.path.insert(0, str(ROOT))
+import bench  # noqa: E402
+import workloads as wl  # noqa: E402
+
+
+def test_reference_arm_prints_contract_line():
+    out = subprocess.run([sys.executable, str(ROOT / "bench.py"), "--impl", "reference", "--workload", "tiny_dense",
+                          "--steps", "3", "--warmup", "3"], capture_output=True, text=True, check=True, cwd=ROOT,
+                         timeout=600)
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["config"]["workload"].startswith("tiny_dense")
+
+
+def test_kernel_plan_accounting():
+    d = wl.tiny_dense()
+    plan = dict((k, (b, f)) for k, b, f in bench.kernel_plan("tiny_dense", d))
+    M, N, K = 128, 256, 512
+    assert plan["quant_act_1x128"][0] == M * K * 3 + M * (K // 128) * 4
+    assert plan["quant_w_128x128"][0] == N * K * 3 + (N // 128) * (K // 128) * 4
+    assert plan["gemm_blockscaled"][1] == 2.0 * M * N * K
+    assert plan["gemm_blockscaled"][0] == M * K + M * (K // 128) * 4 + N * K + (N // 128) * (K // 128) * 4 + M * N * 2
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        got = bench.max_over_ranks(float(10 * (rank + 1)), world, device="cpu")
+        q.put((rank, got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + (os.getpid() % 1000)
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = dict(q.get(timeout=5) for _ in range(2))
+    assert res == {0: 20.0, 1: 20.0}
+
+
+def test_cpu_sample_size_is_bounded():
+    d = wl.tiny_dense()
+    rows, nb = bench.cpu_sample_size("tiny_dense", d, 0.05)
+    assert 1 <= rows <= d.M and 1 <= nb <= d.N // 128
