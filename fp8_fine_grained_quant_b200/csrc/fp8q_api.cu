@@ -45,7 +45,9 @@ cudaError_t opt_in_smem() {
                               GemmSmem<BN, STAGES>::kDynamicBytes);
 }
 
-constexpr int kStages256 = 4;
+// Output tile 128 x kTileN: 64 FP32 accumulators per epilogue thread, four
+// TMEM slab buffers, six 32 KB pipeline stages.
+constexpr int kTileN = 128;
 constexpr int kStages128 = 6;
 
 int device_info(DeviceInfo** out) {
@@ -66,9 +68,6 @@ int device_info(DeviceInfo** out) {
         if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_device_status) != cudaSuccess)
           return FP8Q_ERR_CUDA;
         cudaError_t e = cudaSuccess;
-        if (e == cudaSuccess) e = opt_in_smem<256, kStages256, Sched::kDense>();
-        if (e == cudaSuccess) e = opt_in_smem<256, kStages256, Sched::kContiguous>();
-        if (e == cudaSuccess) e = opt_in_smem<256, kStages256, Sched::kMasked>();
         if (e == cudaSuccess) e = opt_in_smem<128, kStages128, Sched::kDense>();
         if (e == cudaSuccess) e = opt_in_smem<128, kStages128, Sched::kContiguous>();
         if (e == cudaSuccess) e = opt_in_smem<128, kStages128, Sched::kMasked>();
@@ -133,24 +132,6 @@ struct GemmCall {
   int promote;
 };
 
-// Tile width: the candidate whose last wave is fullest, preferring the wide
-// tile (half the shared-memory traffic per FLOP) unless it wastes > 15% more.
-int choose_bn(const GemmCall& g, Sched s, int num_sms) {
-  if (g.N <= 128) return 128;
-  auto eff = [&](int bn) {
-    const double n_tiles = static_cast<double>((g.N + bn - 1) / bn);
-    double m_tiles = static_cast<double>(g.m_tiles) * (s == Sched::kMasked ? g.E : 1);
-    if (s == Sched::kMasked && g.expected_m > 0)
-      m_tiles = static_cast<double>(g.E) * ((g.expected_m + kBlockM - 1) / kBlockM);
-    const double tiles = m_tiles * n_tiles;
-    const double waves = std::ceil(tiles / num_sms);
-    const double work = tiles * bn;                     // useful work in units of 128 x 1 columns
-    const double cost = waves * bn * (bn == 128 ? 1.15 : 1.0);  // narrow tiles run below peak
-    return work / cost;
-  };
-  return eff(128) > eff(256) * 1.0 ? 128 : 256;
-}
-
 template <int BN, int STAGES, Sched S>
 int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
   CUtensorMap ma, mb;
@@ -193,9 +174,7 @@ int run_gemm(const GemmCall& g, cudaStream_t stream) {
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);
   if (rc) return rc;
-  const int bn = choose_bn(g, S, dev->num_sms);
-  if (bn == 128) return launch_gemm<128, kStages128, S>(g, *dev, stream);
-  return launch_gemm<256, kStages256, S>(g, *dev, stream);
+  return launch_gemm<kTileN, kStages128, S>(g, *dev, stream);
 }
 
 int check_operands(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, const void* c) {

@@ -72,12 +72,13 @@ struct GemmSmem {
   static constexpr uint32_t kABytes = kBlockM * kSlabK;  // 16 KB
   static constexpr uint32_t kBBytes = BN * kSlabK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kTmemStride = BN <= 128 ? 128 : 256;  // columns between the two slab buffers
-  static constexpr uint32_t kTmemCols = 2 * kTmemStride;          // power of two >= 32
+  static constexpr uint32_t kTmemStride = BN <= 128 ? 128 : 256;  // columns per TMEM slab buffer
+  static constexpr uint32_t kTmemCols = 512;                      // all of TMEM (one CTA per SM)
+  static constexpr int kAccBufs = kTmemCols / kTmemStride;        // slab buffers in flight
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = STAGES * kABytes;
-  static constexpr uint32_t kOffBars = STAGES * kStageBytes;  // full[S], empty[S], tfull[2], tempty[2], drain
-  static constexpr uint32_t kNumBars = 2 * STAGES + 5;
+  static constexpr uint32_t kOffBars = STAGES * kStageBytes;  // full[S], empty[S], tfull[B], tempty[B], drain
+  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * kAccBufs + 1;
   static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;     // tmem slot, abort flag, total tiles
   static constexpr uint32_t kOffPrefix = (kOffMisc + 16 + 15) / 16 * 16;
   static constexpr uint32_t kBytes = kOffPrefix + 4 * (kMaxMaskedExperts + 1);
@@ -151,20 +152,20 @@ __device__ __forceinline__ bool get_tile(const GemmArgs& a, const int32_t* prefi
 
 // ----------------------------------------------------------------- roles
 // Shared-memory barrier addresses (mbarrier objects, 8 bytes each).
-template <int STAGES>
+template <int STAGES, int ACC>
 struct Bars {
   uint32_t base;
   __device__ uint32_t full(int s) const { return base + 8u * s; }
   __device__ uint32_t empty(int s) const { return base + 8u * (STAGES + s); }
   __device__ uint32_t tfull(int b) const { return base + 8u * (2 * STAGES + b); }
-  __device__ uint32_t tempty(int b) const { return base + 8u * (2 * STAGES + 2 + b); }
-  __device__ uint32_t drain() const { return base + 8u * (2 * STAGES + 4); }
+  __device__ uint32_t tempty(int b) const { return base + 8u * (2 * STAGES + ACC + b); }
+  __device__ uint32_t drain() const { return base + 8u * (2 * STAGES + 2 * ACC); }
 };
 
 // TMA producer (one thread): one pipeline stage per 128-deep K slab.
 template <int BN, int STAGES, Sched S>
 __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensorMap* tma_b, const GemmArgs& args,
-                                     const int32_t* prefix, uint32_t s_base, Bars<STAGES> bars, WaitCtl wc,
+                                     const int32_t* prefix, uint32_t s_base, Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
                                      int32_t total) {
   using L = GemmSmem<BN, STAGES>;
   int stage = 0;
@@ -197,10 +198,12 @@ __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensor
   }
 }
 
-// MMA issuer (one thread): four K = 32 MMAs per slab into a TMEM slab buffer.
+// MMA issuer (one thread): four K = 32 MMAs per slab into one of kAccBufs
+// TMEM slab buffers, used round-robin.
 template <int BN, int STAGES, Sched S>
 __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* prefix, uint32_t s_base,
-                                       Bars<STAGES> bars, WaitCtl wc, int32_t total, uint32_t tmem_base) {
+                                          Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
+                                          int32_t total, uint32_t tmem_base) {
   using L = GemmSmem<BN, STAGES>;
   constexpr uint32_t kIdesc = idesc_e4m3_f32(kBlockM, BN);
   int stage = 0, buf = 0;
@@ -230,8 +233,10 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
       }
       if (args.promote || kb == args.nkb - 1) {
         mma_commit(bars.tfull(buf));
-        buf ^= 1;
-        if (buf == 0) tphase ^= 1u;
+        if (++buf == L::kAccBufs) {
+          buf = 0;
+          tphase ^= 1u;
+        }
       }
     }
   }
@@ -244,16 +249,20 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
 
 // Epilogue warp: promotion of every slab partial into FP32 registers, then the
 // bf16 store of the finished tile.  Warp w owns TMEM lanes 32*(w%4)..+31 (tile
-// rows) and columns [half*BN/2, (half+1)*BN/2).  For BN in {128, 256} each
-// half lies inside one 128-column weight block, so one sb value per slab.
+// rows) and kCols = BN/2 columns.  Each half lies inside one 128-column weight
+// block (BN in {128, 256}), so one sb value per slab.  Per slab the warp loads
+// its columns in groups of up to 64 (two 32-column TMEM loads, one wait), hands
+// the buffer back to the MMA warp as soon as the last group is in registers,
+// and then applies acc += (sa * sb) * partial with packed FP32 FMAs.
 template <int BN, int STAGES, Sched S>
-__device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* prefix, Bars<STAGES> bars, WaitCtl wc,
+__device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* prefix,
+                                         Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
                                          int32_t total, uint32_t tmem_base, int warp, int lane) {
   using L = GemmSmem<BN, STAGES>;
-  constexpr int kHalf = BN / 2;
-  constexpr int kChunk = 32;
-  constexpr int kChunks = kHalf / kChunk;
-  static_assert(kHalf <= 128 && 128 % kHalf == 0, "each half must sit inside one 128-column scale block");
+  constexpr int kCols = BN / 2;
+  constexpr int kGroup = kCols < 64 ? kCols : 64;
+  constexpr int kGroups = kCols / kGroup;
+  static_assert(kCols <= 128 && 128 % kCols == 0 && kGroup % 32 == 0, "each half must sit in one scale block");
   const int quad = warp & 3;
   const int half = (warp - 4) >> 2;
   const int r = quad * 32 + lane;
@@ -266,13 +275,13 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
     Tile tile;
     if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
     const bool row_ok = r < tile.rows;
-    const int col0 = tile.n0 + half * kHalf;
+    const int col0 = tile.n0 + half * kCols;
     const bool col_ok = col0 < args.N;
     const float* sa_row = args.sa + static_cast<int64_t>(tile.a_row + (row_ok ? r : 0)) * nkb;
     const float* sb_row = args.sb + (static_cast<int64_t>(tile.e) * nnb + (col_ok ? col0 / 128 : 0)) * nkb;
-    float acc[kHalf];
+    uint64_t acc[kCols / 2];  // packed pairs of FP32 running sums
 #pragma unroll
-    for (int i = 0; i < kHalf; ++i) acc[i] = 0.0f;
+    for (int i = 0; i < kCols / 2; ++i) acc[i] = 0ull;
 
     const int n_reads = args.promote ? nkb : 1;
     // the next slab's scales are fetched one slab ahead
@@ -280,7 +289,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
     float sb_next = col_ok ? __ldg(sb_row) : 0.0f;
     bool ok = true;
     for (int it = 0; it < n_reads; ++it) {
-      const float scale = sa_next * sb_next;
+      const uint64_t scale2 = pack_f32x2(sa_next * sb_next);
       if (it + 1 < n_reads) {
         sa_next = row_ok ? __ldg(sa_row + it + 1) : 0.0f;
         sb_next = col_ok ? __ldg(sb_row + it + 1) : 0.0f;
@@ -288,36 +297,41 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
       // warp-uniform outcome: the tcgen05.ld below must be executed by all 32 lanes
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(bars.tfull(buf), tphase, wc, 4))) { ok = false; break; }
       tc_fence_after();
-      const uint32_t t_buf = t_lane + buf * L::kTmemStride + half * kHalf;
+      const uint32_t t_buf = t_lane + buf * L::kTmemStride + half * kCols;
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) {
-        uint32_t v[kChunk];
-        tmem_ld_32x32b_x32(t_buf + c * kChunk, v);
-        tmem_ld_wait(v);
+      for (int g = 0; g < kGroups; ++g) {
+        uint32_t v0[32], v1[32];
+        tmem_ld_32x32b_x32(t_buf + g * kGroup, v0);
+        if constexpr (kGroup == 64) tmem_ld_32x32b_x32(t_buf + g * kGroup + 32, v1);
+        tmem_ld_wait(v0);
+        if constexpr (kGroup == 64) reg_fence(v1);
+        if (g == kGroups - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bars.tempty(buf));
+        }
 #pragma unroll
-        for (int j = 0; j < kChunk; j += 2)
-          ffma2(acc[c * kChunk + j], acc[c * kChunk + j + 1], __uint_as_float(v[j]), __uint_as_float(v[j + 1]), scale);
+        for (int j = 0; j < 16; ++j) ffma2_packed(acc[g * (kGroup / 2) + j], v0[2 * j], v0[2 * j + 1], scale2);
+        if constexpr (kGroup == 64) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) ffma2_packed(acc[g * (kGroup / 2) + 16 + j], v1[2 * j], v1[2 * j + 1], scale2);
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bars.tempty(buf));
-      buf ^= 1;
-      if (buf == 0) tphase ^= 1u;
+      if (++buf == L::kAccBufs) {
+        buf = 0;
+        tphase ^= 1u;
+      }
     }
     if (!ok) break;
     if (row_ok && col_ok) {
       __nv_bfloat16* crow = args.c + static_cast<int64_t>(tile.a_row + r) * args.N + col0;
 #pragma unroll
-      for (int j = 0; j < kHalf; j += 8) {
-        __nv_bfloat162 p0 = __floats2bfloat162_rn(acc[j], acc[j + 1]);
-        __nv_bfloat162 p1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
-        __nv_bfloat162 p2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
-        __nv_bfloat162 p3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
+      for (int j = 0; j < kCols; j += 8) {
         uint4 o;
-        o.x = *reinterpret_cast<uint32_t*>(&p0);
-        o.y = *reinterpret_cast<uint32_t*>(&p1);
-        o.z = *reinterpret_cast<uint32_t*>(&p2);
-        o.w = *reinterpret_cast<uint32_t*>(&p3);
+        o.x = bf16x2_from_packed(acc[j / 2]);
+        o.y = bf16x2_from_packed(acc[j / 2 + 1]);
+        o.z = bf16x2_from_packed(acc[j / 2 + 2]);
+        o.w = bf16x2_from_packed(acc[j / 2 + 3]);
         *reinterpret_cast<uint4*>(crow + j) = o;
       }
     }
@@ -335,7 +349,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
-  const Bars<STAGES> bars{s_base + L::kOffBars};
+  const Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars{s_base + L::kOffBars};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
   int32_t* total_slot = reinterpret_cast<int32_t*>(smem + L::kOffMisc + 8);
@@ -349,7 +363,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(bars.full(s), 1);
       mbar_init(bars.empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < L::kAccBufs; ++b) {
       mbar_init(bars.tfull(b), 1);
       mbar_init(bars.tempty(b), 8);  // one arrival per epilogue warp
     }

@@ -182,14 +182,39 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
 }
 
 // ---------------------------------------------------------------- arithmetic
-// Two FP32 fused multiply-adds in one instruction: {d0,d1} = {a0,a1}*{b,b}+{c0,c1}.
-__device__ __forceinline__ void ffma2(float& c0, float& c1, float a0, float a1, float b) {
-  uint64_t a, bb, c;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(bb) : "f"(b));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(c) : "f"(c0), "f"(c1));
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(c) : "l"(a), "l"(bb));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(c0), "=f"(c1) : "l"(c));
+// {x, x} as a packed pair of FP32 values.
+__device__ __forceinline__ uint64_t pack_f32x2(float x) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(x));
+  return r;
+}
+
+// acc += {v0, v1} * scale2, two FP32 fused multiply-adds in one instruction.
+__device__ __forceinline__ void ffma2_packed(uint64_t& acc, uint32_t v0, uint32_t v1, uint64_t scale2) {
+  asm("{\n\t.reg .b64 t;\n\tmov.b64 t, {%1, %2};\n\tfma.rn.f32x2 %0, t, %3, %0;\n\t}"
+      : "+l"(acc)
+      : "r"(v0), "r"(v1), "l"(scale2));
+}
+
+// Packed FP32 pair -> packed bf16 pair (round to nearest even); low half first.
+__device__ __forceinline__ uint32_t bf16x2_from_packed(uint64_t p) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Orders later uses of r after the preceding tcgen05.wait::ld (no instruction).
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
 }
 
 // Two FP32 values -> two E4M3 codes (round to nearest even, saturating to

@@ -43,13 +43,52 @@ __device__ __forceinline__ float group_scale(float amax) {
   return s == 0.0f ? 1.0f : s;
 }
 
-// 8 values / s -> 8 E4M3 codes packed little-endian in two words.
-__device__ __forceinline__ uint2 quantize8(const float (&f)[8], float s) {
+// Division-free quantization with an exactness filter.
+//
+// The code must be E4M3_RNE(fl32(x / s)).  With r = RN(1/s) (s a normal float)
+// and y = RN(x * r), |y - x/s| <= (2^-23 + 2^-48)|x/s| and fl32(x/s) is within
+// 2^-24 |x/s| of x/s, so y and fl32(x/s) are at most ~3 ulps of y apart.  The
+// E4M3 code changes only across a rounding midpoint, so whenever y is more
+// than 16 ulps from every midpoint both round to the same code.  Otherwise
+// (about 3e-5 of values) the exact IEEE quotient is used.
+//
+// Midpoints: for |y| >= 2^-6 the E4M3 grid keeps 3 fraction bits, so a midpoint
+// is a binary32 whose 20 dropped bits equal 0x80000; below 2^-6 the grid is
+// n * 2^-9 and the midpoints are (n + 1/2) * 2^-9.  Values that underflow in
+// the product are far below 2^-10 and give +-0 either way (the sign of x is
+// kept by the multiplication).
+__device__ __forceinline__ bool e4m3_code_is_stable(float y) {
+  const uint32_t b = __float_as_uint(y) & 0x7FFFFFFFu;
+  if (b >= 0x3C800000u) {  // |y| >= 2^-6
+    const int32_t rem = static_cast<int32_t>(b & 0xFFFFFu) - 0x80000;
+    return rem > 16 || rem < -16;
+  }
+  const float t = __uint_as_float(b) * 512.0f;  // exact: grid -> integers
+  return fabsf(t - truncf(t) - 0.5f) > (1.0f / 4096.0f);
+}
+
+// 8 values -> 8 E4M3 codes of fl32(x / s), packed little-endian in two words.
+// `r` = RN(1/s); `exact_only` forces the division (scales that are not normal).
+__device__ __forceinline__ uint2 quantize8(const float (&f)[8], float s, float r, bool exact_only) {
+  float y[8];
+  bool stable = !exact_only;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    y[i] = __fmul_rn(f[i], r);
+    stable = stable && e4m3_code_is_stable(y[i]);
+  }
+  if (!stable) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = __fdiv_rn(f[i], s);
+  }
   uint32_t p[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) p[i] = cvt_e4m3x2(__fdiv_rn(f[2 * i], s), __fdiv_rn(f[2 * i + 1], s));
+  for (int i = 0; i < 4; ++i) p[i] = cvt_e4m3x2(y[2 * i], y[2 * i + 1]);
   return make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
 }
+
+// Scales below this are not safely normal for the reciprocal path.
+constexpr float kMinFastScale = 0x1p-125f;
 
 // ---------------------------------------------------------------------------
 // 1x128 activation tiles.  A tile is 128 bf16 = 256 contiguous bytes; a
@@ -82,8 +121,9 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint4* __res
 #pragma unroll
       for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
       const float sc = group_scale(amax);
+      const float rc = __frcp_rn(sc);
       if (t < num_tiles) {
-        q[t * 16 + sub] = quantize8(f, sc);
+        q[t * 16 + sub] = quantize8(f, sc, rc, sc < kMinFastScale);
         if (sub == 0) s[t] = sc;
       }
     }
@@ -129,12 +169,14 @@ __global__ void __launch_bounds__(256) quant_w_128x128_kernel(const uint8_t* __r
 #pragma unroll
     for (int i = 1; i < 8; ++i) amax = fmaxf(amax, warp_max[i]);
     const float sc = group_scale(amax);
+    const float rc = __frcp_rn(sc);
+    const bool exact_only = sc < kMinFastScale;
     uint8_t* dst = q + row0 * K + kb * 128;
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
       float f[8];
       bf16x8_to_float(v[p], f);
-      *reinterpret_cast<uint2*>(dst + (p * 16 + rsub) * K + sub * 8) = quantize8(f, sc);
+      *reinterpret_cast<uint2*>(dst + (p * 16 + rsub) * K + sub * 8) = quantize8(f, sc, rc, exact_only);
     }
     if (tid == 0) s[b] = sc;
     __syncthreads();  // warp_max is reused by the next block

@@ -143,3 +143,45 @@ def test_moe_masked_full(dev):
     assert_w_exact(d.b, dev)
     assert_act_exact(d.a2.reshape(-1, d.a2.shape[-1]), dev)
     assert_w_exact(d.b2, dev)
+
+
+def _near_midpoint_tiles(seed=17, n_scales=400):
+    """Tiles whose quotients x/s land within a few binary32 ulps of an E4M3
+    rounding midpoint (where a product with 1/s could round differently from
+    the quotient).  Selection only: the expected codes come from the oracle."""
+    rng = np.random.default_rng(seed)
+    pos = np.arange(1, 0x7F80, dtype=np.uint16)  # all positive finite bf16
+    xs_all = wl.bf16_to_f32(pos)
+    tiles = []
+    for _ in range(n_scales):
+        amax = np.float32(wl.bf16_to_f32(wl.bf16_bits(np.float32(np.exp(rng.uniform(-30, 30))))))
+        s = np.float32(amax / np.float32(448.0))
+        if s == 0 or s < np.float32(2.0 ** -125):
+            continue
+        xs = xs_all[xs_all <= amax]
+        qt = (xs / s).astype(np.float32)
+        b = qt.view(np.uint32)
+        normal = qt >= np.float32(2.0 ** -6)
+        rem = (b & np.uint32(0xFFFFF)).astype(np.int64) - 0x80000
+        near = normal & (np.abs(rem) <= 64)
+        t = qt * np.float32(512.0)
+        near |= (~normal) & (np.abs(t - np.trunc(t) - 0.5) <= 2.0 ** -16)
+        pick = xs[near][:127]
+        if pick.size == 0:
+            continue
+        row = np.zeros(128, dtype=np.float32)
+        row[0] = amax
+        row[1:1 + pick.size] = pick * np.where(rng.random(pick.size) < 0.5, -1, 1)
+        tiles.append(row)
+    return np.stack(tiles)
+
+
+def test_quotients_near_e4m3_midpoints(dev):
+    x = _near_midpoint_tiles()
+    assert x.shape[0] > 100
+    bits = wl.bf16_bits(x)
+    assert_act_exact(bits, dev)
+    # the same values as 128x128 weight blocks (one scale per block of 128 such rows)
+    rows = (x.shape[0] // 128) * 128
+    if rows:
+        assert_w_exact(np.ascontiguousarray(bits[:rows]), dev)
