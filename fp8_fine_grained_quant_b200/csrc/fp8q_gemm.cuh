@@ -12,13 +12,14 @@
 //
 // Design (B200):
 //   * persistent CTAs, one per SM, walking a static tile sequence;
-//   * warp 0: TMA producer (one 128-deep K slab of A [128 x 128 B] and
-//     B [BN x 128 B] per pipeline stage, 128-byte swizzle, mbarrier tx count);
-//   * warp 1: allocates TMEM and issues tcgen05.mma.kind::f8f6f4 (M = 128,
-//     N = BN, K = 32, four per slab) into one of two TMEM slab buffers; the
-//     first MMA of every slab overwrites, so each buffer holds exactly one
-//     slab's partial;
-//   * warp 2 builds the masked-layout tile table; warp 3 idles;
+//   * warps 0 and 3: TMA producers for alternate slabs (one 128-deep K slab
+//     of A [128 x 128 B] and B [BN x 128 B] per pipeline stage, 128-byte
+//     swizzle, mbarrier tx count);
+//   * warp 1 allocates TMEM; warps 1 and 2 issue tcgen05.mma.kind::f8f6f4
+//     (M = 128, N = BN, K = 32, four per slab) for alternate slabs into four
+//     TMEM slab buffers; the first MMA of every slab overwrites, so each
+//     buffer holds exactly one slab's partial;
+//   * warp 2 also builds the masked-layout tile table before the main loop;
 //   * warps 4-11: epilogue; warp w reads TMEM lanes 32*(w%4)..+31 (the rows the
 //     hardware lets it access) and half of the BN columns, applies
 //     acc += (sa * sb) * partial with packed FP32 FMAs, releases the buffer,
@@ -77,8 +78,8 @@ struct GemmSmem {
   static constexpr int kAccBufs = kTmemCols / kTmemStride;        // slab buffers in flight
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = STAGES * kABytes;
-  static constexpr uint32_t kOffBars = STAGES * kStageBytes;  // full[S], empty[S], tfull[B], tempty[B], drain
-  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * kAccBufs + 1;
+  static constexpr uint32_t kOffBars = STAGES * kStageBytes;  // full[S], empty[S], tfull[B], tempty[B], drain[2]
+  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * kAccBufs + 2;
   static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;     // tmem slot, abort flag, total tiles
   static constexpr uint32_t kOffPrefix = (kOffMisc + 16 + 15) / 16 * 16;
   static constexpr uint32_t kBytes = kOffPrefix + 4 * (kMaxMaskedExperts + 1);
@@ -159,28 +160,37 @@ struct Bars {
   __device__ uint32_t empty(int s) const { return base + 8u * (STAGES + s); }
   __device__ uint32_t tfull(int b) const { return base + 8u * (2 * STAGES + b); }
   __device__ uint32_t tempty(int b) const { return base + 8u * (2 * STAGES + ACC + b); }
-  __device__ uint32_t drain() const { return base + 8u * (2 * STAGES + 2 * ACC); }
+  __device__ uint32_t drain(int i) const { return base + 8u * (2 * STAGES + 2 * ACC + i); }
 };
 
-// TMA producer (one thread): one pipeline stage per 128-deep K slab.
+// TMA producer: one pipeline stage per 128-deep K slab.  Slabs are numbered
+// in the order this CTA processes them; producer `who` of `n` loads the slabs
+// j with j % n == who (a barrier probe costs ~150+ cycles of the issuing
+// thread's time, so two producers keep the ring full at one slab per ~256
+// cycles).
 template <int BN, int STAGES, Sched S>
 __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensorMap* tma_b, const GemmArgs& args,
-                                     const int32_t* prefix, uint32_t s_base, Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
-                                     int32_t total) {
+                                        const int32_t* prefix, uint32_t s_base,
+                                        Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
+                                        int32_t total, int who, int n) {
   using L = GemmSmem<BN, STAGES>;
   int stage = 0;
   uint32_t phase = 0;
+  uint32_t j = 0;
   uint32_t armed = 0, armed_parity = 0;  // per stage: ever armed / parity of its last phase
-  for (int32_t t = blockIdx.x; t < total && !*wc.abort; t += gridDim.x) {
+  bool ok = true;
+  for (int32_t t = blockIdx.x; ok && t < total && !*wc.abort; t += gridDim.x) {
     Tile tile;
     if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
-    for (int kb = 0; kb < args.nkb; ++kb) {
-      if (!mbar_wait(bars.empty(stage), phase ^ 1u, wc, 1)) break;
-      mbar_arrive_expect_tx(bars.full(stage), L::kStageBytes);
-      tma_load_2d(s_base + L::kOffA + stage * L::kABytes, tma_a, bars.full(stage), kb * kSlabK, tile.a_row);
-      tma_load_2d(s_base + L::kOffB + stage * L::kBBytes, tma_b, bars.full(stage), kb * kSlabK, tile.b_row);
-      armed |= 1u << stage;
-      armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+    for (int kb = 0; kb < args.nkb; ++kb, ++j) {
+      if (static_cast<int>(j % n) == who) {
+        if (!mbar_wait(bars.empty(stage), phase ^ 1u, wc, 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(bars.full(stage), L::kStageBytes);
+        tma_load_2d(s_base + L::kOffA + stage * L::kABytes, tma_a, bars.full(stage), kb * kSlabK, tile.a_row);
+        tma_load_2d(s_base + L::kOffB + stage * L::kBBytes, tma_b, bars.full(stage), kb * kSlabK, tile.b_row);
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+      }
       if (++stage == STAGES) {
         stage = 0;
         phase ^= 1u;
@@ -189,50 +199,58 @@ __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensor
   }
   if (*wc.abort) {
     // let copies still in flight land before the CTA exits (bounded, 1 ms each)
-    for (int s = 0; s < STAGES; ++s)
-      if (armed & (1u << s)) {
+    for (int st = 0; st < STAGES; ++st)
+      if (armed & (1u << st)) {
         const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(bars.full(s), (armed_parity >> s) & 1u) && globaltimer_ns() - t0 < 1000000ull) {
+        while (!mbar_try_wait(bars.full(st), (armed_parity >> st) & 1u) && globaltimer_ns() - t0 < 1000000ull) {
         }
       }
   }
 }
 
-// MMA issuer (one thread): four K = 32 MMAs per slab into one of kAccBufs
-// TMEM slab buffers, used round-robin.
+// MMA issuer: four K = 32 MMAs per slab into one of kAccBufs TMEM slab
+// buffers, used round-robin.  With per-slab promotion every slab starts a
+// fresh accumulator in its own buffer, so slabs are independent and issuer
+// `who` of `n` takes the slabs j with j % n == who: while one issuer waits on
+// a barrier probe the other keeps the tensor pipe fed.  The diagnostic mode
+// (no promotion) accumulates a whole tile in one buffer and uses one issuer.
 template <int BN, int STAGES, Sched S>
 __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* prefix, uint32_t s_base,
                                           Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
-                                          int32_t total, uint32_t tmem_base) {
+                                          int32_t total, uint32_t tmem_base, int who, int n) {
   using L = GemmSmem<BN, STAGES>;
   constexpr uint32_t kIdesc = idesc_e4m3_f32(kBlockM, BN);
   int stage = 0, buf = 0;
   uint32_t phase = 0, tphase = 0;
+  uint32_t j = 0;
   bool ok = true;
   for (int32_t t = blockIdx.x; ok && t < total && !*wc.abort; t += gridDim.x) {
     Tile tile;
     if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
-    for (int kb = 0; kb < args.nkb; ++kb) {
+    for (int kb = 0; kb < args.nkb; ++kb, ++j) {
+      const bool mine = static_cast<int>(j % n) == who;
       const bool new_acc = args.promote || kb == 0;
-      if (new_acc) {
-        if (!mbar_wait(bars.tempty(buf), tphase ^ 1u, wc, 2)) { ok = false; break; }
+      if (mine) {
+        if (new_acc) {
+          if (!mbar_wait(bars.tempty(buf), tphase ^ 1u, wc, 2)) { ok = false; break; }
+          tc_fence_after();
+        }
+        if (!mbar_wait(bars.full(stage), phase, wc, 3)) { ok = false; break; }
         tc_fence_after();
-      }
-      if (!mbar_wait(bars.full(stage), phase, wc, 3)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + buf * L::kTmemStride;
-      const uint64_t adesc = smem_desc_k_sw128(s_base + L::kOffA + stage * L::kABytes);
-      const uint64_t bdesc = smem_desc_k_sw128(s_base + L::kOffB + stage * L::kBBytes);
+        const uint32_t d_tmem = tmem_base + buf * L::kTmemStride;
+        const uint64_t adesc = smem_desc_k_sw128(s_base + L::kOffA + stage * L::kABytes);
+        const uint64_t bdesc = smem_desc_k_sw128(s_base + L::kOffB + stage * L::kBBytes);
 #pragma unroll
-      for (int k = 0; k < kSlabK / 32; ++k)
-        mma_e4m3(d_tmem, adesc + 2u * k, bdesc + 2u * k, kIdesc, (new_acc && k == 0) ? 0u : 1u);
-      mma_commit(bars.empty(stage));
+        for (int k = 0; k < kSlabK / 32; ++k)
+          mma_e4m3(d_tmem, adesc + 2u * k, bdesc + 2u * k, kIdesc, (new_acc && k == 0) ? 0u : 1u);
+        mma_commit(bars.empty(stage));
+        if (args.promote || kb == args.nkb - 1) mma_commit(bars.tfull(buf));
+      }
       if (++stage == STAGES) {
         stage = 0;
         phase ^= 1u;
       }
       if (args.promote || kb == args.nkb - 1) {
-        mma_commit(bars.tfull(buf));
         if (++buf == L::kAccBufs) {
           buf = 0;
           tphase ^= 1u;
@@ -240,10 +258,10 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
       }
     }
   }
-  // every issued MMA completes before TMEM is released
-  mma_commit(bars.drain());
+  // every MMA this thread issued completes before TMEM is released
+  mma_commit(bars.drain(who));
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bars.drain(), 0) && globaltimer_ns() - t0 < args.timeout_ns) {
+  while (!mbar_try_wait(bars.drain(who), 0) && globaltimer_ns() - t0 < args.timeout_ns) {
   }
 }
 
@@ -271,6 +289,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
   const int nnb = args.N / 128;
   int buf = 0;
   uint32_t tphase = 0;
+  bool ready = false;  // the current slab's buffer is already known to be full
   for (int32_t t = blockIdx.x; t < total && !*wc.abort; t += gridDim.x) {
     Tile tile;
     if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
@@ -295,9 +314,13 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
         sb_next = col_ok ? __ldg(sb_row + it + 1) : 0.0f;
       }
       // warp-uniform outcome: the tcgen05.ld below must be executed by all 32 lanes
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bars.tfull(buf), tphase, wc, 4))) { ok = false; break; }
+      if (!ready && !__all_sync(0xFFFFFFFFu, mbar_wait(bars.tfull(buf), tphase, wc, 4))) { ok = false; break; }
       tc_fence_after();
       const uint32_t t_buf = t_lane + buf * L::kTmemStride + half * kCols;
+      // probe the next slab's buffer now; the answer is used after this slab's work
+      const int nbuf = buf + 1 == L::kAccBufs ? 0 : buf + 1;
+      const uint32_t nphase = nbuf == 0 ? (tphase ^ 1u) : tphase;
+      const bool next_done = mbar_test_wait(bars.tfull(nbuf), nphase);
 #pragma unroll
       for (int g = 0; g < kGroups; ++g) {
         uint32_t v0[32], v1[32];
@@ -317,10 +340,9 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
           for (int j = 0; j < 16; ++j) ffma2_packed(acc[g * (kGroup / 2) + 16 + j], v1[2 * j], v1[2 * j + 1], scale2);
         }
       }
-      if (++buf == L::kAccBufs) {
-        buf = 0;
-        tphase ^= 1u;
-      }
+      ready = __all_sync(0xFFFFFFFFu, next_done);
+      buf = nbuf;
+      tphase = nphase;
     }
     if (!ok) break;
     if (row_ok && col_ok) {
@@ -367,7 +389,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(bars.tfull(b), 1);
       mbar_init(bars.tempty(b), 8);  // one arrival per epilogue warp
     }
-    mbar_init(bars.drain(), 1);
+    mbar_init(bars.drain(0), 1);
+    mbar_init(bars.drain(1), 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tma_a);
@@ -393,8 +416,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int32_t total = *total_slot;
 
   if (warp < 4) {
-    if (warp == 0 && lane == 0) produce<BN, STAGES, S>(&tma_a, &tma_b, args, prefix, s_base, bars, wc, total);
-    if (warp == 1 && lane == 0) issue_mma<BN, STAGES, S>(args, prefix, s_base, bars, wc, total, tmem_base);
+    // warps 0 and 3: TMA producers; warps 1 and 2: MMA issuers (one issuer
+    // when a tile accumulates in a single buffer)
+    const int n_mma = args.promote ? 2 : 1;
+    if (lane == 0) {
+      if (warp == 0 || warp == 3)
+        produce<BN, STAGES, S>(&tma_a, &tma_b, args, prefix, s_base, bars, wc, total, warp == 0 ? 0 : 1, 2);
+      else if (warp - 1 < n_mma)
+        issue_mma<BN, STAGES, S>(args, prefix, s_base, bars, wc, total, tmem_base, warp - 1, n_mma);
+    }
   } else {
     epilogue<BN, STAGES, S>(args, prefix, bars, wc, total, tmem_base, warp, lane);
   }

@@ -45,46 +45,44 @@ __device__ __forceinline__ float group_scale(float amax) {
 
 // Division-free quantization with an exactness filter.
 //
-// The code must be E4M3_RNE(fl32(x / s)).  With r = RN(1/s) (s a normal float)
-// and y = RN(x * r), |y - x/s| <= (2^-23 + 2^-48)|x/s| and fl32(x/s) is within
-// 2^-24 |x/s| of x/s, so y and fl32(x/s) are at most ~3 ulps of y apart.  The
-// E4M3 code changes only across a rounding midpoint, so whenever y is more
-// than 16 ulps from every midpoint both round to the same code.  Otherwise
-// (about 3e-5 of values) the exact IEEE quotient is used.
-//
-// Midpoints: for |y| >= 2^-6 the E4M3 grid keeps 3 fraction bits, so a midpoint
-// is a binary32 whose 20 dropped bits equal 0x80000; below 2^-6 the grid is
-// n * 2^-9 and the midpoints are (n + 1/2) * 2^-9.  Values that underflow in
-// the product are far below 2^-10 and give +-0 either way (the sign of x is
-// kept by the multiplication).
-__device__ __forceinline__ bool e4m3_code_is_stable(float y) {
-  const uint32_t b = __float_as_uint(y) & 0x7FFFFFFFu;
-  if (b >= 0x3C800000u) {  // |y| >= 2^-6
-    const int32_t rem = static_cast<int32_t>(b & 0xFFFFFu) - 0x80000;
-    return rem > 16 || rem < -16;
+// The code must be E4M3_RNE(fl32(x / s)).  With r = RN(1/s) (s a normal
+// float), r_lo = RN(r (1 - 2^-20)) and r_hi = RN(r (1 + 2^-20)):
+//   x r_lo = (x/s)(1 - 2^-20)(1 + d), |d| <= 4 * 2^-24, so x r_lo < fl32(x/s)
+//   (and symmetrically x r_hi > fl32(x/s)) for x > 0; the order flips for
+//   x < 0.  So fl32(x/s) lies between the two products y_lo = RN(x r_lo) and
+//   y_hi = RN(x r_hi).  Rounding to E4M3 is monotone, so when y_lo and y_hi get
+//   the same code, fl32(x/s) gets that code too.  When they differ (a quotient
+//   within ~2^-20 of a rounding midpoint, a few in 10^5) the IEEE quotient is
+//   used.  Results below the binary32 normal range are far below the first
+//   E4M3 midpoint (2^-10) and encode to +-0 on every path (the sign of x is
+//   kept by each multiplication).
+// 8 values -> 8 E4M3 codes of fl32(x / s), packed little-endian in two words.
+// `exact_only` forces the division (scales that are not safely normal).
+__device__ __forceinline__ uint2 quantize8(const float (&f)[8], float s, float r_lo, float r_hi, bool exact_only) {
+  uint32_t lo[4], hi[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    lo[i] = cvt_e4m3x2(__fmul_rn(f[2 * i], r_lo), __fmul_rn(f[2 * i + 1], r_lo));
+    hi[i] = cvt_e4m3x2(__fmul_rn(f[2 * i], r_hi), __fmul_rn(f[2 * i + 1], r_hi));
   }
-  const float t = __uint_as_float(b) * 512.0f;  // exact: grid -> integers
-  return fabsf(t - truncf(t) - 0.5f) > (1.0f / 4096.0f);
+  uint2 out = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
+  const uint2 chk = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
+  if (exact_only || out.x != chk.x || out.y != chk.y) {
+    uint32_t p[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[i] = cvt_e4m3x2(__fdiv_rn(f[2 * i], s), __fdiv_rn(f[2 * i + 1], s));
+    out = make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+  }
+  return out;
 }
 
-// 8 values -> 8 E4M3 codes of fl32(x / s), packed little-endian in two words.
-// `r` = RN(1/s); `exact_only` forces the division (scales that are not normal).
-__device__ __forceinline__ uint2 quantize8(const float (&f)[8], float s, float r, bool exact_only) {
-  float y[8];
-  bool stable = !exact_only;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    y[i] = __fmul_rn(f[i], r);
-    stable = stable && e4m3_code_is_stable(y[i]);
-  }
-  if (!stable) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = __fdiv_rn(f[i], s);
-  }
-  uint32_t p[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) p[i] = cvt_e4m3x2(y[2 * i], y[2 * i + 1]);
-  return make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+// The two bracketing reciprocals of a group scale.
+struct RecipPair {
+  float lo, hi;
+};
+__device__ __forceinline__ RecipPair recip_pair(float s) {
+  const float r = __frcp_rn(s);
+  return {__fmul_rn(r, 1.0f - 0x1p-20f), __fmul_rn(r, 1.0f + 0x1p-20f)};
 }
 
 // Scales below this are not safely normal for the reciprocal path.
@@ -121,9 +119,9 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint4* __res
 #pragma unroll
       for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
       const float sc = group_scale(amax);
-      const float rc = __frcp_rn(sc);
+      const RecipPair rp = recip_pair(sc);
       if (t < num_tiles) {
-        q[t * 16 + sub] = quantize8(f, sc, rc, sc < kMinFastScale);
+        q[t * 16 + sub] = quantize8(f, sc, rp.lo, rp.hi, sc < kMinFastScale);
         if (sub == 0) s[t] = sc;
       }
     }
@@ -137,7 +135,7 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint4* __res
 // from HBM once.  Block b = (g * N/128 + nb) * K/128 + kb, also the index of
 // its scale in s[G, N/128, K/128].  Grid-stride over blocks.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) quant_w_128x128_kernel(const uint8_t* __restrict__ w, uint8_t* __restrict__ q,
+__global__ void __launch_bounds__(256, 3) quant_w_128x128_kernel(const uint8_t* __restrict__ w, uint8_t* __restrict__ q,
                                                               float* __restrict__ s, int64_t N, int64_t K,
                                                               int64_t num_blocks) {
   __shared__ float warp_max[8];
@@ -169,14 +167,14 @@ __global__ void __launch_bounds__(256) quant_w_128x128_kernel(const uint8_t* __r
 #pragma unroll
     for (int i = 1; i < 8; ++i) amax = fmaxf(amax, warp_max[i]);
     const float sc = group_scale(amax);
-    const float rc = __frcp_rn(sc);
+    const RecipPair rp = recip_pair(sc);
     const bool exact_only = sc < kMinFastScale;
     uint8_t* dst = q + row0 * K + kb * 128;
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
       float f[8];
       bf16x8_to_float(v[p], f);
-      *reinterpret_cast<uint2*>(dst + (p * 16 + rsub) * K + sub * 8) = quantize8(f, sc, rc, exact_only);
+      *reinterpret_cast<uint2*>(dst + (p * 16 + rsub) * K + sub * 8) = quantize8(f, sc, rp.lo, rp.hi, exact_only);
     }
     if (tid == 0) s[b] = sc;
     __syncthreads();  // warp_max is reused by the next block
