@@ -78,8 +78,9 @@ struct GemmSmem {
   static constexpr int kAccBufs = kTmemCols / kTmemStride;        // slab buffers in flight
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = STAGES * kABytes;
-  static constexpr uint32_t kOffBars = STAGES * kStageBytes;  // full[S], empty[S], tfull[B], tempty[B], drain[2]
-  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * kAccBufs + 2;
+  // full[S], empty[S], tfull[B], tempty[B], drain[2], tpair[2]
+  static constexpr uint32_t kOffBars = STAGES * kStageBytes;
+  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * kAccBufs + 4;
   static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;     // tmem slot, abort flag, total tiles
   static constexpr uint32_t kOffPrefix = (kOffMisc + 16 + 15) / 16 * 16;
   static constexpr uint32_t kBytes = kOffPrefix + 4 * (kMaxMaskedExperts + 1);
@@ -161,6 +162,8 @@ struct Bars {
   __device__ uint32_t tfull(int b) const { return base + 8u * (2 * STAGES + b); }
   __device__ uint32_t tempty(int b) const { return base + 8u * (2 * STAGES + ACC + b); }
   __device__ uint32_t drain(int i) const { return base + 8u * (2 * STAGES + 2 * ACC + i); }
+  // pair barriers: complete when both slabs 2q and 2q+1 (q = pair index) are done
+  __device__ uint32_t tpair(int i) const { return base + 8u * (2 * STAGES + 2 * ACC + 2 + i); }
 };
 
 // TMA producer: one pipeline stage per 128-deep K slab.  Slabs are numbered
@@ -244,7 +247,10 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
         for (int k = 0; k < kSlabK / 32; ++k)
           mma_e4m3(d_tmem, adesc + 2u * k, bdesc + 2u * k, kIdesc, (new_acc && k == 0) ? 0u : 1u);
         mma_commit(bars.empty(stage));
-        if (args.promote || kb == args.nkb - 1) mma_commit(bars.tfull(buf));
+        if (args.promote)
+          mma_commit(bars.tpair((j >> 1) & 1));  // one of the pair's two arrivals
+        else if (kb == args.nkb - 1)
+          mma_commit(bars.tfull(buf));
       }
       if (++stage == STAGES) {
         stage = 0;
@@ -258,6 +264,10 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
       }
     }
   }
+  // An odd total leaves the last pair one arrival short: the issuer of that
+  // last slab supplies both.
+  if (ok && !*wc.abort && args.promote && (j & 1u) && static_cast<int>((j - 1) % n) == who)
+    mma_commit(bars.tpair(((j - 1) >> 1) & 1));
   // every MMA this thread issued completes before TMEM is released
   mma_commit(bars.drain(who));
   const uint64_t t0 = globaltimer_ns();
@@ -290,6 +300,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
   int buf = 0;
   uint32_t tphase = 0;
   bool ready = false;  // the current slab's buffer is already known to be full
+  uint32_t j = 0;      // slabs (promotion) or tiles (no promotion) consumed so far
   for (int32_t t = blockIdx.x; t < total && !*wc.abort; t += gridDim.x) {
     Tile tile;
     if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
@@ -313,14 +324,27 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
         sa_next = row_ok ? __ldg(sa_row + it + 1) : 0.0f;
         sb_next = col_ok ? __ldg(sb_row + it + 1) : 0.0f;
       }
-      // warp-uniform outcome: the tcgen05.ld below must be executed by all 32 lanes
-      if (!ready && !__all_sync(0xFFFFFFFFu, mbar_wait(bars.tfull(buf), tphase, wc, 4))) { ok = false; break; }
+      // Completion of the partial in this slab's buffer.  With promotion the
+      // MMA warps signal pairs of slabs (j even, j + 1) on one barrier, so a
+      // warp blocks at most once per two slabs, and the probe of the next
+      // pair is issued during the second slab and read after its work.
+      // Without promotion one barrier per tile buffer.  Warp-uniform: the
+      // tcgen05.ld below must be executed by all 32 lanes.
+      const uint32_t q = j >> 1;
+      if (!ready) {
+        const bool got = args.promote ? mbar_wait(bars.tpair(q & 1u), (q >> 1) & 1u, wc, 4)
+                                      : mbar_wait(bars.tfull(buf), tphase, wc, 4);
+        if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
+      }
       tc_fence_after();
       const uint32_t t_buf = t_lane + buf * L::kTmemStride + half * kCols;
-      // probe the next slab's buffer now; the answer is used after this slab's work
       const int nbuf = buf + 1 == L::kAccBufs ? 0 : buf + 1;
       const uint32_t nphase = nbuf == 0 ? (tphase ^ 1u) : tphase;
-      const bool next_done = mbar_test_wait(bars.tfull(nbuf), nphase);
+      bool next_done = true;  // even slab: its odd partner is covered by the same pair
+      if (!args.promote)
+        next_done = mbar_test_wait(bars.tfull(nbuf), nphase);
+      else if (j & 1u)
+        next_done = mbar_test_wait(bars.tpair((q + 1) & 1u), ((q + 1) >> 1) & 1u);
 #pragma unroll
       for (int g = 0; g < kGroups; ++g) {
         uint32_t v0[32], v1[32];
@@ -334,27 +358,28 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
           if (lane == 0) mbar_arrive(bars.tempty(buf));
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) ffma2_packed(acc[g * (kGroup / 2) + j], v0[2 * j], v0[2 * j + 1], scale2);
+        for (int i = 0; i < 16; ++i) ffma2_packed(acc[g * (kGroup / 2) + i], v0[2 * i], v0[2 * i + 1], scale2);
         if constexpr (kGroup == 64) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) ffma2_packed(acc[g * (kGroup / 2) + 16 + j], v1[2 * j], v1[2 * j + 1], scale2);
+          for (int i = 0; i < 16; ++i) ffma2_packed(acc[g * (kGroup / 2) + 16 + i], v1[2 * i], v1[2 * i + 1], scale2);
         }
       }
       ready = __all_sync(0xFFFFFFFFu, next_done);
       buf = nbuf;
       tphase = nphase;
+      ++j;
     }
     if (!ok) break;
     if (row_ok && col_ok) {
       __nv_bfloat16* crow = args.c + static_cast<int64_t>(tile.a_row + r) * args.N + col0;
 #pragma unroll
-      for (int j = 0; j < kCols; j += 8) {
+      for (int c = 0; c < kCols; c += 8) {
         uint4 o;
-        o.x = bf16x2_from_packed(acc[j / 2]);
-        o.y = bf16x2_from_packed(acc[j / 2 + 1]);
-        o.z = bf16x2_from_packed(acc[j / 2 + 2]);
-        o.w = bf16x2_from_packed(acc[j / 2 + 3]);
-        *reinterpret_cast<uint4*>(crow + j) = o;
+        o.x = bf16x2_from_packed(acc[c / 2]);
+        o.y = bf16x2_from_packed(acc[c / 2 + 1]);
+        o.z = bf16x2_from_packed(acc[c / 2 + 2]);
+        o.w = bf16x2_from_packed(acc[c / 2 + 3]);
+        *reinterpret_cast<uint4*>(crow + c) = o;
       }
     }
   }
@@ -391,6 +416,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     mbar_init(bars.drain(0), 1);
     mbar_init(bars.drain(1), 1);
+    mbar_init(bars.tpair(0), 2);  // one commit from each MMA issuer
+    mbar_init(bars.tpair(1), 2);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tma_a);
