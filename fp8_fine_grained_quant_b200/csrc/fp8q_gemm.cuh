@@ -43,6 +43,7 @@ constexpr int kSlabK = 128;  // promotion interval = scale slab
 constexpr int kGemmThreads = 384;  // warpgroup 0: TMA + MMA (+ scheduler set-up); 1-2: epilogue
 constexpr int kMaxMaskedExperts = 1024;
 
+
 struct GemmArgs {
   const float* sa;           // [rows of A][nkb]
   const float* sb;           // [E][N/128][nkb]
@@ -78,9 +79,9 @@ struct GemmSmem {
   static constexpr int kAccBufs = kTmemCols / kTmemStride;        // slab buffers in flight
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = STAGES * kABytes;
-  // full[S], empty[S], tfull[B], tempty[B], drain[2], tpair[2]
+  // full[S], empty[S], tfull[B], tempty[B], drain[2]
   static constexpr uint32_t kOffBars = STAGES * kStageBytes;
-  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * kAccBufs + 4;
+  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * kAccBufs + 2;
   static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;     // tmem slot, abort flag, total tiles
   static constexpr uint32_t kOffPrefix = (kOffMisc + 16 + 15) / 16 * 16;
   static constexpr uint32_t kBytes = kOffPrefix + 4 * (kMaxMaskedExperts + 1);
@@ -153,7 +154,33 @@ __device__ __forceinline__ bool get_tile(const GemmArgs& a, const int32_t* prefi
 }
 
 // ----------------------------------------------------------------- roles
-// Shared-memory barrier addresses (mbarrier objects, 8 bytes each).
+//
+// Barrier protocol.  Slabs are numbered j = 0, 1, ... in the order this CTA
+// processes them (tiles of its static sequence, then 128-deep K slabs within
+// a tile).  Slab j uses pipeline stage s = j % STAGES and, with promotion,
+// TMEM slab buffer j % kAccBufs.
+//   full[s]  : slab j's operands have landed (TMA transaction bytes) and, with
+//              promotion, TMEM buffer j % kAccBufs is free again: the eight
+//              epilogue warps arrive once they have read slab j - kAccBufs out
+//              of it (for the first kAccBufs slabs they arrive up front).
+//              Arrivals: 1 (producer) + 8 (epilogue) with promotion, else 1.
+//   empty[s] : the four MMAs of slab j have completed (one tcgen05.commit):
+//              stage s may be refilled (producer, for slab j + STAGES) and,
+//              with promotion, the partial in buffer j % kAccBufs is final
+//              (epilogue, for slab j).
+//   tfull/tempty[b] : only without promotion (the accumulation diagnostic),
+//              where a whole tile accumulates in buffer b.
+// Every role consumes in slab order, so no phase is re-armed before all its
+// waiters have passed it: the MMAs of slab j + STAGES wait for the epilogue's
+// release of slab j + STAGES - kAccBufs >= j, which it gives only after it has
+// observed empty[s] for slab j, and the producer observes empty[s] for slab j
+// before it loads slab j + STAGES.
+//
+// Each waiting role costs its thread ~150 cycles per barrier probe, and an MMA
+// instruction is accepted only as the tensor pipe frees up, so the TMA and MMA
+// roles are split over two threads each (slabs alternate between them) and
+// each issues one probe and one commit per slab.
+
 template <int STAGES, int ACC>
 struct Bars {
   uint32_t base;
@@ -162,31 +189,24 @@ struct Bars {
   __device__ uint32_t tfull(int b) const { return base + 8u * (2 * STAGES + b); }
   __device__ uint32_t tempty(int b) const { return base + 8u * (2 * STAGES + ACC + b); }
   __device__ uint32_t drain(int i) const { return base + 8u * (2 * STAGES + 2 * ACC + i); }
-  // pair barriers: complete when both slabs 2q and 2q+1 (q = pair index) are done
-  __device__ uint32_t tpair(int i) const { return base + 8u * (2 * STAGES + 2 * ACC + 2 + i); }
 };
 
-// TMA producer: one pipeline stage per 128-deep K slab.  Slabs are numbered
-// in the order this CTA processes them; producer `who` of `n` loads the slabs
-// j with j % n == who (a barrier probe costs ~150+ cycles of the issuing
-// thread's time, so two producers keep the ring full at one slab per ~256
-// cycles).
+// TMA producer `who` of two: loads the slabs j with j % 2 == who.
 template <int BN, int STAGES, Sched S>
 __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensorMap* tma_b, const GemmArgs& args,
                                         const int32_t* prefix, uint32_t s_base,
                                         Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
-                                        int32_t total, int who, int n) {
+                                        int32_t total, uint32_t who) {
   using L = GemmSmem<BN, STAGES>;
   int stage = 0;
-  uint32_t phase = 0;
-  uint32_t j = 0;
+  uint32_t phase = 0, j = 0;
   uint32_t armed = 0, armed_parity = 0;  // per stage: ever armed / parity of its last phase
   bool ok = true;
   for (int32_t t = blockIdx.x; ok && t < total && !*wc.abort; t += gridDim.x) {
     Tile tile;
     if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
     for (int kb = 0; kb < args.nkb; ++kb, ++j) {
-      if (static_cast<int>(j % n) == who) {
+      if ((j & 1u) == who) {
         if (!mbar_wait(bars.empty(stage), phase ^ 1u, wc, 1)) { ok = false; break; }
         mbar_arrive_expect_tx(bars.full(stage), L::kStageBytes);
         tma_load_2d(s_base + L::kOffA + stage * L::kABytes, tma_a, bars.full(stage), kb * kSlabK, tile.a_row);
@@ -211,52 +231,46 @@ __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensor
   }
 }
 
-// MMA issuer: four K = 32 MMAs per slab into one of kAccBufs TMEM slab
-// buffers, used round-robin.  With per-slab promotion every slab starts a
-// fresh accumulator in its own buffer, so slabs are independent and issuer
-// `who` of `n` takes the slabs j with j % n == who: while one issuer waits on
-// a barrier probe the other keeps the tensor pipe fed.  The diagnostic mode
-// (no promotion) accumulates a whole tile in one buffer and uses one issuer.
+// MMA issuer `who` of `n`: four K = 32 MMAs per slab.  With promotion every
+// slab starts a fresh accumulator in its own TMEM buffer, so slabs are
+// independent and two issuers take alternate slabs.  Without promotion a tile
+// accumulates in one buffer and one issuer (n = 1) does all of it.
 template <int BN, int STAGES, Sched S>
 __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* prefix, uint32_t s_base,
                                           Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
-                                          int32_t total, uint32_t tmem_base, int who, int n) {
+                                          int32_t total, uint32_t tmem_base, uint32_t who, uint32_t n) {
   using L = GemmSmem<BN, STAGES>;
   constexpr uint32_t kIdesc = idesc_e4m3_f32(kBlockM, BN);
+  const bool promote = args.promote != 0;
+  const uint32_t mask = n - 1;  // n is 1 or 2
   int stage = 0, buf = 0;
-  uint32_t phase = 0, tphase = 0;
-  uint32_t j = 0;
+  uint32_t phase = 0, tphase = 0, j = 0;
   bool ok = true;
   for (int32_t t = blockIdx.x; ok && t < total && !*wc.abort; t += gridDim.x) {
     Tile tile;
     if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
     for (int kb = 0; kb < args.nkb; ++kb, ++j) {
-      const bool mine = static_cast<int>(j % n) == who;
-      const bool new_acc = args.promote || kb == 0;
-      if (mine) {
-        if (new_acc) {
+      if ((j & mask) == who) {
+        if (!promote && kb == 0) {
           if (!mbar_wait(bars.tempty(buf), tphase ^ 1u, wc, 2)) { ok = false; break; }
-          tc_fence_after();
         }
         if (!mbar_wait(bars.full(stage), phase, wc, 3)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * L::kTmemStride;
         const uint64_t adesc = smem_desc_k_sw128(s_base + L::kOffA + stage * L::kABytes);
         const uint64_t bdesc = smem_desc_k_sw128(s_base + L::kOffB + stage * L::kBBytes);
+        const uint32_t fresh = (promote || kb == 0) ? 0u : 1u;
+        mma_e4m3(d_tmem, adesc, bdesc, kIdesc, fresh);
 #pragma unroll
-        for (int k = 0; k < kSlabK / 32; ++k)
-          mma_e4m3(d_tmem, adesc + 2u * k, bdesc + 2u * k, kIdesc, (new_acc && k == 0) ? 0u : 1u);
+        for (int k = 1; k < kSlabK / 32; ++k) mma_e4m3(d_tmem, adesc + 2u * k, bdesc + 2u * k, kIdesc, 1u);
         mma_commit(bars.empty(stage));
-        if (args.promote)
-          mma_commit(bars.tpair((j >> 1) & 1));  // one of the pair's two arrivals
-        else if (kb == args.nkb - 1)
-          mma_commit(bars.tfull(buf));
+        if (!promote && kb == args.nkb - 1) mma_commit(bars.tfull(buf));
       }
       if (++stage == STAGES) {
         stage = 0;
         phase ^= 1u;
       }
-      if (args.promote || kb == args.nkb - 1) {
+      if (promote || kb == args.nkb - 1) {
         if (++buf == L::kAccBufs) {
           buf = 0;
           tphase ^= 1u;
@@ -264,10 +278,6 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
       }
     }
   }
-  // An odd total leaves the last pair one arrival short: the issuer of that
-  // last slab supplies both.
-  if (ok && !*wc.abort && args.promote && (j & 1u) && static_cast<int>((j - 1) % n) == who)
-    mma_commit(bars.tpair(((j - 1) >> 1) & 1));
   // every MMA this thread issued completes before TMEM is released
   mma_commit(bars.drain(who));
   const uint64_t t0 = globaltimer_ns();
@@ -277,11 +287,12 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
 
 // Epilogue warp: promotion of every slab partial into FP32 registers, then the
 // bf16 store of the finished tile.  Warp w owns TMEM lanes 32*(w%4)..+31 (tile
-// rows) and kCols = BN/2 columns.  Each half lies inside one 128-column weight
-// block (BN in {128, 256}), so one sb value per slab.  Per slab the warp loads
-// its columns in groups of up to 64 (two 32-column TMEM loads, one wait), hands
-// the buffer back to the MMA warp as soon as the last group is in registers,
-// and then applies acc += (sa * sb) * partial with packed FP32 FMAs.
+// rows) and kCols = BN/2 columns; for BN in {128, 256} each half lies inside
+// one 128-column weight block, so one sb value per slab.  Per slab the warp
+// loads its columns (two 32-column TMEM loads, one wait), hands the buffer
+// back as soon as the values are in registers, then applies
+// acc += (sa * sb) * partial.  The completion probe of the next slab is issued
+// before this slab's work and read after it.
 template <int BN, int STAGES, Sched S>
 __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* prefix,
                                          Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
@@ -290,17 +301,19 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
   constexpr int kCols = BN / 2;
   constexpr int kGroup = kCols < 64 ? kCols : 64;
   constexpr int kGroups = kCols / kGroup;
+  constexpr int kAcc = L::kAccBufs;
   static_assert(kCols <= 128 && 128 % kCols == 0 && kGroup % 32 == 0, "each half must sit in one scale block");
+  static_assert(kAcc < STAGES, "buffer releases are posted on the stage barrier of a later slab");
+  const bool promote = args.promote != 0;
   const int quad = warp & 3;
   const int half = (warp - 4) >> 2;
   const int r = quad * 32 + lane;
   const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
   const int nkb = args.nkb;
   const int nnb = args.N / 128;
-  int buf = 0;
-  uint32_t tphase = 0;
-  bool ready = false;  // the current slab's buffer is already known to be full
-  uint32_t j = 0;      // slabs (promotion) or tiles (no promotion) consumed so far
+  int buf = 0, stage = 0;
+  uint32_t tphase = 0, phase = 0;
+  bool ready = false;  // the current slab (or tile, without promotion) is known complete
   for (int32_t t = blockIdx.x; t < total && !*wc.abort; t += gridDim.x) {
     Tile tile;
     if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
@@ -309,42 +322,35 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
     const bool col_ok = col0 < args.N;
     const float* sa_row = args.sa + static_cast<int64_t>(tile.a_row + (row_ok ? r : 0)) * nkb;
     const float* sb_row = args.sb + (static_cast<int64_t>(tile.e) * nnb + (col_ok ? col0 / 128 : 0)) * nkb;
-    uint64_t acc[kCols / 2];  // packed pairs of FP32 running sums
+    float acc[kCols];
 #pragma unroll
-    for (int i = 0; i < kCols / 2; ++i) acc[i] = 0ull;
+    for (int i = 0; i < kCols; ++i) acc[i] = 0.0f;
 
-    const int n_reads = args.promote ? nkb : 1;
+    const int n_reads = promote ? nkb : 1;
     // the next slab's scales are fetched one slab ahead
     float sa_next = row_ok ? __ldg(sa_row) : 0.0f;
     float sb_next = col_ok ? __ldg(sb_row) : 0.0f;
     bool ok = true;
     for (int it = 0; it < n_reads; ++it) {
-      const uint64_t scale2 = pack_f32x2(sa_next * sb_next);
+      const float scale = sa_next * sb_next;
       if (it + 1 < n_reads) {
         sa_next = row_ok ? __ldg(sa_row + it + 1) : 0.0f;
         sb_next = col_ok ? __ldg(sb_row + it + 1) : 0.0f;
       }
-      // Completion of the partial in this slab's buffer.  With promotion the
-      // MMA warps signal pairs of slabs (j even, j + 1) on one barrier, so a
-      // warp blocks at most once per two slabs, and the probe of the next
-      // pair is issued during the second slab and read after its work.
-      // Without promotion one barrier per tile buffer.  Warp-uniform: the
-      // tcgen05.ld below must be executed by all 32 lanes.
-      const uint32_t q = j >> 1;
+      // Warp-uniform outcome: the tcgen05.ld below must be executed by all 32 lanes.
       if (!ready) {
-        const bool got = args.promote ? mbar_wait(bars.tpair(q & 1u), (q >> 1) & 1u, wc, 4)
-                                      : mbar_wait(bars.tfull(buf), tphase, wc, 4);
+        const bool got = promote ? mbar_wait(bars.empty(stage), phase, wc, 4) : mbar_wait(bars.tfull(buf), tphase, wc, 4);
         if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
       }
       tc_fence_after();
       const uint32_t t_buf = t_lane + buf * L::kTmemStride + half * kCols;
-      const int nbuf = buf + 1 == L::kAccBufs ? 0 : buf + 1;
-      const uint32_t nphase = nbuf == 0 ? (tphase ^ 1u) : tphase;
-      bool next_done = true;  // even slab: its odd partner is covered by the same pair
-      if (!args.promote)
-        next_done = mbar_test_wait(bars.tfull(nbuf), nphase);
-      else if (j & 1u)
-        next_done = mbar_test_wait(bars.tpair((q + 1) & 1u), ((q + 1) >> 1) & 1u);
+      // position of the next slab (promotion) or tile (no promotion)
+      const int nbuf = buf + 1 == kAcc ? 0 : buf + 1;
+      const uint32_t ntphase = nbuf == 0 ? (tphase ^ 1u) : tphase;
+      const int nstage = stage + 1 == STAGES ? 0 : stage + 1;
+      const uint32_t nphase = nstage == 0 ? (phase ^ 1u) : phase;
+      const bool next_done = promote ? mbar_test_wait(bars.empty(nstage), nphase)
+                                     : mbar_test_wait(bars.tfull(nbuf), ntphase);
 #pragma unroll
       for (int g = 0; g < kGroups; ++g) {
         uint32_t v0[32], v1[32];
@@ -353,21 +359,36 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
         tmem_ld_wait(v0);
         if constexpr (kGroup == 64) reg_fence(v1);
         if (g == kGroups - 1) {
+          // buffer free: with promotion it serves slab j + kAcc, whose stage barrier takes the arrival
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bars.tempty(buf));
+          if (lane == 0) {
+            if (promote) {
+              int rs = stage + kAcc;
+              if (rs >= STAGES) rs -= STAGES;
+              mbar_arrive(bars.full(rs));
+            } else {
+              mbar_arrive(bars.tempty(buf));
+            }
+          }
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) ffma2_packed(acc[g * (kGroup / 2) + i], v0[2 * i], v0[2 * i + 1], scale2);
+        for (int i = 0; i < 32; ++i) acc[g * kGroup + i] = fmaf(__uint_as_float(v0[i]), scale, acc[g * kGroup + i]);
         if constexpr (kGroup == 64) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) ffma2_packed(acc[g * (kGroup / 2) + 16 + i], v1[2 * i], v1[2 * i + 1], scale2);
+          for (int i = 0; i < 32; ++i)
+            acc[g * kGroup + 32 + i] = fmaf(__uint_as_float(v1[i]), scale, acc[g * kGroup + 32 + i]);
         }
       }
       ready = __all_sync(0xFFFFFFFFu, next_done);
-      buf = nbuf;
-      tphase = nphase;
-      ++j;
+      if (promote) {
+        buf = nbuf;
+        stage = nstage;
+        phase = nphase;
+      } else {
+        buf = nbuf;
+        tphase = ntphase;
+      }
     }
     if (!ok) break;
     if (row_ok && col_ok) {
@@ -375,10 +396,10 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
 #pragma unroll
       for (int c = 0; c < kCols; c += 8) {
         uint4 o;
-        o.x = bf16x2_from_packed(acc[c / 2]);
-        o.y = bf16x2_from_packed(acc[c / 2 + 1]);
-        o.z = bf16x2_from_packed(acc[c / 2 + 2]);
-        o.w = bf16x2_from_packed(acc[c / 2 + 3]);
+        o.x = bf16x2_rn(acc[c], acc[c + 1]);
+        o.y = bf16x2_rn(acc[c + 2], acc[c + 3]);
+        o.z = bf16x2_rn(acc[c + 4], acc[c + 5]);
+        o.w = bf16x2_rn(acc[c + 6], acc[c + 7]);
         *reinterpret_cast<uint4*>(crow + c) = o;
       }
     }
@@ -396,7 +417,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
-  const Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars{s_base + L::kOffBars};
+  const Bars<STAGES, L::kAccBufs> bars{s_base + L::kOffBars};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
   int32_t* total_slot = reinterpret_cast<int32_t*>(smem + L::kOffMisc + 8);
@@ -404,11 +425,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl wc{args.timeout_ns, args.status, abort_flag};
+  const bool promote = args.promote != 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bars.full(s), 1);
-      mbar_init(bars.empty(s), 1);
+    for (int st = 0; st < STAGES; ++st) {
+      mbar_init(bars.full(st), promote ? 1 + 8 : 1);  // producer (+ the eight epilogue warps)
+      mbar_init(bars.empty(st), 1);
     }
     for (int b = 0; b < L::kAccBufs; ++b) {
       mbar_init(bars.tfull(b), 1);
@@ -416,8 +438,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     mbar_init(bars.drain(0), 1);
     mbar_init(bars.drain(1), 1);
-    mbar_init(bars.tpair(0), 2);  // one commit from each MMA issuer
-    mbar_init(bars.tpair(1), 2);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tma_a);
@@ -445,14 +465,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp < 4) {
     // warps 0 and 3: TMA producers; warps 1 and 2: MMA issuers (one issuer
     // when a tile accumulates in a single buffer)
-    const int n_mma = args.promote ? 2 : 1;
+    const uint32_t n_mma = promote ? 2u : 1u;
     if (lane == 0) {
       if (warp == 0 || warp == 3)
-        produce<BN, STAGES, S>(&tma_a, &tma_b, args, prefix, s_base, bars, wc, total, warp == 0 ? 0 : 1, 2);
-      else if (warp - 1 < n_mma)
+        produce<BN, STAGES, S>(&tma_a, &tma_b, args, prefix, s_base, bars, wc, total, warp == 0 ? 0u : 1u);
+      else if (static_cast<uint32_t>(warp - 1) < n_mma)
         issue_mma<BN, STAGES, S>(args, prefix, s_base, bars, wc, total, tmem_base, warp - 1, n_mma);
     }
   } else {
+    // all TMEM slab buffers start free: release them for the first slabs
+    if (promote && lane == 0)
+      for (int b = 0; b < L::kAccBufs; ++b) mbar_arrive(bars.full(b));
     epilogue<BN, STAGES, S>(args, prefix, bars, wc, total, tmem_base, warp, lane);
   }
 

@@ -224,6 +224,13 @@ __device__ __forceinline__ uint32_t bf16x2_from_packed(uint64_t p) {
   return r;
 }
 
+// Two FP32 values -> packed bf16 pair (round to nearest even); `lo` first in memory.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // Orders later uses of r after the preceding tcgen05.wait::ld (no instruction).
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
   asm volatile(""
