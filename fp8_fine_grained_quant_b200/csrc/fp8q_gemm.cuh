@@ -322,9 +322,9 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
     const bool col_ok = col0 < args.N;
     const float* sa_row = args.sa + static_cast<int64_t>(tile.a_row + (row_ok ? r : 0)) * nkb;
     const float* sb_row = args.sb + (static_cast<int64_t>(tile.e) * nnb + (col_ok ? col0 / 128 : 0)) * nkb;
-    float acc[kCols];
+    uint64_t acc[kCols / 2];  // packed pairs of FP32 running sums
 #pragma unroll
-    for (int i = 0; i < kCols; ++i) acc[i] = 0.0f;
+    for (int i = 0; i < kCols / 2; ++i) acc[i] = 0ull;
 
     const int n_reads = promote ? nkb : 1;
     // the next slab's scales are fetched one slab ahead
@@ -332,7 +332,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
     float sb_next = col_ok ? __ldg(sb_row) : 0.0f;
     bool ok = true;
     for (int it = 0; it < n_reads; ++it) {
-      const float scale = sa_next * sb_next;
+      const uint64_t scale2 = pack_f32x2(sa_next * sb_next);
       if (it + 1 < n_reads) {
         sa_next = row_ok ? __ldg(sa_row + it + 1) : 0.0f;
         sb_next = col_ok ? __ldg(sb_row + it + 1) : 0.0f;
@@ -351,13 +351,11 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
       const uint32_t nphase = nstage == 0 ? (phase ^ 1u) : phase;
       const bool next_done = promote ? mbar_test_wait(bars.empty(nstage), nphase)
                                      : mbar_test_wait(bars.tfull(nbuf), ntphase);
+      static_assert(kGroup == 64, "the promotion loads 64 columns per group");
 #pragma unroll
       for (int g = 0; g < kGroups; ++g) {
-        uint32_t v0[32], v1[32];
-        tmem_ld_32x32b_x32(t_buf + g * kGroup, v0);
-        if constexpr (kGroup == 64) tmem_ld_32x32b_x32(t_buf + g * kGroup + 32, v1);
-        tmem_ld_wait(v0);
-        if constexpr (kGroup == 64) reg_fence(v1);
+        uint64_t v[32];
+        tmem_ld_32x32b_x64_pairs(t_buf + g * kGroup, v);
         if (g == kGroups - 1) {
           // buffer free: with promotion it serves slab j + kAcc, whose stage barrier takes the arrival
           tc_fence_before();
@@ -373,12 +371,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
           }
         }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[g * kGroup + i] = fmaf(__uint_as_float(v0[i]), scale, acc[g * kGroup + i]);
-        if constexpr (kGroup == 64) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            acc[g * kGroup + 32 + i] = fmaf(__uint_as_float(v1[i]), scale, acc[g * kGroup + 32 + i]);
-        }
+        for (int i = 0; i < 32; ++i) ffma2(acc[g * 32 + i], v[i], scale2);
       }
       ready = __all_sync(0xFFFFFFFFu, next_done);
       if (promote) {
@@ -396,10 +389,10 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
 #pragma unroll
       for (int c = 0; c < kCols; c += 8) {
         uint4 o;
-        o.x = bf16x2_rn(acc[c], acc[c + 1]);
-        o.y = bf16x2_rn(acc[c + 2], acc[c + 3]);
-        o.z = bf16x2_rn(acc[c + 4], acc[c + 5]);
-        o.w = bf16x2_rn(acc[c + 6], acc[c + 7]);
+        o.x = bf16x2_from_pair(acc[c / 2]);
+        o.y = bf16x2_from_pair(acc[c / 2 + 1]);
+        o.z = bf16x2_from_pair(acc[c / 2 + 2]);
+        o.w = bf16x2_from_pair(acc[c / 2 + 3]);
         *reinterpret_cast<uint4*>(crow + c) = o;
       }
     }

@@ -187,6 +187,69 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
+// 32 lanes x 64 consecutive 32-bit columns (two 32-column loads), waited for
+// and returned as 32 packed pairs of FP32 values (column 2i in the low half of
+// p[i]).  The pairing happens after the wait inside one asm block, so the
+// register allocator can place each pair directly.
+__device__ __forceinline__ void tmem_ld_32x32b_x64_pairs(uint32_t taddr, uint64_t (&p)[32]) {
+  asm volatile(
+      "{\n\t.reg .b32 r0,r1,r2,r3,r4,r5,r6,r7,r8,r9,r10,r11,r12,r13,r14,r15,r16,r17,r18,r19,r20,r21,r22,r23,r24,r25,r26,r27,r28,r29,r30,r31;\n\t"
+      ".reg .b32 q0,q1,q2,q3,q4,q5,q6,q7,q8,q9,q10,q11,q12,q13,q14,q15,q16,q17,q18,q19,q20,q21,q22,q23,q24,q25,q26,q27,q28,q29,q30,q31;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {r0,r1,r2,r3,r4,r5,r6,r7,r8,r9,r10,r11,r12,r13,r14,r15,r16,r17,r18,r19,r20,r21,r22,r23,r24,r25,r26,r27,r28,r29,r30,r31}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {q0,q1,q2,q3,q4,q5,q6,q7,q8,q9,q10,q11,q12,q13,q14,q15,q16,q17,q18,q19,q20,q21,q22,q23,q24,q25,q26,q27,q28,q29,q30,q31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t"
+      "mov.b64 %0, {r0, r1};\n\t"
+      "mov.b64 %1, {r2, r3};\n\t"
+      "mov.b64 %2, {r4, r5};\n\t"
+      "mov.b64 %3, {r6, r7};\n\t"
+      "mov.b64 %4, {r8, r9};\n\t"
+      "mov.b64 %5, {r10, r11};\n\t"
+      "mov.b64 %6, {r12, r13};\n\t"
+      "mov.b64 %7, {r14, r15};\n\t"
+      "mov.b64 %8, {r16, r17};\n\t"
+      "mov.b64 %9, {r18, r19};\n\t"
+      "mov.b64 %10, {r20, r21};\n\t"
+      "mov.b64 %11, {r22, r23};\n\t"
+      "mov.b64 %12, {r24, r25};\n\t"
+      "mov.b64 %13, {r26, r27};\n\t"
+      "mov.b64 %14, {r28, r29};\n\t"
+      "mov.b64 %15, {r30, r31};\n\t"
+      "mov.b64 %16, {q0, q1};\n\t"
+      "mov.b64 %17, {q2, q3};\n\t"
+      "mov.b64 %18, {q4, q5};\n\t"
+      "mov.b64 %19, {q6, q7};\n\t"
+      "mov.b64 %20, {q8, q9};\n\t"
+      "mov.b64 %21, {q10, q11};\n\t"
+      "mov.b64 %22, {q12, q13};\n\t"
+      "mov.b64 %23, {q14, q15};\n\t"
+      "mov.b64 %24, {q16, q17};\n\t"
+      "mov.b64 %25, {q18, q19};\n\t"
+      "mov.b64 %26, {q20, q21};\n\t"
+      "mov.b64 %27, {q22, q23};\n\t"
+      "mov.b64 %28, {q24, q25};\n\t"
+      "mov.b64 %29, {q26, q27};\n\t"
+      "mov.b64 %30, {q28, q29};\n\t"
+      "mov.b64 %31, {q30, q31};\n\t"
+      "}"
+      : "=l"(p[0]), "=l"(p[1]), "=l"(p[2]), "=l"(p[3]), "=l"(p[4]), "=l"(p[5]), "=l"(p[6]), "=l"(p[7]), "=l"(p[8]), "=l"(p[9]), "=l"(p[10]), "=l"(p[11]), "=l"(p[12]), "=l"(p[13]), "=l"(p[14]), "=l"(p[15]), "=l"(p[16]), "=l"(p[17]), "=l"(p[18]), "=l"(p[19]), "=l"(p[20]), "=l"(p[21]), "=l"(p[22]), "=l"(p[23]), "=l"(p[24]), "=l"(p[25]), "=l"(p[26]), "=l"(p[27]), "=l"(p[28]), "=l"(p[29]), "=l"(p[30]), "=l"(p[31])
+      : "r"(taddr), "r"(taddr + 32)
+      : "memory");
+}
+
+// acc += pair * scale2: two FP32 fused multiply-adds in one instruction.
+__device__ __forceinline__ void ffma2(uint64_t& acc, uint64_t pair, uint64_t scale2) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(pair), "l"(scale2));
+}
+
+// Packed FP32 pair -> packed bf16 pair (round to nearest even); low half first in memory.
+__device__ __forceinline__ uint32_t bf16x2_from_pair(uint64_t p) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // Waits for this thread's outstanding tcgen05.ld; the registers are passed
 // through so no use of them can be scheduled before the wait.
 __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
