@@ -14,6 +14,9 @@
 #include "fp8q.h"
 #include "fp8q_gemm.cuh"
 #include "fp8q_ptx.cuh"
+#ifndef FP8Q_ACT_UNROLL
+#define FP8Q_ACT_UNROLL 2
+#endif
 #include "fp8q_quant.cuh"
 
 namespace fp8q {
@@ -214,18 +217,18 @@ int fp8_quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, fl
   if (M < 0 || K < 0 || K % 128) return FP8Q_ERR_SHAPE;
   if (M == 0 || K == 0) return FP8Q_OK;
   if (!x_bf16 || !q || !s) return FP8Q_ERR_NULL;
-  if (!aligned(x_bf16, 16) || !aligned(q, 16) || !aligned(s, 4)) return FP8Q_ERR_ALIGN;
+  if (!aligned(x_bf16, 32) || !aligned(q, 16) || !aligned(s, 4)) return FP8Q_ERR_ALIGN;
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);
   if (rc) return rc;
   const int64_t tiles = M * (K / 128);
-  constexpr int kUnroll = 4;
-  const int64_t per_cta = (256 / 16) * kUnroll;
+  constexpr int kUnroll = FP8Q_ACT_UNROLL;
+  const int64_t per_cta = (256 / 8) * kUnroll;
   int64_t grid = (tiles + per_cta - 1) / per_cta;
   const int64_t cap = static_cast<int64_t>(dev->num_sms) * 8;
   if (grid > cap) grid = cap;
   quant_act_1x128_kernel<kUnroll><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
-      static_cast<const uint4*>(x_bf16), reinterpret_cast<uint2*>(q), s, tiles);
+      static_cast<const uint8_t*>(x_bf16), q, s, tiles);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FP8Q_OK;
@@ -236,7 +239,7 @@ int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, uin
   if (G < 0 || N < 0 || K < 0 || N % 128 || K % 128) return FP8Q_ERR_SHAPE;
   if (G == 0 || N == 0 || K == 0) return FP8Q_OK;
   if (!w_bf16 || !q || !s) return FP8Q_ERR_NULL;
-  if (!aligned(w_bf16, 16) || !aligned(q, 16) || !aligned(s, 4)) return FP8Q_ERR_ALIGN;
+  if (!aligned(w_bf16, 32) || !aligned(q, 16) || !aligned(s, 4)) return FP8Q_ERR_ALIGN;
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);
   if (rc) return rc;
@@ -244,7 +247,7 @@ int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, uin
   const int64_t cap = static_cast<int64_t>(dev->num_sms) * 64;
   const int64_t grid = blocks < cap ? blocks : cap;
   quant_w_128x128_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(static_cast<const uint8_t*>(w_bf16), q, s,
-                                                                           N, K, blocks);
+                                                                           K, blocks);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FP8Q_OK;

@@ -322,4 +322,41 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   return v;
 }
 
+// 32 bytes in one 256-bit load (read-only, not kept in L1); p 32-byte aligned.
+__device__ __forceinline__ void ld_nc_v8(const void* p, uint32_t (&w)[8]) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+               : "l"(p));
+}
+
+// The two bf16 of a 32-bit word as a packed pair of FP32 values (the bf16 at
+// the lower address in the low half).  bf16 is the top half of a binary32.
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+  return r;
+}
+
+// Packed FP32 product, each half rounded to nearest even.
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Two packed FP32 pairs -> four E4M3 codes (saturating RNE), in pair order,
+// low byte first.
+__device__ __forceinline__ uint32_t e4m3x4_from_f32x2(uint64_t p0, uint64_t p1) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 c0, c1;\n\t.reg .f32 a0, a1, a2, a3;\n\t"
+      "mov.b64 {a0, a1}, %1;\n\t"
+      "mov.b64 {a2, a3}, %2;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 c0, a1, a0;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 c1, a3, a2;\n\t"
+      "mov.b32 %0, {c0, c1};\n\t}"
+      : "=r"(r)
+      : "l"(p0), "l"(p1));
+  return r;
+}
+
 }  // namespace fp8q

@@ -30,8 +30,8 @@
  *    saturating at +-448, subnormal E4M3 codes down to 2^-9, sign of zero kept.
  *  - Argument errors return a non-zero status before anything is launched
  *    (no side effects).  A failed launch returns FP8Q_ERR_CUDA.
- *  - Pointer alignment: bf16 / FP8 / output pointers 16 bytes; scale and index
- *    pointers 4 bytes.
+ *  - Pointer alignment: the quantizers' bf16 inputs 32 bytes; every other
+ *    bf16 / FP8 / output pointer 16 bytes; scale and index pointers 4 bytes.
  *  - Non-finite inputs are outside the contract (results unspecified, no fault).
  *  - Every on-device wait is bounded (default 4 s, see fp8q_set_wait_timeout_ns);
  *    a wait that runs out records FP8Q_ERR_TIMEOUT in a device status word,

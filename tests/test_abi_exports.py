@@ -52,7 +52,8 @@ def test_status_strings():
     assert fq.status_string(99) == "unknown status"
 
 
-A16 = 0x10000  # a 16-byte aligned fake address; never dereferenced
+A16 = 0x10000  # a 256-byte aligned fake address; never dereferenced
+A16_ONLY = 0x10010  # 16-byte but not 32-byte aligned
 A4 = 0x10004   # 4-byte aligned only
 A1 = 0x10001
 
@@ -69,6 +70,7 @@ def _call(name, *args):
     ((None, 4, 128, A16, A16, None), fq.ERR_NULL),
     ((A16, 4, 128, None, A16, None), fq.ERR_NULL),
     ((A4, 4, 128, A16, A16, None), fq.ERR_ALIGN),
+    ((A16_ONLY, 4, 128, A16, A16, None), fq.ERR_ALIGN),  # bf16 input: 32 bytes
     ((A16, 4, 128, A4, A16, None), fq.ERR_ALIGN),
     ((A16, 4, 128, A16, A1, None), fq.ERR_ALIGN),
 ])
@@ -82,6 +84,7 @@ def test_quant_act_validation(args, expect):
     ((A16, 0, 128, 128, A16, A16, None), fq.OK),
     ((None, 1, 128, 128, A16, A16, None), fq.ERR_NULL),
     ((A16, 2, 128, 128, A16, A1, None), fq.ERR_ALIGN),
+    ((A16_ONLY, 1, 128, 128, A16, A16, None), fq.ERR_ALIGN),  # bf16 input: 32 bytes
 ])
 def test_quant_w_validation(args, expect):
     assert _call("fp8_quant_w_128x128", *args) == expect

@@ -185,3 +185,42 @@ def test_quotients_near_e4m3_midpoints(dev):
     rows = (x.shape[0] // 128) * 128
     if rows:
         assert_w_exact(np.ascontiguousarray(bits[:rows]), dev)
+
+
+def _tiles_with_every_amax(stride=1, seed=7):
+    """One 128-element group per finite non-negative bf16 value a (every
+    `stride`-th one): element 0 is a, the rest are random values of magnitude
+    at most a, either sign.  Returns the bf16 bits, [groups, 128]."""
+    amax_bits = np.arange(0, 0x7F80, stride, dtype=np.uint32)
+    a = (amax_bits << 16).view(np.float32)
+    rng = np.random.default_rng(seed)
+    u = rng.random((a.size, TILE), dtype=np.float32)
+    sign = np.where(rng.random((a.size, TILE)) < 0.5, -1.0, 1.0).astype(np.float32)
+    x = wl.bf16_bits(a[:, None] * u * sign)
+    x[:, 0] = amax_bits.astype(np.uint16)
+    return x
+
+
+def test_every_bf16_amax_act(dev):
+    """All 32640 finite non-negative bf16 amax values, one tile each: the
+    division-free scale and the codes must equal the oracle's IEEE results."""
+    x = _tiles_with_every_amax()
+    assert x.shape[0] == 255 * 128
+    assert_act_exact(x.reshape(255, 128 * TILE), dev)
+
+
+def test_every_16th_bf16_amax_w(dev):
+    """Every 16th bf16 amax value, one 128x128 weight block each."""
+    groups = _tiles_with_every_amax(stride=16, seed=8)   # 2040 groups of 128
+    nb = groups.shape[0]
+    rng = np.random.default_rng(9)
+    blocks = np.empty((nb, TILE, TILE), dtype=np.uint16)
+    # each block: the group as its first row, the other rows a shuffled copy
+    # scaled down by a power of two (exact in bf16 unless it underflows)
+    f = wl.bf16_to_f32(groups)
+    for i in range(nb):
+        rows = np.stack([rng.permutation(f[i]) for _ in range(TILE - 1)]) * np.float32(0.5)
+        blocks[i, 0] = groups[i]
+        blocks[i, 1:] = wl.bf16_bits(rows)
+    w = blocks.reshape(nb * TILE, TILE)   # G = 1, N = 128 * nb, K = 128
+    assert_w_exact(w, dev)
