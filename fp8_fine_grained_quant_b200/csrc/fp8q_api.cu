@@ -14,9 +14,6 @@
 #include "fp8q.h"
 #include "fp8q_gemm.cuh"
 #include "fp8q_ptx.cuh"
-#ifndef FP8Q_ACT_UNROLL
-#define FP8Q_ACT_UNROLL 2
-#endif
 #include "fp8q_quant.cuh"
 
 namespace fp8q {
@@ -222,7 +219,7 @@ int fp8_quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, fl
   int rc = device_info(&dev);
   if (rc) return rc;
   const int64_t tiles = M * (K / 128);
-  constexpr int kUnroll = FP8Q_ACT_UNROLL;
+  constexpr int kUnroll = 2;  // tiles per lane group in flight (64 bytes of loads per lane)
   const int64_t per_cta = (256 / 8) * kUnroll;
   int64_t grid = (tiles + per_cta - 1) / per_cta;
   const int64_t cap = static_cast<int64_t>(dev->num_sms) * 8;
