@@ -39,10 +39,10 @@ std::mutex g_dev_mu;
 
 // Per-device set-up, done once: SM count, arch check, status-word address,
 // and the dynamic shared-memory opt-in of every GEMM instantiation.
-template <int BN, int STAGES, Sched S>
+template <int BN, int STAGES, Sched S, bool kPromote>
 cudaError_t opt_in_smem() {
-  return cudaFuncSetAttribute(gemm_blockscaled_kernel<BN, STAGES, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              GemmSmem<BN, STAGES>::kDynamicBytes);
+  return cudaFuncSetAttribute(gemm_blockscaled_kernel<BN, STAGES, S, kPromote>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, GemmSmem<BN, STAGES>::kDynamicBytes);
 }
 
 // Output tile 128 x kTileN: 64 FP32 accumulators per epilogue thread, four
@@ -68,9 +68,10 @@ int device_info(DeviceInfo** out) {
         if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_device_status) != cudaSuccess)
           return FP8Q_ERR_CUDA;
         cudaError_t e = cudaSuccess;
-        if (e == cudaSuccess) e = opt_in_smem<128, kStages128, Sched::kDense>();
-        if (e == cudaSuccess) e = opt_in_smem<128, kStages128, Sched::kContiguous>();
-        if (e == cudaSuccess) e = opt_in_smem<128, kStages128, Sched::kMasked>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kDense, true>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kDense, false>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kContiguous, true>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kMasked, true>();
         if (e != cudaSuccess) return FP8Q_ERR_CUDA;
       }
       d.ready = true;
@@ -132,7 +133,7 @@ struct GemmCall {
   int promote;
 };
 
-template <int BN, int STAGES, Sched S>
+template <int BN, int STAGES, Sched S, bool kPromote>
 int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
   CUtensorMap ma, mb;
   int rc = make_operand_map(&ma, g.qa, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K), kBlockM);
@@ -153,7 +154,6 @@ int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
   a.E = static_cast<int32_t>(g.E);
   a.m_tiles = static_cast<int32_t>(g.m_tiles);
   a.n_tiles = static_cast<int32_t>((g.N + BN - 1) / BN);
-  a.promote = g.promote;
   int64_t max_tiles = g.m_tiles * a.n_tiles * (S == Sched::kMasked ? g.E : 1);
   const int grid = static_cast<int>(max_tiles < dev.num_sms ? max_tiles : dev.num_sms);
   if (grid <= 0) return FP8Q_OK;
@@ -163,7 +163,7 @@ int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = GemmSmem<BN, STAGES>::kDynamicBytes;
   cfg.stream = stream;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<BN, STAGES, S>, ma, mb, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<BN, STAGES, S, kPromote>, ma, mb, a);
   if (e != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FP8Q_OK;
@@ -174,7 +174,10 @@ int run_gemm(const GemmCall& g, cudaStream_t stream) {
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);
   if (rc) return rc;
-  return launch_gemm<kTileN, kStages128, S>(g, *dev, stream);
+  if (g.promote) return launch_gemm<kTileN, kStages128, S, true>(g, *dev, stream);
+  // only the dense form has the unpromoted (accumulation diagnostic) build
+  if constexpr (S == Sched::kDense) return launch_gemm<kTileN, kStages128, S, false>(g, *dev, stream);
+  return FP8Q_ERR_UNSUPPORTED;
 }
 
 int check_operands(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, const void* c) {

@@ -58,7 +58,6 @@ struct GemmArgs {
   int32_t E;
   int32_t m_tiles;           // dense: ceil(M/128); contiguous: M_tot/128; masked: cap/128
   int32_t n_tiles;           // ceil(N / BN)
-  int32_t promote;           // 1: per-slab promotion; 0: accumulate all of K in TMEM (diagnostic)
 };
 
 struct Tile {
@@ -235,13 +234,13 @@ __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensor
 // slab starts a fresh accumulator in its own TMEM buffer, so slabs are
 // independent and two issuers take alternate slabs.  Without promotion a tile
 // accumulates in one buffer and one issuer (n = 1) does all of it.
-template <int BN, int STAGES, Sched S>
+template <int BN, int STAGES, Sched S, bool kPromote>
 __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* prefix, uint32_t s_base,
                                           Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
                                           int32_t total, uint32_t tmem_base, uint32_t who, uint32_t n) {
   using L = GemmSmem<BN, STAGES>;
   constexpr uint32_t kIdesc = idesc_e4m3_f32(kBlockM, BN);
-  const bool promote = args.promote != 0;
+  constexpr bool promote = kPromote;
   const uint32_t mask = n - 1;  // n is 1 or 2
   int stage = 0, buf = 0;
   uint32_t phase = 0, tphase = 0, j = 0;
@@ -293,7 +292,7 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
 // back as soon as the values are in registers, then applies
 // acc += (sa * sb) * partial.  The completion probe of the next slab is issued
 // before this slab's work and read after it.
-template <int BN, int STAGES, Sched S>
+template <int BN, int STAGES, Sched S, bool kPromote>
 __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* prefix,
                                          Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
                                          int32_t total, uint32_t tmem_base, int warp, int lane) {
@@ -304,7 +303,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
   constexpr int kAcc = L::kAccBufs;
   static_assert(kCols <= 128 && 128 % kCols == 0 && kGroup % 32 == 0, "each half must sit in one scale block");
   static_assert(kAcc < STAGES, "buffer releases are posted on the stage barrier of a later slab");
-  const bool promote = args.promote != 0;
+  constexpr bool promote = kPromote;
   const int quad = warp & 3;
   const int half = (warp - 4) >> 2;
   const int r = quad * 32 + lane;
@@ -327,15 +326,16 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
     for (int i = 0; i < kCols / 2; ++i) acc[i] = 0ull;
 
     const int n_reads = promote ? nkb : 1;
-    // the next slab's scales are fetched one slab ahead
-    float sa_next = row_ok ? __ldg(sa_row) : 0.0f;
-    float sb_next = col_ok ? __ldg(sb_row) : 0.0f;
+    // the next slab's scales are fetched one slab ahead (rows past the valid
+    // ones read row 0's scales: their sums are never stored)
+    float sa_next = __ldg(sa_row);
+    float sb_next = __ldg(sb_row);
     bool ok = true;
     for (int it = 0; it < n_reads; ++it) {
       const uint64_t scale2 = pack_f32x2(sa_next * sb_next);
       if (it + 1 < n_reads) {
-        sa_next = row_ok ? __ldg(sa_row + it + 1) : 0.0f;
-        sb_next = col_ok ? __ldg(sb_row + it + 1) : 0.0f;
+        sa_next = __ldg(sa_row + it + 1);
+        sb_next = __ldg(sb_row + it + 1);
       }
       // Warp-uniform outcome: the tcgen05.ld below must be executed by all 32 lanes.
       if (!ready) {
@@ -400,7 +400,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
 }
 
 // ----------------------------------------------------------------- kernel
-template <int BN, int STAGES, Sched S>
+template <int BN, int STAGES, Sched S, bool kPromote>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                             const GemmArgs args) {
@@ -418,7 +418,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl wc{args.timeout_ns, args.status, abort_flag};
-  const bool promote = args.promote != 0;
+  constexpr bool promote = kPromote;
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < STAGES; ++st) {
@@ -463,13 +463,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (warp == 0 || warp == 3)
         produce<BN, STAGES, S>(&tma_a, &tma_b, args, prefix, s_base, bars, wc, total, warp == 0 ? 0u : 1u);
       else if (static_cast<uint32_t>(warp - 1) < n_mma)
-        issue_mma<BN, STAGES, S>(args, prefix, s_base, bars, wc, total, tmem_base, warp - 1, n_mma);
+        issue_mma<BN, STAGES, S, kPromote>(args, prefix, s_base, bars, wc, total, tmem_base, warp - 1, n_mma);
     }
   } else {
     // all TMEM slab buffers start free: release them for the first slabs
     if (promote && lane == 0)
       for (int b = 0; b < L::kAccBufs; ++b) mbar_arrive(bars.full(b));
-    epilogue<BN, STAGES, S>(args, prefix, bars, wc, total, tmem_base, warp, lane);
+    epilogue<BN, STAGES, S, kPromote>(args, prefix, bars, wc, total, tmem_base, warp, lane);
   }
 
   __syncwarp();
