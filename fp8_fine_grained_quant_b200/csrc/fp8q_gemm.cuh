@@ -162,7 +162,8 @@ __device__ __forceinline__ bool get_tile(const GemmArgs& a, const int32_t* prefi
 //              promotion, TMEM buffer j % kAccBufs is free again: the eight
 //              epilogue warps arrive once they have read slab j - kAccBufs out
 //              of it (for the first kAccBufs slabs they arrive up front).
-//              Arrivals: 1 (producer) + 8 (epilogue) with promotion, else 1.
+//              Arrivals: 1 (producer) + 256 (every epilogue lane, once its
+//              own TMEM loads are complete) with promotion, else 1.
 //   empty[s] : the four MMAs of slab j have completed (one tcgen05.commit):
 //              stage s may be refilled (producer, for slab j + STAGES) and,
 //              with promotion, the partial in buffer j % kAccBufs is final
@@ -359,15 +360,13 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
         if (g == kGroups - 1) {
           // buffer free: with promotion it serves slab j + kAcc, whose stage barrier takes the arrival
           tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            if (promote) {
-              int rs = stage + kAcc;
-              if (rs >= STAGES) rs -= STAGES;
-              mbar_arrive(bars.full(rs));
-            } else {
-              mbar_arrive(bars.tempty(buf));
-            }
+          if (promote) {
+            int rs = stage + kAcc;
+            if (rs >= STAGES) rs -= STAGES;
+            mbar_arrive(bars.full(rs));
+          } else {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.tempty(buf));
           }
         }
 #pragma unroll
@@ -422,7 +421,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < STAGES; ++st) {
-      mbar_init(bars.full(st), promote ? 1 + 8 : 1);  // producer (+ the eight epilogue warps)
+      mbar_init(bars.full(st), promote ? 1 + 8 * 32 : 1);  // producer (+ every lane of the eight epilogue warps)
       mbar_init(bars.empty(st), 1);
     }
     for (int b = 0; b < L::kAccBufs; ++b) {
@@ -466,8 +465,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         issue_mma<BN, STAGES, S, kPromote>(args, prefix, s_base, bars, wc, total, tmem_base, warp - 1, n_mma);
     }
   } else {
-    // all TMEM slab buffers start free: release them for the first slabs
-    if (promote && lane == 0)
+    // all TMEM slab buffers start free: every lane releases them for the first slabs
+    if (promote)
       for (int b = 0; b < L::kAccBufs; ++b) mbar_arrive(bars.full(b));
     epilogue<BN, STAGES, S, kPromote>(args, prefix, bars, wc, total, tmem_base, warp, lane);
   }
