@@ -117,10 +117,10 @@ __device__ __forceinline__ void zero8(uint32_t (&w)[8]) {
 // lanes (32 bytes each) own one tile per step, so a warp covers four tiles.
 // Tile t = m * (K/128) + kb, which is also the index of its scale in
 // s[M, K/128].  Each lane group handles kUnroll tiles per iteration (loads
-// issued together) in a grid-stride loop.
+// issued together) in a grid-stride loop; five CTAs fit per SM.
 // ---------------------------------------------------------------------------
 template <int kUnroll>
-__global__ void __launch_bounds__(256) quant_act_1x128_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
+__global__ void __launch_bounds__(256, 5) quant_act_1x128_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
                                                               float* __restrict__ s, int64_t num_tiles) {
   const int sub = threadIdx.x & 7;
   const int64_t grp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 3;
