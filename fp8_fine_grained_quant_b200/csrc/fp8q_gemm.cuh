@@ -333,11 +333,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
     float sb_next = __ldg(sb_row);
     bool ok = true;
     for (int it = 0; it < n_reads; ++it) {
-      const uint64_t scale2 = pack_f32x2(sa_next * sb_next);
-      if (it + 1 < n_reads) {
-        sa_next = __ldg(sa_row + it + 1);
-        sb_next = __ldg(sb_row + it + 1);
-      }
+      uint64_t scale2;
       // Warp-uniform outcome: the tcgen05.ld below must be executed by all 32 lanes.
       if (!ready) {
         const bool got = promote ? mbar_wait(bars.empty(stage), phase, wc, 4) : mbar_wait(bars.tfull(buf), tphase, wc, 4);
@@ -367,6 +363,17 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
           } else {
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.tempty(buf));
+          }
+        }
+        if (g == 0) {
+          // The slab's scales are consumed here, after its TMEM load and
+          // buffer release, and the next slab's are requested right after:
+          // each load has a whole slab to arrive, and no buffer release (a
+          // release-ordered arrival) waits behind an outstanding load.
+          scale2 = pack_f32x2(sa_next * sb_next);
+          if (it + 1 < n_reads) {
+            sa_next = __ldg(sa_row + it + 1);
+            sb_next = __ldg(sb_row + it + 1);
           }
         }
 #pragma unroll
