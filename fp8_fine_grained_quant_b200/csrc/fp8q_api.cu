@@ -39,9 +39,9 @@ std::mutex g_dev_mu;
 
 // Per-device set-up, done once: SM count, arch check, status-word address,
 // and the dynamic shared-memory opt-in of every GEMM instantiation.
-template <int BN, int STAGES, Sched S, bool kPromote>
+template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales>
 cudaError_t opt_in_smem() {
-  return cudaFuncSetAttribute(gemm_blockscaled_kernel<BN, STAGES, S, kPromote>,
+  return cudaFuncSetAttribute(gemm_blockscaled_kernel<BN, STAGES, S, kPromote, kTmaScales>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, GemmSmem<BN, STAGES>::kDynamicBytes);
 }
 
@@ -68,10 +68,13 @@ int device_info(DeviceInfo** out) {
         if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_device_status) != cudaSuccess)
           return FP8Q_ERR_CUDA;
         cudaError_t e = cudaSuccess;
-        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kDense, true>();
-        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kDense, false>();
-        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kContiguous, true>();
-        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kMasked, true>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kDense, true, true>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kDense, true, false>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kDense, false, false>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kContiguous, true, true>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kContiguous, true, false>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kMasked, true, true>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kMasked, true, false>();
         if (e != cudaSuccess) return FP8Q_ERR_CUDA;
       }
       d.ready = true;
@@ -116,6 +119,22 @@ int make_operand_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
+// Scale tensor [rows, nkb] f32 as a 2-D map with a box of 4 slabs x box_rows
+// rows (the GEMM stages a group of 4 slabs' scales at once).  Needs nkb % 4 ==
+// 0 and a 16-byte-aligned base; rows past the end read as zero.
+int make_scale_map(CUtensorMap* map, const float* base, uint64_t rows, uint64_t nkb, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FP8Q_ERR_CUDA;
+  const cuuint64_t dims[2] = {nkb, rows};
+  const cuuint64_t strides[1] = {nkb * 4};
+  const cuuint32_t box[2] = {4, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- GEMM launch
 struct GemmCall {
   const uint8_t* qa;
@@ -133,13 +152,22 @@ struct GemmCall {
   int promote;
 };
 
-template <int BN, int STAGES, Sched S, bool kPromote>
+template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales>
 int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, msa, msb;
+  std::memset(&msa, 0, sizeof msa);
+  std::memset(&msb, 0, sizeof msb);
   int rc = make_operand_map(&ma, g.qa, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K), kBlockM);
   if (rc) return rc;
   rc = make_operand_map(&mb, g.qb, static_cast<uint64_t>(g.E * g.N), static_cast<uint64_t>(g.K), BN);
   if (rc) return rc;
+  if constexpr (kTmaScales) {
+    const uint64_t nkb = static_cast<uint64_t>(g.K / kSlabK);
+    rc = make_scale_map(&msa, g.sa, static_cast<uint64_t>(g.a_rows), nkb, kBlockM);
+    if (rc) return rc;
+    rc = make_scale_map(&msb, g.sb, static_cast<uint64_t>(g.E * (g.N / 128)), nkb, 1);
+    if (rc) return rc;
+  }
   GemmArgs a;
   a.sa = g.sa;
   a.sb = g.sb;
@@ -163,7 +191,8 @@ int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = GemmSmem<BN, STAGES>::kDynamicBytes;
   cfg.stream = stream;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<BN, STAGES, S, kPromote>, ma, mb, a);
+  cudaError_t e =
+      cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<BN, STAGES, S, kPromote, kTmaScales>, ma, mb, msa, msb, a);
   if (e != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FP8Q_OK;
@@ -174,9 +203,15 @@ int run_gemm(const GemmCall& g, cudaStream_t stream) {
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);
   if (rc) return rc;
-  if (g.promote) return launch_gemm<kTileN, kStages128, S, true>(g, *dev, stream);
+  if (g.promote) {
+    // scales staged by TMA with the operands when their rows are 16-byte
+    // multiples (K % 512 == 0) and both scale tensors are 16-byte aligned
+    if ((g.K / kSlabK) % 4 == 0 && aligned(g.sa, 16) && aligned(g.sb, 16))
+      return launch_gemm<kTileN, kStages128, S, true, true>(g, *dev, stream);
+    return launch_gemm<kTileN, kStages128, S, true, false>(g, *dev, stream);
+  }
   // only the dense form has the unpromoted (accumulation diagnostic) build
-  if constexpr (S == Sched::kDense) return launch_gemm<kTileN, kStages128, S, false>(g, *dev, stream);
+  if constexpr (S == Sched::kDense) return launch_gemm<kTileN, kStages128, S, false, false>(g, *dev, stream);
   return FP8Q_ERR_UNSUPPORTED;
 }
 

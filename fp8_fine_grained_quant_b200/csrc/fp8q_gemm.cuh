@@ -83,7 +83,17 @@ struct GemmSmem {
   static constexpr uint32_t kNumBars = 2 * STAGES + 2 * kAccBufs + 2;
   static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;     // tmem slot, abort flag, total tiles
   static constexpr uint32_t kOffPrefix = (kOffMisc + 16 + 15) / 16 * 16;
-  static constexpr uint32_t kBytes = kOffPrefix + 4 * (kMaxMaskedExperts + 1);
+  // Scale ring (TMA-staged scales): per group of kScaleGroup slabs, the 128
+  // tile rows' activation scales as a [128][kScaleGroup] f32 box and the
+  // weight block's kScaleGroup scales.
+  static constexpr int kScaleGroup = 4;
+  static constexpr int kScaleSlots = 4;
+  static constexpr uint32_t kSaSlotBytes = kBlockM * kScaleGroup * 4;  // 2 KB
+  static constexpr uint32_t kSbSlotBytes = kScaleGroup * 4;             // 16 B
+  static constexpr uint32_t kSbSlotStride = 128;                        // TMA destinations 128-byte aligned
+  static constexpr uint32_t kOffSa = (kOffPrefix + 4 * (kMaxMaskedExperts + 1) + 127) / 128 * 128;
+  static constexpr uint32_t kOffSb = kOffSa + kScaleSlots * kSaSlotBytes;
+  static constexpr uint32_t kBytes = kOffSb + kScaleSlots * kSbSlotStride;
   static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
@@ -176,6 +186,14 @@ __device__ __forceinline__ bool get_tile(const GemmArgs& a, const int32_t* prefi
 // observed empty[s] for slab j, and the producer observes empty[s] for slab j
 // before it loads slab j + STAGES.
 //
+// TMA-staged scales: the scales of slabs 4g..4g+3 of a tile (group g) arrive
+// with slab 4g's stage (same full[] barrier) in scale slot g % 4.  The slot is
+// rewritten for group g + 4, by the producer of slab 4g + 16, only after
+// empty[] of slab 4g + 10, which needs the epilogue's releases of slab 4g + 6:
+// by then every epilogue warp has read the scales of slabs <= 4g + 5.  The
+// epilogue reads a slab's scales after observing that slab's MMAs complete,
+// and those MMAs were issued after full[] of slab 4g (the copies landed).
+//
 // Each waiting role costs its thread ~150 cycles per barrier probe, and an MMA
 // instruction is accepted only as the tensor pipe frees up, so the TMA and MMA
 // roles are split over two threads each (slabs alternate between them) and
@@ -192,28 +210,41 @@ struct Bars {
 };
 
 // TMA producer `who` of two: loads the slabs j with j % 2 == who.
-template <int BN, int STAGES, Sched S>
-__device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensorMap* tma_b, const GemmArgs& args,
+template <int BN, int STAGES, Sched S, bool kTmaScales>
+__device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensorMap* tma_b,
+                                        const CUtensorMap* tma_sa, const CUtensorMap* tma_sb, const GemmArgs& args,
                                         const int32_t* prefix, uint32_t s_base,
                                         Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
                                         int32_t total, uint32_t who) {
   using L = GemmSmem<BN, STAGES>;
+  const int nnb = args.N / 128;
   int stage = 0;
   uint32_t phase = 0, j = 0;
+  uint32_t group = 0;  // scale groups so far (kTmaScales)
   uint32_t armed = 0, armed_parity = 0;  // per stage: ever armed / parity of its last phase
   bool ok = true;
   for (int32_t t = blockIdx.x; ok && t < total && !*wc.abort; t += gridDim.x) {
     Tile tile;
     if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
     for (int kb = 0; kb < args.nkb; ++kb, ++j) {
+      const bool group_start = kTmaScales && (kb % L::kScaleGroup) == 0;
       if ((j & 1u) == who) {
         if (!mbar_wait(bars.empty(stage), phase ^ 1u, wc, 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(bars.full(stage), L::kStageBytes);
+        mbar_arrive_expect_tx(bars.full(stage),
+                              L::kStageBytes + (group_start ? L::kSaSlotBytes + L::kSbSlotBytes : 0u));
         tma_load_2d(s_base + L::kOffA + stage * L::kABytes, tma_a, bars.full(stage), kb * kSlabK, tile.a_row);
         tma_load_2d(s_base + L::kOffB + stage * L::kBBytes, tma_b, bars.full(stage), kb * kSlabK, tile.b_row);
+        if (group_start) {
+          // x = kb is a multiple of 4 f32: a 16-byte-aligned start
+          const uint32_t slot = group % L::kScaleSlots;
+          tma_load_2d(s_base + L::kOffSa + slot * L::kSaSlotBytes, tma_sa, bars.full(stage), kb, tile.a_row);
+          tma_load_2d(s_base + L::kOffSb + slot * L::kSbSlotStride, tma_sb, bars.full(stage), kb,
+                      tile.e * nnb + tile.n0 / 128);
+        }
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
       }
+      if (group_start) ++group;
       if (++stage == STAGES) {
         stage = 0;
         phase ^= 1u;
@@ -293,8 +324,8 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
 // back as soon as the values are in registers, then applies
 // acc += (sa * sb) * partial.  The completion probe of the next slab is issued
 // before this slab's work and read after it.
-template <int BN, int STAGES, Sched S, bool kPromote>
-__device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* prefix,
+template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales>
+__device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, const int32_t* prefix,
                                          Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
                                          int32_t total, uint32_t tmem_base, int warp, int lane) {
   using L = GemmSmem<BN, STAGES>;
@@ -304,6 +335,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
   constexpr int kAcc = L::kAccBufs;
   static_assert(kCols <= 128 && 128 % kCols == 0 && kGroup % 32 == 0, "each half must sit in one scale block");
   static_assert(kAcc < STAGES, "buffer releases are posted on the stage barrier of a later slab");
+  static_assert(kPromote || !kTmaScales, "staged scales serve the per-slab promotion only");
   constexpr bool promote = kPromote;
   const int quad = warp & 3;
   const int half = (warp - 4) >> 2;
@@ -314,6 +346,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
   int buf = 0, stage = 0;
   uint32_t tphase = 0, phase = 0;
   bool ready = false;  // the current slab (or tile, without promotion) is known complete
+  uint32_t group = 0;  // scale groups so far (kTmaScales)
   for (int32_t t = blockIdx.x; t < total && !*wc.abort; t += gridDim.x) {
     Tile tile;
     if (!get_tile<S, BN>(args, prefix, t, tile)) continue;
@@ -329,8 +362,8 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
     const int n_reads = promote ? nkb : 1;
     // the next slab's scales are fetched one slab ahead (rows past the valid
     // ones read row 0's scales: their sums are never stored)
-    float sa_next = __ldg(sa_row);
-    float sb_next = __ldg(sb_row);
+    float sa_next = kTmaScales ? 0.0f : __ldg(sa_row);
+    float sb_next = kTmaScales ? 0.0f : __ldg(sb_row);
     bool ok = true;
     for (int it = 0; it < n_reads; ++it) {
       uint64_t scale2;
@@ -338,6 +371,15 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
       if (!ready) {
         const bool got = promote ? mbar_wait(bars.empty(stage), phase, wc, 4) : mbar_wait(bars.tfull(buf), tphase, wc, 4);
         if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
+      }
+      float sa_smem = 0.0f, sb_smem = 0.0f;
+      if constexpr (kTmaScales) {
+        // this slab's scales, staged with its group's first stage
+        const uint32_t slot = group % L::kScaleSlots;
+        const uint32_t k = static_cast<uint32_t>(it % L::kScaleGroup);
+        sa_smem = lds_f32(s_base + L::kOffSa + slot * L::kSaSlotBytes + r * (L::kScaleGroup * 4) + k * 4);
+        sb_smem = lds_f32(s_base + L::kOffSb + slot * L::kSbSlotStride + k * 4);
+        if (k == L::kScaleGroup - 1) ++group;
       }
       tc_fence_after();
       const uint32_t t_buf = t_lane + buf * L::kTmemStride + half * kCols;
@@ -366,14 +408,18 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
           }
         }
         if (g == 0) {
-          // The slab's scales are consumed here, after its TMEM load and
-          // buffer release, and the next slab's are requested right after:
-          // each load has a whole slab to arrive, and no buffer release (a
-          // release-ordered arrival) waits behind an outstanding load.
-          scale2 = pack_f32x2(sa_next * sb_next);
-          if (it + 1 < n_reads) {
-            sa_next = __ldg(sa_row + it + 1);
-            sb_next = __ldg(sb_row + it + 1);
+          if constexpr (kTmaScales) {
+            scale2 = pack_f32x2(sa_smem * sb_smem);
+          } else {
+            // The slab's scales are consumed here, after its TMEM load and
+            // buffer release, and the next slab's are requested right after:
+            // each load has a whole slab to arrive, and no buffer release (a
+            // release-ordered arrival) waits behind an outstanding load.
+            scale2 = pack_f32x2(sa_next * sb_next);
+            if (it + 1 < n_reads) {
+              sa_next = __ldg(sa_row + it + 1);
+              sb_next = __ldg(sb_row + it + 1);
+            }
           }
         }
 #pragma unroll
@@ -406,9 +452,10 @@ __device__ __forceinline__ void epilogue(const GemmArgs& args, const int32_t* pr
 }
 
 // ----------------------------------------------------------------- kernel
-template <int BN, int STAGES, Sched S, bool kPromote>
+template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                            const __grid_constant__ CUtensorMap tma_sa, const __grid_constant__ CUtensorMap tma_sb,
                             const GemmArgs args) {
   using L = GemmSmem<BN, STAGES>;
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "UMMA N for M=128 must be a multiple of 16 in [16,256]");
@@ -441,6 +488,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_barrier_init();
     tma_prefetch_map(&tma_a);
     tma_prefetch_map(&tma_b);
+    if constexpr (kTmaScales) {
+      tma_prefetch_map(&tma_sa);
+      tma_prefetch_map(&tma_sb);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
@@ -467,7 +518,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t n_mma = promote ? 2u : 1u;
     if (lane == 0) {
       if (warp == 0 || warp == 3)
-        produce<BN, STAGES, S>(&tma_a, &tma_b, args, prefix, s_base, bars, wc, total, warp == 0 ? 0u : 1u);
+        produce<BN, STAGES, S, kTmaScales>(&tma_a, &tma_b, &tma_sa, &tma_sb, args, prefix, s_base, bars, wc, total,
+                                           warp == 0 ? 0u : 1u);
       else if (static_cast<uint32_t>(warp - 1) < n_mma)
         issue_mma<BN, STAGES, S, kPromote>(args, prefix, s_base, bars, wc, total, tmem_base, warp - 1, n_mma);
     }
@@ -475,7 +527,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // all TMEM slab buffers start free: every lane releases them for the first slabs
     if (promote)
       for (int b = 0; b < L::kAccBufs; ++b) mbar_arrive(bars.full(b));
-    epilogue<BN, STAGES, S, kPromote>(args, prefix, bars, wc, total, tmem_base, warp, lane);
+    epilogue<BN, STAGES, S, kPromote, kTmaScales>(s_base, args, prefix, bars, wc, total, tmem_base, warp, lane);
   }
 
   __syncwarp();

@@ -65,6 +65,31 @@ def test_dense_small_full(dev, M, N, K):
     assert_gemm_close(bf16_bits_of(c), ref, "dense %dx%dx%d" % (M, N, K))
 
 
+def _misaligned_copy(t):
+    """Same values, at an address 4 bytes past a 16-byte boundary."""
+    buf = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+    view = buf[1:].view(t.shape)
+    view.copy_(t)
+    assert view.data_ptr() % 16 == 4
+    return view
+
+
+@pytest.mark.parametrize("M,N,K", [(257, 512, 1024), (128, 384, 2048)])
+def test_scale_staging_paths_agree(dev, M, N, K):
+    """K % 512 == 0 with 16-byte-aligned scales stages the scales through
+    shared memory with the operands; unaligned scales take the global-load
+    path.  Both must give the same bits (and match the oracle)."""
+    rng = np.random.default_rng(M + N + K)
+    a = rng.standard_normal((M, K)).astype(np.float32) * np.exp(rng.standard_normal(K)).astype(np.float32)
+    b = (0.02 * rng.standard_normal((N, K))).astype(np.float32)
+    (qa, sa, qb, sb), (oqa, osa, oqb, osb) = _quantize_both(wl.bf16_bits(a), wl.bf16_bits(b), dev)
+    staged = fq.fp8_gemm_blockscaled(qa, sa, qb, sb)
+    loaded = fq.fp8_gemm_blockscaled(qa, _misaligned_copy(sa), qb, _misaligned_copy(sb))
+    _finish(dev)
+    assert torch.equal(staged.view(torch.int16), loaded.view(torch.int16))
+    assert_gemm_close(bf16_bits_of(staged), oracle.gemm_blockscaled(oqa, osa, oqb, osb), "staged %dx%dx%d" % (M, N, K))
+
+
 def test_tiny_dense_workload(dev):
     d = wl.tiny_dense()
     (qa, sa, qb, sb), (oqa, osa, oqb, osb) = _quantize_both(d.a, d.b, dev)
