@@ -260,7 +260,7 @@ int fp8_quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, fl
   constexpr int kUnroll = 2;  // tiles per lane group in flight (64 bytes of loads per lane)
   const int64_t per_cta = (256 / 8) * kUnroll;
   int64_t grid = (tiles + per_cta - 1) / per_cta;
-  const int64_t cap = static_cast<int64_t>(dev->num_sms) * 8;
+  const int64_t cap = static_cast<int64_t>(dev->num_sms) * 10;  // two full waves of 5 resident CTAs per SM
   if (grid > cap) grid = cap;
   quant_act_1x128_kernel<kUnroll><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
       static_cast<const uint8_t*>(x_bf16), q, s, tiles);
