@@ -157,10 +157,11 @@ __global__ void __launch_bounds__(256, 5) quant_act_1x128_kernel(const uint8_t* 
 // 128x128 weight blocks.  One 256-thread CTA per block: eight lanes cover one
 // 256-byte row segment, 32 rows per pass, 4 passes; the block (32 KB) stays in
 // registers between the amax reduction and the quantization, so it is read
-// from HBM once.  Block b = (g * N/128 + nb) * K/128 + kb, also the index of
+// from HBM once (four CTAs per SM; the compiler keeps a few words of it in
+// local memory).  Block b = (g * N/128 + nb) * K/128 + kb, also the index of
 // its scale in s[G, N/128, K/128].  Grid-stride over blocks.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256, 3) quant_w_128x128_kernel(const uint8_t* __restrict__ w,
+__global__ void __launch_bounds__(256, 4) quant_w_128x128_kernel(const uint8_t* __restrict__ w,
                                                                  uint8_t* __restrict__ q, float* __restrict__ s,
                                                                  int64_t K, int64_t num_blocks) {
   __shared__ float warp_max[2][8];  // alternate halves: one CTA barrier per block
