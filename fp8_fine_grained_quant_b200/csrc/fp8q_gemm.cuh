@@ -14,7 +14,9 @@
 //   * persistent CTAs, one per SM, walking a static tile sequence;
 //   * warps 0 and 3: TMA producers for alternate slabs (one 128-deep K slab
 //     of A [128 x 128 B] and B [BN x 128 B] per pipeline stage, 128-byte
-//     swizzle, mbarrier tx count);
+//     swizzle, mbarrier tx count); when the scale rows allow it (K % 512 ==
+//     0, 16-byte-aligned scale tensors) the scales of every 4 slabs come by
+//     TMA with the first of them, into a small shared ring;
 //   * warp 1 allocates TMEM; warps 1 and 2 issue tcgen05.mma.kind::f8f6f4
 //     (M = 128, N = BN, K = 32, four per slab) for alternate slabs into four
 //     TMEM slab buffers; the first MMA of every slab overwrites, so each
@@ -23,8 +25,11 @@
 //   * warps 4-11: epilogue; warp w reads TMEM lanes 32*(w%4)..+31 (the rows the
 //     hardware lets it access) and half of the BN columns, applies
 //     acc += (sa * sb) * partial with packed FP32 FMAs, releases the buffer,
-//     and after the last slab stores bf16.  The MMA of slab k+1 runs while
-//     slab k is being promoted.
+//     and after the last slab stores bf16.  The MMAs of slabs k+1..k+3 run
+//     while slab k is being promoted;
+//   * promotion is a compile-time parameter: the unpromoted build (all of K
+//     accumulated in TMEM, a diagnostic of accumulation precision) is a
+//     separate instance;
 //   * every mbarrier wait is bounded; a wait that runs out records a timeout
 //     in the device status word and all roles drain and return.
 #pragma once
