@@ -45,6 +45,9 @@ SUSTAINED_AFTER_S = 1.0
 
 
 # ---------------------------------------------------------------------------- helpers
+METRIC = "FP8 block-scaled GEMM TFLOPS (step = 1x128 act quant + 128x128 weight quant + GEMM)"
+
+
 def load_peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -323,10 +326,10 @@ def run_reference(args, name):
               "(%d x %d), GEMM of %d x %d outputs over K=%d" % (rows, nb, TILE * nb, d.a.shape[-1], rows, TILE * nb,
                                                                d.a.shape[-1]))
     line = {
-        "impl": "reference", "metric": "FP8 block-scaled GEMM TFLOPS", "value": value, "unit": "TFLOP/s",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": describe(name, d),
+        "config": dict(describe(name, d), parallelism="single"),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -450,7 +453,7 @@ def run_ours(args, name):
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(name, d)
     line = {
-        "metric": "FP8 block-scaled GEMM TFLOPS (step = 1x128 act quant + 128x128 weight quant + GEMM)",
+        "metric": METRIC,
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3", "data": "synthetic",
