@@ -99,6 +99,10 @@ FP8Q_API int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64
  *   qb : [N, K] E4M3, sb : [N/128, K/128] f32 (from fp8_quant_w_128x128, G = 1)
  *   c_bf16 : [M, N] bf16, written (every element).
  * K >= 128 and K, N multiples of 128; any M >= 0 (M == 0 or N == 0: no-op).
+ * Performance note (all three GEMM forms): when K is a multiple of 512 and
+ * sa, sb are 16-byte aligned, the scales travel to the SM with the operand
+ * tiles (TMA); otherwise each is fetched from global memory.  The results
+ * are bit-identical either way.
  */
 FP8Q_API int fp8_gemm_blockscaled(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, void* c_bf16,
                          int64_t M, int64_t N, int64_t K, cudaStream_t stream);
