@@ -355,6 +355,32 @@ def traffic_for(kernel: str, name: str):
     return None
 
 
+def gemm_roofline(plan, kernels, peaks, fp8_peak, bf16_peak, sustained, name):
+    """Roofline entry for the step's GEMM (the dominant kernel).  Its bound
+    follows from its arithmetic intensity against the ridge of the two
+    measured peaks: tensor-bound for the dense and contiguous shapes,
+    HBM-bound for the masked decode (few rows per expert, every active
+    expert's weights read once)."""
+    gemm_label, gemm_bytes, gemm_flops = [(l, b, f) for l, b, f in plan if f][0]
+    g = kernels[gemm_label]
+    intensity = gemm_flops / gemm_bytes
+    ridge = fp8_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    peak_note = "%s (%s bf16 %.1f TFLOP/s x %.0f fp8/bf16 nominal ratio)" % (
+        peaks["source"], "sustained" if sustained else "burst", bf16_peak, FP8_OVER_BF16)
+    if intensity >= ridge:
+        roofline = {"bound": "tensor", "kernel": gemm_label, "achieved": g["tflops"], "peak": fp8_peak,
+                    "unit": "TFLOP/s", "frac": g["tflops"] / fp8_peak, "peak_source": peak_note}
+    else:
+        roofline = {"bound": "hbm", "kernel": gemm_label, "achieved": g["gbs"], "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": g["gbs"] / peaks["hbm_gbs"],
+                    "peak_source": "%s copy bandwidth" % peaks["source"],
+                    "tensor_frac": g["tflops"] / fp8_peak, "tensor_peak_source": peak_note}
+    roofline.update(traffic=traffic_for(gemm_label, name), algorithmic_flops_per_launch=gemm_flops,
+                    algorithmic_bytes_per_launch=gemm_bytes, intensity_flop_per_byte=intensity,
+                    ridge_flop_per_byte=ridge)
+    return roofline
+
+
 def run_ours(args, name):
     import torch
     rank, world, local = dist_env()
@@ -427,27 +453,7 @@ def run_ours(args, name):
             ent.update(tflops=kflops / avg_ms / 1e9, frac_of_fp8_peak=kflops / avg_ms / 1e9 / fp8_peak)
         ent.update(gbs=nbytes / avg_ms / 1e6, frac_of_hbm=nbytes / avg_ms / 1e6 / peaks["hbm_gbs"])
         kernels[label] = ent
-    gemm_label, gemm_bytes_, gemm_flops_ = [(l, b, f) for l, b, f in plan if f][0]
-    g = kernels[gemm_label]
-    # dominant kernel: the GEMM.  Its bound follows from its arithmetic
-    # intensity against the ridge of the two measured peaks: tensor-bound for
-    # the dense and contiguous shapes, HBM-bound for the masked decode (few
-    # rows per expert, every active expert's weights read once).
-    intensity = gemm_flops_ / gemm_bytes_
-    ridge = fp8_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    peak_note = "%s (%s bf16 %.1f TFLOP/s x %.0f fp8/bf16 nominal ratio)" % (
-        peaks["source"], "sustained" if sustained else "burst", bf16_peak, FP8_OVER_BF16)
-    if intensity >= ridge:
-        roofline = {"bound": "tensor", "kernel": gemm_label, "achieved": g["tflops"], "peak": fp8_peak,
-                    "unit": "TFLOP/s", "frac": g["tflops"] / fp8_peak, "peak_source": peak_note}
-    else:
-        roofline = {"bound": "hbm", "kernel": gemm_label, "achieved": g["gbs"], "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s", "frac": g["gbs"] / peaks["hbm_gbs"], "peak_source": "%s copy bandwidth" % (
-                        peaks["source"]),
-                    "tensor_frac": g["tflops"] / fp8_peak, "tensor_peak_source": peak_note}
-    roofline.update(traffic=traffic_for(gemm_label, name), algorithmic_flops_per_launch=gemm_flops_,
-                    algorithmic_bytes_per_launch=gemm_bytes_, intensity_flop_per_byte=intensity,
-                    ridge_flop_per_byte=ridge)
+    roofline = gemm_roofline(plan, kernels, peaks, fp8_peak, bf16_peak, sustained, name)
     value = world * flops * args.steps / (elapsed_ms / 1e3) / 1e12
     cpu = None
     if world == 1 and not args.no_cpu_baseline:

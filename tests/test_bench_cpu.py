@@ -71,3 +71,31 @@ def test_cpu_sample_size_is_bounded():
     d = wl.tiny_dense()
     rows, nb = bench.cpu_sample_size("tiny_dense", d, 0.05)
     assert 1 <= rows <= d.M and 1 <= nb <= d.N // 128
+
+
+def test_gemm_roofline_bound_follows_intensity():
+    """Dense shapes are tensor-bound; the masked decode (few rows per expert)
+    falls below the ridge and is reported against HBM."""
+    from types import SimpleNamespace
+    import numpy as np
+    peaks = {"hbm_gbs": 6545.0, "source": "measured"}
+    fp8 = 2 * 1627.8
+
+    def kernels_for(plan, ms=1.0):
+        return {l: {"avg_ms": ms, "tflops": (f / ms / 1e9) if f else 0.0, "gbs": b / ms / 1e6} for l, b, f in plan}
+
+    dense = SimpleNamespace(M=4096, N=7168, K=7168)
+    plan = bench.kernel_plan("dense_fprop", dense)
+    r = bench.gemm_roofline(plan, kernels_for(plan), peaks, fp8, 1627.8, False, "dense_fprop")
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["intensity_flop_per_byte"] > r["ridge_flop_per_byte"]
+
+    E, cap, K, N, K2, N2 = 32, 256, 7168, 4096, 2048, 7168
+    masked_m = np.full(E, 156, dtype=np.int32)
+    shape = lambda *dims: SimpleNamespace(shape=dims)  # noqa: E731  (kernel_plan reads shapes only)
+    masked = SimpleNamespace(a=shape(E, cap, K), b=shape(E, N, K), a2=shape(E, cap, K2), b2=shape(E, N2, K2),
+                             masked_m=masked_m,
+                             flops=lambda second: 2.0 * masked_m.sum() * (N2 * K2 if second else N * K))
+    plan = bench.kernel_plan("moe_masked", masked)
+    r = bench.gemm_roofline(plan, kernels_for(plan), peaks, fp8, 1627.8, False, "moe_masked")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and 0 < r["tensor_frac"] < 1
+    assert r["intensity_flop_per_byte"] < r["ridge_flop_per_byte"]
