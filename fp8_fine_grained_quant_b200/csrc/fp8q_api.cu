@@ -1,5 +1,5 @@
 // fp8q_api.cu -- the C ABI declared in include/fp8q.h: argument validation,
-// TMA descriptor encoding, tile-shape choice and launches on the caller's
+// TMA descriptor encoding, kernel-instance choice and launches on the caller's
 // stream.  One translation unit holds every kernel so the device status word
 // is a single symbol.
 #include <cuda.h>
