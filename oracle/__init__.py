@@ -64,6 +64,8 @@ def _load():
     lib.orc_quant_act_1x128.argtypes = [P, I64, I64, P, P]
     lib.orc_quant_w_128x128.argtypes = [P, I64, I64, I64, P, P]
     lib.orc_quant_tensor.argtypes = [P, I64, P, P]
+    lib.orc_quant_with_scale.argtypes = [P, I64, ctypes.c_float, P]
+    lib.orc_quant_with_scale.restype = ctypes.c_int
     lib.orc_gemm_blockscaled.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
     lib.orc_grouped_contiguous.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, I64, P]
     lib.orc_grouped_masked.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, I64, P]
@@ -171,6 +173,14 @@ def quant_tensor(x_bf16: np.ndarray):
     s = np.empty(1, dtype=np.float32)
     _check(_load().orc_quant_tensor(_ptr(x), x.size, _ptr(q), _ptr(s)), "quant_tensor")
     return q, float(s[0])
+
+
+def quant_with_scale(x_bf16: np.ndarray, s: float) -> np.ndarray:
+    """E4M3 codes of fl32(x / s) for a given scale s (delayed scaling)."""
+    x = _bf16(x_bf16)
+    q = np.empty(x.shape, dtype=np.uint8)
+    _check(_load().orc_quant_with_scale(_ptr(x), x.size, float(s), _ptr(q)), "quant_with_scale")
+    return q
 
 
 # --------------------------------------------------------------------------- GEMMs

@@ -188,8 +188,8 @@ int orc_quant_w_128x128(const uint16_t* w, int64_t G, int64_t N, int64_t K, uint
 }
 
 /* Per-tensor quantization (the standard practice [P1] contrasts with the
- * fine-grained scheme): one scale for all n elements.  Used only by the
- * accumulation-drift diagnostic. */
+ * fine-grained scheme): one scale for all n elements.  Used by the
+ * accumulation-drift diagnostic and the scaling-accuracy study. */
 int orc_quant_tensor(const uint16_t* x, int64_t n, uint8_t* q, float* s_out) {
   if (n < 0) return -1;
   float amax = 0.0f;
@@ -201,6 +201,17 @@ int orc_quant_tensor(const uint16_t* x, int64_t n, uint8_t* q, float* s_out) {
   *s_out = sc;
 #pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < n; ++i) q[i] = orc_e4m3_encode(bf16_to_float(x[i]) / sc);
+  return 0;
+}
+
+/* Quantization with a given scale (delayed scaling, which the codingmall page
+ * contrasts with online scaling: the scale comes from earlier iterations'
+ * maxima, so values beyond 448 * s saturate at +-448).  Used only by the
+ * scaling-accuracy study. */
+int orc_quant_with_scale(const uint16_t* x, int64_t n, float s, uint8_t* q) {
+  if (n < 0 || !(s > 0.0f)) return -1;
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) q[i] = orc_e4m3_encode(bf16_to_float(x[i]) / s);
   return 0;
 }
 

@@ -205,3 +205,58 @@ def test_bf16_generator_rounding_matches_torch():
 def test_rejects_bad_shapes(orc):
     with pytest.raises(ValueError):
         orc.quant_w_128x128(np.zeros((100, 128), dtype=np.uint16))
+
+
+# --------------------------------------------------------------------------- delayed scaling (given scale)
+def _golden_bf16_encodings():
+    out = []
+    for tok in golden_lines("e4m3_encodings.txt"):
+        if tok[0] == "decode" or tok[0].lower() == "nan":
+            continue
+        v = np.float32(hexfloat(tok[0]))
+        b = bf16_bits(np.array([v], dtype=np.float32))
+        if bf16_to_f32(b)[0] == v:  # exactly a bf16 value
+            out.append((b[0], int(tok[1], 16)))
+    return out
+
+
+def test_quant_with_scale_golden_encodings(orc):
+    """With s = 1 the codes are the hand-computed encodings; with s = 2^-3 and
+    inputs scaled by 2^-3 (exact in bf16) they are the same codes."""
+    cases = _golden_bf16_encodings()
+    assert len(cases) >= 15
+    bits = np.array([b for b, _ in cases], dtype=np.uint16)
+    codes = np.array([c for _, c in cases], dtype=np.uint8)
+    assert np.array_equal(orc.quant_with_scale(bits, 1.0), codes)
+    scaled = bf16_bits(bf16_to_f32(bits) * np.float32(0.125))
+    assert np.array_equal(bf16_to_f32(scaled), bf16_to_f32(bits) * np.float32(0.125))
+    assert np.array_equal(orc.quant_with_scale(scaled, 0.125), codes)
+
+
+def test_quant_with_scale_saturates_beyond_448s(orc):
+    x = bf16_bits(np.array([[1e-3, -1e-3, 5.0, -7.0, 0.0]], dtype=np.float32))
+    q = orc.quant_with_scale(x, 1e-6)  # every nonzero |x| / s is at least 1000 > 448
+    assert list(q[0]) == [0x7E, 0xFE, 0x7E, 0xFE, 0x00]
+
+
+def test_quant_with_scale_at_current_amax_is_per_tensor(orc):
+    d = tiny_dense()
+    q_t, s_t = orc.quant_tensor(d.a)
+    assert np.array_equal(orc.quant_with_scale(d.a, s_t), q_t)
+
+
+def test_scaling_study_orders_the_schemes(orc):
+    """On the outlier workload: fine-grained groups beat one scale per tensor,
+    and a delayed scale that has not seen a new outlier clips it (large
+    error) while the fine-grained scheme is unaffected."""
+    from oracle.scaling_accuracy import study
+    d = tiny_dense()
+    rows = np.arange(d.a.shape[0], dtype=np.int64)
+    r = {x["name"]: x for x in study(d.a, d.b, rows)}
+    fine = r["fine-grained 1x128 / 128x128, online"]
+    tensor = r["per-tensor, online"]
+    spike_delayed = r["per-tensor, delayed (new outlier at 4x the history max)"]
+    spike_fine = r["fine-grained, online, same new outlier"]
+    assert fine["act_err"] < tensor["act_err"] and fine["fro_rel"] < tensor["fro_rel"]
+    assert spike_delayed["fro_rel"] > 3 * spike_fine["fro_rel"]
+    assert spike_fine["fro_rel"] < 1.1 * fine["fro_rel"]
