@@ -66,6 +66,10 @@ def _load():
     lib.orc_quant_tensor.argtypes = [P, I64, P, P]
     lib.orc_quant_with_scale.argtypes = [P, I64, ctypes.c_float, P]
     lib.orc_quant_with_scale.restype = ctypes.c_int
+    lib.orc_quant_act_128x1.argtypes = [P, I64, I64, P, P]
+    lib.orc_quant_act_128x1.restype = ctypes.c_int
+    lib.orc_gemm_1d1d.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
+    lib.orc_gemm_1d1d.restype = ctypes.c_int
     lib.orc_gemm_blockscaled.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
     lib.orc_grouped_contiguous.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, I64, P]
     lib.orc_grouped_masked.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, I64, P]
@@ -153,6 +157,17 @@ def quant_act_1x128(x_bf16: np.ndarray):
     return q, s
 
 
+def quant_act_128x1(x_bf16: np.ndarray):
+    """[M,K] bf16 bits -> (q [M,K] codes, s [ceil(M/128),K] float32): groups of
+    128 tokens per channel (the token-axis tiles of the weight gradient)."""
+    x = _bf16(x_bf16)
+    M, K = x.shape
+    q = np.empty((M, K), dtype=np.uint8)
+    s = np.empty(((M + TILE - 1) // TILE, K), dtype=np.float32)
+    _check(_load().orc_quant_act_128x1(_ptr(x), M, K, _ptr(q), _ptr(s)), "quant_act_128x1")
+    return q, s
+
+
 def quant_w_128x128(w_bf16: np.ndarray):
     """[N,K] or [G,N,K] bf16 bits -> (q, s [.., N/128, K/128])."""
     w = _bf16(w_bf16)
@@ -207,6 +222,33 @@ def gemm_blockscaled(qa, sa, qb, sb, rows=None) -> np.ndarray:
     _check(_load().orc_gemm_blockscaled(_ptr(qa, "u8"), _ptr(sa, "f32"), _ptr(qb, "u8"), _ptr(sb, "f32"), M, N, K, _ptr(r), nr, _ptr(C)),
            "gemm_blockscaled")
     return C
+
+
+def gemm_1d1d(qa, sa, qb, sb, rows=None) -> np.ndarray:
+    """float64 C = A * B^T with per-row, per-slab scales on both operands
+    (sa [M,K/128], sb [N,K/128]); optional row subset."""
+    M, K = qa.shape
+    N = qb.shape[0]
+    _shapes(sa, (M, K // TILE), qb, (N, K), sb, (N, K // TILE))
+    r, nr = _rows(rows)
+    C = np.empty((nr if r is not None else M, N), dtype=np.float64)
+    _check(_load().orc_gemm_1d1d(_ptr(np.ascontiguousarray(qa), "u8"), _ptr(np.ascontiguousarray(sa), "f32"),
+                                 _ptr(np.ascontiguousarray(qb), "u8"), _ptr(np.ascontiguousarray(sb), "f32"),
+                                 M, N, K, _ptr(r), nr, _ptr(C)), "gemm_1d1d")
+    return C
+
+
+def wgrad(q_dy, s_dy, q_x, s_x, rows=None) -> np.ndarray:
+    """dW [N,K] = dY^T X from token-axis quantized dY [M,N] and X [M,K]
+    (quant_act_128x1 of each; M a multiple of 128).  Rows index N."""
+    return gemm_1d1d(np.ascontiguousarray(q_dy.T), np.ascontiguousarray(s_dy.T),
+                     np.ascontiguousarray(q_x.T), np.ascontiguousarray(s_x.T), rows)
+
+
+def dgrad(q_dy, s_dy, q_w, s_w, rows=None) -> np.ndarray:
+    """dX [M,K] = dY W from 1x128-quantized dY [M,N] and 128x128-quantized
+    W [N,K]: the forward GEMM with W's codes and block scales transposed."""
+    return gemm_blockscaled(q_dy, s_dy, np.ascontiguousarray(q_w.T), np.ascontiguousarray(s_w.T), rows)
 
 
 def grouped_contiguous(qa, sa, qb, sb, m_indices, rows=None, out=None) -> np.ndarray:

@@ -158,6 +158,34 @@ int orc_quant_act_1x128(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, flo
   return 0;
 }
 
+/* Activation quantization along the token axis (128x1 tiles): x is [M, K]
+ * (tokens x channels); the group of (mb, k) is column k, rows 128*mb..+127
+ * (fewer in a ragged last block).  s is [ceil(M/128), K].  The backward
+ * GEMM that contracts over tokens (Wgrad, [P1] Figure 6: Fprop, Dgrad and
+ * Wgrad all in FP8) needs its operands grouped along the contraction, so the
+ * 1x128 rule is applied to the transposed tensor; the pages do not spell
+ * this layout out, it is the reading that keeps every scale constant within
+ * a 128-deep slab of the contraction. */
+int orc_quant_act_128x1(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s) {
+  if (M < 0 || K < 0) return -1;
+  const int64_t nmb = (M + ORC_TILE - 1) / ORC_TILE;
+#pragma omp parallel for schedule(static)
+  for (int64_t k = 0; k < K; ++k) {
+    for (int64_t mb = 0; mb < nmb; ++mb) {
+      const int64_t m0 = mb * ORC_TILE, m1 = m0 + ORC_TILE < M ? m0 + ORC_TILE : M;
+      float amax = 0.0f;
+      for (int64_t m = m0; m < m1; ++m) {
+        float a = fabsf(bf16_to_float(x[m * K + k]));
+        if (a > amax) amax = a;
+      }
+      float sc = group_scale(amax);
+      s[mb * K + k] = sc;
+      for (int64_t m = m0; m < m1; ++m) q[m * K + k] = orc_e4m3_encode(bf16_to_float(x[m * K + k]) / sc);
+    }
+  }
+  return 0;
+}
+
 /* Weight quantization, 128x128 blocks: w is [G, N, K] (K fastest, i.e. the
  * usual [out_features, in_features] layout, G = 1 for one matrix).  The group
  * of block (g, nb, kb) is rows 128*nb..+127 and columns 128*kb..+127: one
@@ -256,6 +284,37 @@ int orc_gemm_blockscaled(const uint8_t* qa, const float* sa, const uint8_t* qb, 
   for (int64_t i = 0; i < count; ++i) {
     int64_t m = rows ? rows[i] : i;
     gemm_one_row(qa + m * K, sa + m * nkb, qb, sb, N, K, dec, C + i * N);
+  }
+  return 0;
+}
+
+/* Both operands scaled per row and per 128-deep slab ("1D x 1D"): qa [M,K]
+ * with sa [M,K/128], qb [N,K] with sb [N,K/128]:
+ *   C[m,n] = sum_kb sa[m,kb] * sb[n,kb] * sum_{k in slab kb} dA[m,k] * dB[n,k]
+ * This is the weight-gradient GEMM once both of its operands are grouped
+ * along the token axis (each token-slab of a channel has its own scale).
+ * Exact per slab in double, like orc_gemm_blockscaled. */
+int orc_gemm_1d1d(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, int64_t M, int64_t N,
+                  int64_t K, const int64_t* rows, int64_t nrows, double* C) {
+  if (M < 0 || N < 0 || K < 0 || K % ORC_TILE) return -1;
+  double dec[256];
+  orc_e4m3_decode_table(dec);
+  const int64_t nkb = K / ORC_TILE;
+  const int64_t count = rows ? nrows : M;
+  for (int64_t i = 0; i < count; ++i)
+    if (rows && (rows[i] < 0 || rows[i] >= M)) return -2;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < count; ++i) {
+    const int64_t m = rows ? rows[i] : i;
+    for (int64_t n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int64_t kb = 0; kb < nkb; ++kb) {
+        double part = 0.0;
+        for (int64_t k = kb * ORC_TILE; k < (kb + 1) * ORC_TILE; ++k) part += dec[qa[m * K + k]] * dec[qb[n * K + k]];
+        acc += (double)sa[m * nkb + kb] * (double)sb[n * nkb + kb] * part;
+      }
+      C[i * N + n] = acc;
+    }
   }
   return 0;
 }

@@ -217,3 +217,92 @@ def test_drift_grows_with_k_and_promotion_removes_it(orc):
     assert all(x < y for x, y in zip(rel_unpromoted, rel_unpromoted[1:])), rel_unpromoted
     assert rel_unpromoted[2] > 10 * rel_promoted[2], (rel_unpromoted, rel_promoted)
     assert max(rel_promoted) < 2e-3
+
+
+# --------------------------------------------------------------------------- backward GEMMs (oracle side)
+def _rand_bits(rng, shape, scale=1.0, outliers=0):
+    x = (scale * rng.standard_normal(shape)).astype(np.float32)
+    if outliers:
+        idx = rng.choice(x.size, size=outliers, replace=False)
+        x.reshape(-1)[idx] *= 100.0
+    return bf16_bits(x)
+
+
+def test_token_axis_tiles_are_transposed_1x128(orc):
+    """128x1 tiles of X are the 1x128 tiles of X^T: same codes, same scales."""
+    rng = np.random.default_rng(30)
+    x = _rand_bits(rng, (256, 384), outliers=7)
+    q, s = orc.quant_act_128x1(x)
+    qt, st = orc.quant_act_1x128(np.ascontiguousarray(x.T))
+    assert np.array_equal(q, qt.T)
+    assert np.array_equal(s.view(np.uint32), st.T.view(np.uint32))
+
+
+def test_token_axis_ragged_last_group(orc):
+    """A ragged last group of tokens takes its scale from its own rows only."""
+    x = np.zeros((200, 2), dtype=np.float32)
+    x[:128, 0] = 1.0
+    x[5, 0] = 448.0          # first group of column 0: amax 448 -> scale 1
+    x[128:, 0] = 2.0         # last group (72 rows): amax 2 -> scale fl32(2/448)
+    x[150, 1] = -3.5         # column 1: only the last group is non-zero
+    q, s = orc.quant_act_128x1(bf16_bits(x))
+    assert s.shape == (2, 2)
+    assert s[0, 0] == 1.0 and s[0, 1] == 1.0  # zero group -> 1
+    assert s[1, 0] == np.float32(np.float32(2.0) / np.float32(448.0))
+    assert s[1, 1] == np.float32(np.float32(3.5) / np.float32(448.0))
+    assert q[5, 0] == 0x7E and q[0, 0] == orc.e4m3_encode(1.0)
+    assert q[150, 1] == 0xFE and np.all(q[128:, 0] == 0x7E)
+
+
+def test_1d1d_with_blockwise_equal_scales_is_the_blockscaled_gemm(orc):
+    rng = np.random.default_rng(31)
+    M, N, K = 96, 256, 384
+    qa, sa = orc.quant_act_1x128(_rand_bits(rng, (M, K), outliers=3))
+    qb, sb = orc.quant_w_128x128(_rand_bits(rng, (N, K), scale=0.02))
+    c_block = orc.gemm_blockscaled(qa, sa, qb, sb)
+    c_1d1d = orc.gemm_1d1d(qa, sa, qb, np.repeat(sb, TILE, axis=0))
+    assert np.array_equal(c_block, c_1d1d)
+
+
+def test_1d1d_is_the_dequantized_product(orc):
+    """Per-row scales on both sides: the result is the product of the
+    dequantized operands (a library float64 matmul of decoded codes times
+    scales), to float64 rounding."""
+    rng = np.random.default_rng(32)
+    M, N, K = 64, 160, 512
+    qa = rng.integers(0, 256, (M, K), dtype=np.uint8)
+    qb = rng.integers(0, 256, (N, K), dtype=np.uint8)
+    qa[(qa & 0x7F) == 0x7F] = 0  # no NaN codes
+    qb[(qb & 0x7F) == 0x7F] = 0
+    sa = rng.uniform(0.5, 2.0, (M, K // TILE)).astype(np.float32)
+    sb = rng.uniform(0.5, 2.0, (N, K // TILE)).astype(np.float32)
+    deq_a = _decode(qa) * np.repeat(sa.astype(np.float64), TILE, axis=1)
+    deq_b = _decode(qb) * np.repeat(sb.astype(np.float64), TILE, axis=1)
+    ref = deq_a @ deq_b.T
+    got = orc.gemm_1d1d(qa, sa, qb, sb)
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_wgrad_and_dgrad_compose_from_the_quantizers(orc):
+    """dW = dY^T X on token-axis tiles and dX = dY W on the forward tiles equal
+    the products of the dequantized tensors (library matmul)."""
+    rng = np.random.default_rng(33)
+    M, N, K = 256, 256, 384  # tokens, output channels, input channels
+    dy = _rand_bits(rng, (M, N), outliers=5)
+    x = _rand_bits(rng, (M, K), outliers=5)
+    w = _rand_bits(rng, (N, K), scale=0.02)
+    q_dy, s_dy = orc.quant_act_128x1(dy)
+    q_x, s_x = orc.quant_act_128x1(x)
+    dw = orc.wgrad(q_dy, s_dy, q_x, s_x)
+    deq_dy = _decode(q_dy) * np.repeat(s_dy.astype(np.float64), TILE, axis=0)
+    deq_x = _decode(q_x) * np.repeat(s_x.astype(np.float64), TILE, axis=0)
+    ref_w = deq_dy.T @ deq_x
+    assert dw.shape == (N, K)
+    assert np.allclose(dw, ref_w, rtol=1e-12, atol=1e-12 * np.abs(ref_w).max())
+    q_dy1, s_dy1 = orc.quant_act_1x128(dy)
+    q_w, s_w = orc.quant_w_128x128(w)
+    dx = orc.dgrad(q_dy1, s_dy1, q_w, s_w)
+    ref_x = (_decode(q_dy1) * np.repeat(s_dy1.astype(np.float64), TILE, axis=1)) @ (
+        _decode(q_w) * np.repeat(np.repeat(s_w.astype(np.float64), TILE, axis=0), TILE, axis=1))
+    assert dx.shape == (M, K)
+    assert np.allclose(dx, ref_x, rtol=1e-12, atol=1e-12 * np.abs(ref_x).max())
