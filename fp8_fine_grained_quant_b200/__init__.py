@@ -10,6 +10,8 @@ Names and semantics match the C entry points:
 
 * :func:`fp8_quant_act_1x128`  -- bf16 [M,K] -> E4M3 [M,K] + f32 scales [M,K/128]
 * :func:`fp8_quant_w_128x128`  -- bf16 [N,K] or [G,N,K] -> E4M3 + f32 scales [..,N/128,K/128]
+* :func:`fp8_quant_act_128x1`  -- bf16 [M,K] -> E4M3 [M,K] + f32 scales [ceil(M/128),K] (token-axis tiles)
+* :func:`fp8_transpose_w_128x128` -- block-quantized W [..,N,K] -> W^T [..,K,N] (codes and block scales)
 * :func:`fp8_gemm_blockscaled` -- C = A * B^T (bf16) with per-128-slab promotion
 * :func:`fp8_grouped_gemm_contiguous` -- MoE grouped GEMM, contiguous layout
 * :func:`fp8_grouped_gemm_masked`     -- MoE grouped GEMM, masked layout
@@ -22,7 +24,8 @@ from pathlib import Path
 import torch
 
 __all__ = [
-    "fp8_quant_act_1x128", "fp8_quant_w_128x128", "fp8_gemm_blockscaled", "fp8_grouped_gemm_contiguous",
+    "fp8_quant_act_1x128", "fp8_quant_w_128x128", "fp8_quant_act_128x1", "fp8_transpose_w_128x128",
+    "fp8_gemm_blockscaled", "fp8_grouped_gemm_contiguous",
     "fp8_grouped_gemm_masked", "fp8_gemm_unpromoted_diag", "get_device_error", "set_wait_timeout_ns",
     "selftest_wait_timeout", "launch_count", "status_string", "Fp8qError", "lib", "LIB_PATH", "EXPORTS",
 ]
@@ -38,6 +41,8 @@ _I64 = ctypes.c_int64
 EXPORTS = {
     "fp8_quant_act_1x128": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
     "fp8_quant_w_128x128": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
+    "fp8_quant_act_128x1": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
+    "fp8_transpose_w_128x128": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P]),
     "fp8_gemm_blockscaled": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "fp8_grouped_gemm_contiguous": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "fp8_grouped_gemm_masked": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P]),
@@ -147,6 +152,48 @@ def fp8_quant_w_128x128(w: torch.Tensor, q: torch.Tensor | None = None, s: torch
         _check(lib().fp8_quant_w_128x128(_p(w), G, N, K, _p(q), _p(s), _stream(stream, w.device)),
                "fp8_quant_w_128x128")
     return q, s
+
+
+def fp8_quant_act_128x1(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None, stream=None):
+    """Token-axis (128x1) quantization.  Returns (q [M,K] float8_e4m3fn, s [ceil(M/128),K] f32)."""
+    _dev(x, "x", _BF16, (2,))
+    M, K = x.shape
+    nmb = (M + TILE - 1) // TILE
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+    if s is None:
+        s = torch.empty((nmb, K), dtype=torch.float32, device=x.device)
+    _dev(q, "q", _FP8)
+    _dev(s, "s", _F32)
+    if q.numel() != M * K or s.numel() != nmb * K:
+        raise ValueError("output sizes do not match x")
+    with torch.cuda.device(x.device):
+        _check(lib().fp8_quant_act_128x1(_p(x), M, K, _p(q), _p(s), _stream(stream, x.device)), "fp8_quant_act_128x1")
+    return q, s
+
+
+def fp8_transpose_w_128x128(q: torch.Tensor, s: torch.Tensor, qt: torch.Tensor | None = None,
+                            st: torch.Tensor | None = None, stream=None):
+    """Block-quantized W [N,K] or [G,N,K] (codes + [..,N/128,K/128] scales) -> W^T codes [..,K,N] and
+    scales [..,K/128,N/128].  With them, fp8_gemm_blockscaled(q_dy, s_dy, qt, st) is dX = dY W."""
+    _dev(q, "q", _FP8, (2, 3))
+    _dev(s, "s", _F32)
+    G, N, K = (1,) + tuple(q.shape) if q.dim() == 2 else tuple(q.shape)
+    lead = tuple(q.shape[:-2])
+    if s.numel() != G * (N // TILE) * (K // TILE):
+        raise ValueError("scale size does not match q")
+    if qt is None:
+        qt = torch.empty(lead + (K, N), dtype=torch.float8_e4m3fn, device=q.device)
+    if st is None:
+        st = torch.empty(lead + (K // TILE, N // TILE), dtype=torch.float32, device=q.device)
+    _dev(qt, "qt", _FP8)
+    _dev(st, "st", _F32)
+    if qt.numel() != G * N * K or st.numel() != G * (N // TILE) * (K // TILE):
+        raise ValueError("output sizes do not match q")
+    with torch.cuda.device(q.device):
+        _check(lib().fp8_transpose_w_128x128(_p(q), _p(s), G, N, K, _p(qt), _p(st), _stream(stream, q.device)),
+               "fp8_transpose_w_128x128")
+    return qt, st
 
 
 def _gemm_operands(qa, sa, qb, sb):

@@ -288,6 +288,42 @@ int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, uin
   return FP8Q_OK;
 }
 
+int fp8_quant_act_128x1(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
+  if (M < 0 || K < 0 || K % 128) return FP8Q_ERR_SHAPE;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (!x_bf16 || !q || !s) return FP8Q_ERR_NULL;
+  if (!aligned(x_bf16, 16) || !aligned(q, 16) || !aligned(s, 16)) return FP8Q_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  const int64_t blocks = ((M + 127) / 128) * (K / 128);
+  const int64_t cap = static_cast<int64_t>(dev->num_sms) * 16;
+  const int64_t grid = blocks < cap ? blocks : cap;
+  quant_act_128x1_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(static_cast<const uint8_t*>(x_bf16), q, s,
+                                                                           M, K, blocks);
+  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
+int fp8_transpose_w_128x128(const uint8_t* q, const float* s, int64_t G, int64_t N, int64_t K, uint8_t* qt,
+                            float* st, cudaStream_t stream) {
+  if (G < 0 || N < 0 || K < 0 || N % 128 || K % 128) return FP8Q_ERR_SHAPE;
+  if (G == 0 || N == 0 || K == 0) return FP8Q_OK;
+  if (!q || !s || !qt || !st) return FP8Q_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(qt, 16) || !aligned(s, 4) || !aligned(st, 4)) return FP8Q_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  const int64_t blocks = G * (N / 128) * (K / 128);
+  const int64_t cap = static_cast<int64_t>(dev->num_sms) * 16;
+  const int64_t grid = blocks < cap ? blocks : cap;
+  transpose_w_128x128_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(q, s, qt, st, N, K, blocks);
+  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
 static int dense_common(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, void* c, int64_t M,
                         int64_t N, int64_t K, int promote, cudaStream_t stream) {
   if (M < 0 || N < 0 || K < 128 || K % 128 || N % 128 || M >= kMaxRows || N >= kMaxRows || K >= kMaxRows)

@@ -265,6 +265,15 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
 }
 
 
+// 16 bytes in one 128-bit load (read-only, not kept in L1); p 16-byte aligned.
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 // 32 bytes in one 256-bit load (read-only, not kept in L1); p 32-byte aligned.
 __device__ __forceinline__ void ld_nc_v8(const void* p, uint32_t (&w)[8]) {
   asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"

@@ -198,4 +198,163 @@ __global__ void __launch_bounds__(256, 4) quant_w_128x128_kernel(const uint8_t* 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Token-axis tiles (128x1) for the weight-gradient GEMM, which contracts over
+// tokens: the group of (mb, k) is channel k over tokens 128*mb..+127 (fewer in
+// a ragged last block).  One 256-thread CTA per 128-token x 128-channel block:
+// thread t owns channels 8*(t%16)..+7 of rows 8*(t/16)..+7, so a warp reads
+// two rows of 256 contiguous bytes per load.  The per-channel amax is reduced
+// over the 16 row groups (a shuffle, then shared memory across the 8 warps);
+// each channel's codes use its own scale, with the same exact division-free
+// filter as the other quantizers.  s is [ceil(M/128), K].
+// ---------------------------------------------------------------------------
+
+// Codes of fl32(x / s_c) for the 8 bf16 in w (4 words; element i uses column
+// scale sc[i]) by IEEE division: the exact path.
+__device__ __noinline__ uint2 quantize8_cols_exact(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float s0,
+                                                   float s1, float s2, float s3, float s4, float s5, float s6,
+                                                   float s7) {
+  const uint32_t w[4] = {w0, w1, w2, w3};
+  const float sc[8] = {s0, s1, s2, s3, s4, s5, s6, s7};
+  uint32_t c[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float a0 = __fdiv_rn(__uint_as_float(w[2 * h] << 16), sc[4 * h]);
+    const float a1 = __fdiv_rn(__uint_as_float(w[2 * h] & 0xFFFF0000u), sc[4 * h + 1]);
+    const float a2 = __fdiv_rn(__uint_as_float(w[2 * h + 1] << 16), sc[4 * h + 2]);
+    const float a3 = __fdiv_rn(__uint_as_float(w[2 * h + 1] & 0xFFFF0000u), sc[4 * h + 3]);
+    c[h] = cvt_e4m3x2(a0, a1) | (cvt_e4m3x2(a2, a3) << 16);
+  }
+  return make_uint2(c[0], c[1]);
+}
+
+__global__ void __launch_bounds__(256) quant_act_128x1_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
+                                                              float* __restrict__ s, int64_t M, int64_t K,
+                                                              int64_t num_blocks) {
+  __shared__ float col_max[8][16][8];  // [warp][column group][column]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cg = tid & 15, rg = tid >> 4;
+  const int64_t nkc = K >> 7;
+  for (int64_t b = blockIdx.x; b < num_blocks; b += gridDim.x) {
+    const int64_t mb = b / nkc, kc = b % nkc;
+    const int64_t col0 = kc * 128 + cg * 8;
+    const int64_t row0 = mb * 128 + rg * 8;
+    uint4 v[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int64_t row = row0 + r;
+      v[r] = row < M ? ld_nc_v4(x + (row * K + col0) * 2) : make_uint4(0, 0, 0, 0);
+    }
+    // per-column maxima over this thread's 8 rows
+    float m[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) m[c] = 0.0f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const uint32_t w[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        m[2 * i] = fmaxf(m[2 * i], fabsf(__uint_as_float(w[i] << 16)));
+        m[2 * i + 1] = fmaxf(m[2 * i + 1], fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
+      }
+    }
+    // lanes l and l ^ 16 hold the same columns (two row groups of the warp)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) m[c] = fmaxf(m[c], __shfl_xor_sync(0xFFFFFFFFu, m[c], 16));
+    if (lane < 16) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) col_max[warp][cg][c] = m[c];
+    }
+    __syncthreads();
+    float sc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float a = col_max[0][cg][c];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) a = fmaxf(a, col_max[w][cg][c]);
+      sc[c] = group_scale(a);
+    }
+    __syncthreads();  // col_max is reused by the next block
+    if (rg == 0) {
+      float* sd = s + mb * K + col0;
+      *reinterpret_cast<float4*>(sd) = make_float4(sc[0], sc[1], sc[2], sc[3]);
+      *reinterpret_cast<float4*>(sd + 4) = make_float4(sc[4], sc[5], sc[6], sc[7]);
+    }
+    // bracketing reciprocals per column, paired as the packed products need them
+    uint64_t lo2[4], hi2[4];
+    bool exact_only = false;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float r0 = __frcp_rn(sc[2 * i]), r1 = __frcp_rn(sc[2 * i + 1]);
+      asm("mov.b64 %0, {%1, %2};" : "=l"(lo2[i]) : "f"(__fmul_rn(r0, 1.0f - 0x1p-20f)), "f"(__fmul_rn(r1, 1.0f - 0x1p-20f)));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[i]) : "f"(__fmul_rn(r0, 1.0f + 0x1p-20f)), "f"(__fmul_rn(r1, 1.0f + 0x1p-20f)));
+      exact_only |= sc[2 * i] < kMinFastScale || sc[2 * i + 1] < kMinFastScale;
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int64_t row = row0 + r;
+      if (row >= M) break;
+      const uint32_t w[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+      uint32_t lo[2], hi[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint64_t x0 = bf16x2_to_f32x2(w[2 * h]), x1 = bf16x2_to_f32x2(w[2 * h + 1]);
+        lo[h] = e4m3x4_from_f32x2(mul_f32x2(x0, lo2[2 * h]), mul_f32x2(x1, lo2[2 * h + 1]));
+        hi[h] = e4m3x4_from_f32x2(mul_f32x2(x0, hi2[2 * h]), mul_f32x2(x1, hi2[2 * h + 1]));
+      }
+      uint2 out = make_uint2(lo[0], lo[1]);
+      if (exact_only || ((lo[0] ^ hi[0]) | (lo[1] ^ hi[1])) != 0u)
+        out = quantize8_cols_exact(w[0], w[1], w[2], w[3], sc[0], sc[1], sc[2], sc[3], sc[4], sc[5], sc[6], sc[7]);
+      *reinterpret_cast<uint2*>(q + row * K + col0) = out;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Transposition of 128x128-block-quantized weights: codes [G, N, K] -> [G, K, N]
+// and block scales [G, N/128, K/128] -> [G, K/128, N/128].  A 128x128 block of
+// W^T is the transpose of W's block (same amax, same scale, the same codes),
+// so the forward GEMM on the transposed codes computes dY * W (the
+// activation-gradient GEMM).  One 256-thread CTA per block through a padded
+// shared tile; 16-byte loads and stores.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) transpose_w_128x128_kernel(const uint8_t* __restrict__ qw,
+                                                                  const float* __restrict__ sw,
+                                                                  uint8_t* __restrict__ qt, float* __restrict__ st,
+                                                                  int64_t N, int64_t K, int64_t num_blocks) {
+  constexpr int kPitch = 128 + 16;  // bytes per shared row (keeps 16-byte alignment)
+  __shared__ __align__(16) uint8_t tile[128 * kPitch];
+  const int tid = threadIdx.x;
+  const int64_t nkb = K >> 7, nnb = N >> 7;
+  for (int64_t b = blockIdx.x; b < num_blocks; b += gridDim.x) {
+    const int64_t g = b / (nnb * nkb), rem = b % (nnb * nkb);
+    const int64_t nb = rem / nkb, kb = rem % nkb;
+    const uint8_t* src = qw + (g * N + nb * 128) * K + kb * 128;
+    // 128 rows x 8 chunks of 16 bytes: thread t loads chunks t, t+256, t+512, t+768
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = tid + 256 * i, row = c >> 3, ch = c & 7;
+      *reinterpret_cast<uint4*>(tile + row * kPitch + ch * 16) =
+          ld_nc_v4(src + static_cast<int64_t>(row) * K + ch * 16);
+    }
+    __syncthreads();
+    uint8_t* dst = qt + (g * K + kb * 128) * N + nb * 128;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = tid + 256 * i, orow = c >> 3, ch = c & 7;  // output row = input column
+      uint32_t wv[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t acc = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc |= static_cast<uint32_t>(tile[(ch * 16 + w * 4 + j) * kPitch + orow]) << (8 * j);
+        wv[w] = acc;
+      }
+      *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(orow) * N + ch * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    }
+    if (tid == 0) st[(g * nkb + kb) * nnb + nb] = sw[(g * nnb + nb) * nkb + kb];
+    __syncthreads();  // the tile is reused by the next block
+  }
+}
+
 }  // namespace fp8q

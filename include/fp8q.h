@@ -89,6 +89,34 @@ FP8Q_API int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64
                         cudaStream_t stream);
 
 /*
+ * Activation quantization along the token axis, 128x1 tiles (for the weight
+ * gradient dW = dY^T X, which contracts over tokens; "The Insider Secrets Of
+ * Deepseek Discovered", Figure 6: Fprop, Dgrad and Wgrad all run in FP8).
+ * Same per-group rule as fp8_quant_act_1x128, over a channel's run of 128
+ * tokens instead of a token's run of 128 channels.
+ *   x_bf16 : [M, K] bf16 (tokens x channels), read only.
+ *   q      : [M, K] E4M3 codes, written.
+ *   s      : [ceil(M/128), K] float32, written; s[mb, k] is the scale of
+ *            x[128*mb .. min(M, 128*mb+128) - 1, k] (a ragged last group of
+ *            tokens takes its own scale).
+ * K must be a multiple of 128; any M >= 0.  x, q and s 16-byte aligned.
+ */
+FP8Q_API int fp8_quant_act_128x1(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream);
+
+/*
+ * Transposition of 128x128-block-quantized weights (for the activation
+ * gradient dX = dY W, the Dgrad GEMM of the same Figure 6): a 128x128 block
+ * of W^T has the same amax, scale and codes as W's block, transposed.
+ *   q  : [G, N, K] E4M3 codes, s : [G, N/128, K/128] (from fp8_quant_w_128x128)
+ *   qt : [G, K, N] E4M3 codes, st : [G, K/128, N/128], written.
+ * Then fp8_gemm_blockscaled(q_dy, s_dy, qt, st, dX, M, K, N) computes
+ * dX = dY W with dY 1x128-quantized (fp8_quant_act_1x128 of dY [M, N]).
+ * N, K multiples of 128.  q, qt 16-byte aligned; s, st 4-byte aligned.
+ */
+FP8Q_API int fp8_transpose_w_128x128(const uint8_t* q, const float* s, int64_t G, int64_t N, int64_t K, uint8_t* qt,
+                                     float* st, cudaStream_t stream);
+
+/*
  * Dense block-scaled FP8 GEMM, C = A * B^T, with promotion at every 128-wide
  * K slab ("The Insider Secrets Of Deepseek Discovered", Figure 7 (b); codingmall
  * page, increased accumulation precision):

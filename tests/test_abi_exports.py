@@ -136,3 +136,24 @@ def test_binding_rejects_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         fq.fp8_quant_act_1x128(torch.zeros(4, 128, dtype=torch.bfloat16))
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((A16, 4, 100, A16, A16, None), fq.ERR_SHAPE),    # K not a multiple of 128
+    ((A16, -1, 128, A16, A16, None), fq.ERR_SHAPE),
+    ((A16, 0, 128, A16, A16, None), fq.OK),
+    ((None, 4, 128, A16, A16, None), fq.ERR_NULL),
+    ((A16, 4, 128, A16, A4, None), fq.ERR_ALIGN),     # scales written as 16-byte vectors
+])
+def test_quant_act_128x1_validation(args, expect):
+    assert _call("fp8_quant_act_128x1", *args) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((A16, A16, 1, 100, 128, A16, A16, None), fq.ERR_SHAPE),
+    ((A16, A16, 1, 128, 0, A16, A16, None), fq.OK),
+    ((A16, None, 1, 128, 128, A16, A16, None), fq.ERR_NULL),
+    ((A16, A16, 1, 128, 128, A4, A16, None), fq.ERR_ALIGN),
+])
+def test_transpose_w_validation(args, expect):
+    assert _call("fp8_transpose_w_128x128", *args) == expect

@@ -1,0 +1,98 @@
+"""GPU kernels of the backward GEMMs' operands vs the oracle (bit for bit).
+
+Dgrad (dX = dY W) is the forward GEMM on W's block-quantized codes and scales
+transposed; Wgrad (dW = dY^T X) needs both operands grouped along tokens
+(128x1 tiles).  "The Insider Secrets Of Deepseek Discovered", Figure 6: all
+three GEMMs of a linear layer run in FP8.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import fp8_fine_grained_quant_b200 as fq
+import workloads as wl
+from parity import assert_gemm_close, bf16_bits_of, bytes_of, to_torch_bf16
+
+pytestmark = pytest.mark.gpu
+TILE = 128
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+def _bits(rng, shape, scale=1.0, outliers=0, chan=False):
+    x = (scale * rng.standard_normal(shape)).astype(np.float32)
+    if chan:
+        x *= np.exp(rng.standard_normal(shape[-1])).astype(np.float32)
+    if outliers:
+        idx = rng.choice(x.size, size=outliers, replace=False)
+        x.reshape(-1)[idx] = np.where(rng.random(outliers) < 0.5, -200.0, 200.0)
+    return wl.bf16_bits(x)
+
+
+@pytest.mark.parametrize("M,K", [(128, 128), (256, 384), (200, 256), (1, 128), (1000, 640)])
+def test_token_axis_quant_matches_oracle(dev, M, K):
+    rng = np.random.default_rng(M * 7 + K)
+    x = _bits(rng, (M, K), outliers=max(1, M * K // 5000), chan=True)
+    if M > 10:
+        x[3, :] = 0      # a zero token
+        x[:, 5] = 0      # a zero channel: scale 1
+    q, s = fq.fp8_quant_act_128x1(to_torch_bf16(x, dev))
+    torch.cuda.synchronize(dev)
+    oq, os_ = oracle.quant_act_128x1(x)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+    assert np.array_equal(bytes_of(q).reshape(M, K), oq)
+
+
+def test_token_axis_quant_every_bf16_amax(dev):
+    """Every 16th finite non-negative bf16 value as the amax of one group."""
+    amax_bits = np.arange(0, 0x7F80, 16, dtype=np.uint32)
+    a = (amax_bits << 16).view(np.float32)
+    rng = np.random.default_rng(5)
+    g = a.size                                    # 2040 groups = channels
+    x = (a[None, :] * rng.random((TILE, g), dtype=np.float32)
+         * np.where(rng.random((TILE, g)) < 0.5, -1.0, 1.0).astype(np.float32))
+    xb = wl.bf16_bits(x)
+    xb[7, :] = amax_bits.astype(np.uint16)        # the amax of each channel's group
+    K = (g + TILE - 1) // TILE * TILE
+    xb = np.pad(xb, ((0, 0), (0, K - g)))
+    q, s = fq.fp8_quant_act_128x1(to_torch_bf16(xb, dev))
+    torch.cuda.synchronize(dev)
+    oq, os_ = oracle.quant_act_128x1(xb)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+    assert np.array_equal(bytes_of(q).reshape(xb.shape), oq)
+
+
+@pytest.mark.parametrize("shape", [(128, 128), (256, 384), (3, 128, 256)])
+def test_weight_transpose(dev, shape):
+    rng = np.random.default_rng(sum(shape))
+    w = _bits(rng, shape, scale=0.02)
+    q, s = fq.fp8_quant_w_128x128(to_torch_bf16(w, dev))
+    qt, st = fq.fp8_transpose_w_128x128(q, s)
+    torch.cuda.synchronize(dev)
+    qn, sn = bytes_of(q).reshape(shape), s.cpu().numpy()
+    assert np.array_equal(bytes_of(qt).reshape(shape[:-2] + (shape[-1], shape[-2])), np.swapaxes(qn, -1, -2))
+    assert np.array_equal(st.cpu().numpy(), np.swapaxes(sn, -1, -2))
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 384), (200, 512, 256)])
+def test_dgrad_through_the_forward_gemm(dev, M, N, K):
+    """dX = dY W: 1x128 tiles of dY, W's blocks transposed, the forward GEMM."""
+    rng = np.random.default_rng(M + N + K)
+    dy = _bits(rng, (M, N), outliers=4, chan=True)
+    w = _bits(rng, (N, K), scale=0.02)
+    q_dy, s_dy = fq.fp8_quant_act_1x128(to_torch_bf16(dy, dev))
+    q_w, s_w = fq.fp8_quant_w_128x128(to_torch_bf16(w, dev))
+    qt, st = fq.fp8_transpose_w_128x128(q_w, s_w)
+    dx = fq.fp8_gemm_blockscaled(q_dy, s_dy, qt, st)
+    torch.cuda.synchronize(dev)
+    assert fq.get_device_error(device=dev) == fq.OK
+    oq_dy, os_dy = oracle.quant_act_1x128(dy)
+    oq_w, os_w = oracle.quant_w_128x128(w)
+    ref = oracle.dgrad(oq_dy, os_dy, oq_w, os_w)
+    assert_gemm_close(bf16_bits_of(dx), ref, "dgrad %dx%dx%d" % (M, N, K))
