@@ -151,6 +151,10 @@ class ClockSampler:
 # ---------------------------------------------------------------------------- workloads
 def make_workload(name: str):
     import workloads as wl
+    if name == "dense_dgrad":
+        # the activation-gradient GEMM of the dense_fprop layer: dY takes the
+        # shape and distribution of the forward activations, W is the weight
+        return wl.dense_fprop()
     return wl.CONFIGS[name]()
 
 
@@ -158,6 +162,9 @@ def describe(name: str, d) -> dict:
     if name in ("tiny_dense", "dense_fprop", "long_k"):
         return {"workload": "%s M=%d N=%d K=%d" % (name, d.M, d.N, d.K), "M": d.M, "N": d.N, "K": d.K,
                 "seed": d.meta["seed"]}
+    if name == "dense_dgrad":
+        return {"workload": "dense_dgrad dX[M,K] = dY[M,N] W[N,K] M=%d N=%d K=%d" % (d.M, d.N, d.K), "M": d.M,
+                "N": d.N, "K": d.K, "seed": d.meta["seed"]}
     if name == "moe_contiguous":
         return {"workload": "moe_contiguous E=%d M_tot=%d (valid %d) N=%d K=%d" % (d.E, d.M_tot, int(d.counts.sum()),
                                                                                  d.N, d.K),
@@ -208,6 +215,12 @@ def kernel_plan(name, d):
         M, N, K = d.M, d.N, d.K
         return [("quant_act_1x128", qa_bytes(M, K), 0.0), ("quant_w_128x128", qw_bytes(1, N, K), 0.0),
                 ("gemm_blockscaled", gemm_bytes(M, N, K), 2.0 * M * N * K)]
+    if name == "dense_dgrad":
+        # dY is d.a [M, Nout], W is d.b [Nout, K]; dX = dY W is [M, K]
+        M, Nout, K = d.M, d.N, d.K
+        return [("quant_act_1x128", qa_bytes(M, Nout), 0.0), ("quant_w_128x128", qw_bytes(1, Nout, K), 0.0),
+                ("transpose_w_128x128", 2 * Nout * K + 2 * 4 * (Nout // TILE) * (K // TILE), 0.0),
+                ("gemm_dgrad", gemm_bytes(M, K, Nout), 2.0 * M * Nout * K)]
     if name == "moe_contiguous":
         return [("quant_act_1x128", qa_bytes(d.M_tot, d.K), 0.0), ("quant_w_128x128", qw_bytes(d.E, d.N, d.K), 0.0),
                 ("grouped_gemm_contiguous", gemm_bytes(d.M_tot, d.N, d.K, d.E), d.flops)]
@@ -247,6 +260,11 @@ def launch_step(name, d, s, fq, events=None):
         return c2
     rec(0, 0); qa, sa = fq.fp8_quant_act_1x128(s["a"], s.get("qa"), s.get("sa")); rec(0, 1)
     rec(1, 0); qb, sb = fq.fp8_quant_w_128x128(s["b"], s.get("qb"), s.get("sb")); rec(1, 1)
+    if name == "dense_dgrad":
+        rec(2, 0); qt, st = fq.fp8_transpose_w_128x128(qb, sb, s.get("qt"), s.get("st")); rec(2, 1)
+        rec(3, 0); c = fq.fp8_gemm_blockscaled(qa, sa, qt, st, out=s.get("c")); rec(3, 1)
+        s.update(qa=qa, sa=sa, qb=qb, sb=sb, qt=qt, st=st, c=c)
+        return c
     rec(2, 0)
     if name == "moe_contiguous":
         c = fq.fp8_grouped_gemm_contiguous(qa, sa, qb, sb, s["mi"], out=s.get("c"))
@@ -541,7 +559,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dense_fprop",
-                    choices=["tiny_dense", "dense_fprop", "long_k", "moe_contiguous", "moe_masked"])
+                    choices=["tiny_dense", "dense_fprop", "long_k", "moe_contiguous", "moe_masked", "dense_dgrad"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -99,3 +99,13 @@ def test_gemm_roofline_bound_follows_intensity():
     r = bench.gemm_roofline(plan, kernels_for(plan), peaks, fp8, 1627.8, False, "moe_masked")
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and 0 < r["tensor_frac"] < 1
     assert r["intensity_flop_per_byte"] < r["ridge_flop_per_byte"]
+
+
+def test_dgrad_plan_counts_the_transposed_gemm():
+    from types import SimpleNamespace
+    d = SimpleNamespace(M=4096, N=7168, K=7168)
+    plan = bench.kernel_plan("dense_dgrad", d)
+    labels = [l for l, _, _ in plan]
+    assert labels == ["quant_act_1x128", "quant_w_128x128", "transpose_w_128x128", "gemm_dgrad"]
+    assert plan[-1][2] == 2.0 * 4096 * 7168 * 7168
+    assert plan[2][1] == 2 * 7168 * 7168 + 8 * 56 * 56
