@@ -1,0 +1,178 @@
+"""Host model of the GEMM's barrier protocol, run under random schedules.
+
+The kernel's roles meet only through mbarriers (fp8q_gemm.cuh, "Barrier
+protocol"):
+  * producer threads on alternate slabs: wait empty[s] (the slab STAGES back
+    is done with the stage), then the TMA copies land on full[s] (operands,
+    and with staged scales the 4-slab scale box at each group start);
+  * MMA issuers on alternate slabs: wait full[s], issue, and one commit per
+    slab arrives on empty[s] once the MMAs complete;
+  * epilogue warps: wait empty[s] for slab j, read TMEM buffer j % ACC and the
+    scale slot of j's group, then every lane arrives on full[(s + ACC) % STAGES]
+    (the stage barrier of slab j + ACC, which reuses the buffer).
+Waits are parity waits, as on the device.  This model replays the protocol
+with asynchronous copy and MMA completion under many random interleavings and
+checks that every schedule finishes (no deadlock), that no parity wait passes
+on the wrong phase, and that no stage, TMEM buffer or scale slot is
+overwritten while a reader still needs its old contents.
+"""
+import random
+
+import pytest
+
+
+class Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.done = count, count, 0  # done = completed phases
+
+    def arrive(self, n=1):
+        self.pending -= n
+        assert self.pending >= 0, "more arrivals than the phase expects"
+        if self.pending == 0:
+            self.done += 1
+            self.pending = self.count
+
+    def passes(self, phase_index):
+        """Parity wait for phase `phase_index`; also checks it is not an alias."""
+        ok = (self.done % 2) != (phase_index % 2)
+        if ok:
+            assert self.done >= phase_index + 1, "parity wait passed on an earlier phase"
+        return ok
+
+
+def simulate(tiles, nkb, stages=6, acc=4, warps=8, lanes=32, producers=2, issuers=2, staged_scales=True,
+             slots=4, group=4, seed=0, max_steps=2_000_000):
+    rng = random.Random(seed)
+    J = tiles * nkb
+    full = [Bar(1 + warps * lanes) for _ in range(stages)]
+    empty = [Bar(1) for _ in range(stages)]
+    # epilogue: all TMEM buffers start free (every lane arrives up front)
+    for b in range(acc):
+        full[b].arrive(warps * lanes)
+
+    stage_slab = [None] * stages        # slab whose operands are in the stage
+    stage_readers = [0] * stages        # MMAs still to read the stage (0/1)
+    buf_slab = [None] * acc             # slab whose partial is in the TMEM buffer
+    buf_readers = [0] * acc             # epilogue warps still to read it
+    slot_group = [None] * slots         # scale group held by each slot
+    slot_readers = [0] * slots          # (warp, slab) reads still due from the slot
+
+    prod_next = list(range(producers))  # next slab of each producer
+    mma_next = list(range(issuers))
+    epi_next = [0] * warps
+    inflight_tma, inflight_mma = [], []
+    finished = [0] * J                  # epilogue warps done with slab j
+
+    def group_of(j):
+        return (j // nkb) * ((nkb + group - 1) // group) + (j % nkb) // group
+
+    def runnable():
+        acts = []
+        for p in range(producers):
+            j = prod_next[p]
+            if j < J and empty[j % stages].passes(j // stages - 1 if j >= stages else -1) or (j < J and j < stages):
+                acts.append(("prod", p))
+        for i in range(issuers):
+            j = mma_next[i]
+            if j < J and full[j % stages].passes(j // stages):
+                acts.append(("mma", i))
+        for w in range(warps):
+            j = epi_next[w]
+            if j < J and empty[j % stages].passes(j // stages):
+                acts.append(("epi", w))
+        if inflight_tma:
+            acts.append(("tma_land", None))
+        if inflight_mma:
+            acts.append(("mma_done", None))
+        return acts
+
+    steps = 0
+    while sum(finished) < J * warps:
+        acts = runnable()
+        assert acts, "deadlock at finished=%s" % finished
+        kind, who = rng.choice(acts)
+        steps += 1
+        assert steps < max_steps
+        if kind == "prod":
+            j = prod_next[who]
+            s = j % stages
+            assert stage_readers[s] == 0, "stage refilled before its MMA read it"
+            gstart = staged_scales and (j % nkb) % group == 0
+            if gstart:
+                g = group_of(j)
+                sl = g % slots
+                assert slot_readers[sl] == 0, "scale slot %d rewritten while group %s is still read" % (
+                    sl, slot_group[sl])
+            inflight_tma.append((j, s, gstart))
+            prod_next[who] += producers
+        elif kind == "tma_land":
+            j, s, gstart = inflight_tma.pop(rng.randrange(len(inflight_tma)))
+            stage_slab[s] = j
+            stage_readers[s] = 1
+            if gstart:
+                g = group_of(j)
+                sl = g % slots
+                slot_group[sl] = g
+                n_in_group = min(group, nkb - (j % nkb))
+                slot_readers[sl] = warps * n_in_group
+            full[s].arrive(1)
+        elif kind == "mma":
+            j = mma_next[who]
+            s, b = j % stages, j % acc
+            assert stage_slab[s] == j, "MMA read a stage holding another slab"
+            assert buf_readers[b] == 0, "TMEM buffer overwritten before the epilogue read it"
+            inflight_mma.append((j, s, b))
+            mma_next[who] += issuers
+        elif kind == "mma_done":
+            # commits complete in issue order per issuer; any order across issuers is allowed
+            idx = rng.randrange(len(inflight_mma))
+            j, s, b = inflight_mma.pop(idx)
+            stage_readers[s] = 0
+            buf_slab[b] = j
+            buf_readers[b] = warps
+            empty[s].arrive(1)
+        else:  # epilogue warp
+            j = epi_next[who]
+            s, b = j % stages, j % acc
+            assert buf_slab[b] == j, "epilogue read a buffer holding another slab"
+            buf_readers[b] -= 1
+            if staged_scales:
+                sl = group_of(j) % slots
+                assert slot_group[sl] == group_of(j), "scale slot holds another group"
+                slot_readers[sl] -= 1
+            full[(s + acc) % stages].arrive(lanes)  # every lane of the warp
+            finished[j] += 1
+            epi_next[who] += 1
+    return steps
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_protocol_random_schedules(seed):
+    simulate(tiles=3, nkb=8, seed=seed)
+
+
+@pytest.mark.parametrize("nkb", [4, 12])
+def test_protocol_tile_lengths(nkb):
+    for seed in range(4):
+        simulate(tiles=4, nkb=nkb, seed=100 + seed)
+
+
+def test_protocol_without_staged_scales():
+    for seed in range(4):
+        simulate(tiles=3, nkb=5, staged_scales=False, seed=200 + seed)
+
+
+def test_too_few_scale_slots_is_caught():
+    """Two slots are not enough: a schedule that rewrites a slot too early exists."""
+    with pytest.raises(AssertionError, match="scale slot"):
+        for seed in range(200):
+            simulate(tiles=2, nkb=16, slots=2, seed=300 + seed)
+
+
+
+def test_other_stage_and_buffer_counts():
+    """The protocol does not depend on the particular 6 stages x 4 buffers:
+    any ACC <= STAGES keeps every invariant (the kernel uses ACC < STAGES)."""
+    for stages, acc in [(5, 4), (4, 4), (8, 2), (3, 2)]:
+        for seed in range(3):
+            simulate(tiles=3, nkb=8, stages=stages, acc=acc, seed=500 + 10 * stages + seed)
