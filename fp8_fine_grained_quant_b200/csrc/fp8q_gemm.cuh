@@ -340,6 +340,11 @@ __device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, 
   constexpr int kAcc = L::kAccBufs;
   static_assert(kCols <= 128 && 128 % kCols == 0 && kGroup % 32 == 0, "each half must sit in one scale block");
   static_assert(kAcc < STAGES, "buffer releases are posted on the stage barrier of a later slab");
+  static_assert(L::kScaleSlots * L::kScaleGroup >= STAGES + kAcc + L::kScaleGroup - 1,
+                "a scale slot is rewritten only after every epilogue warp has read its previous group");
+  static_assert(STAGES % 2 == 0,
+                "two threads take alternate slabs per role; with an even stage count each waits only on its "
+                "own stages, so no parity wait can pass on an earlier phase");
   static_assert(kPromote || !kTmaScales, "staged scales serve the per-slab promotion only");
   constexpr bool promote = kPromote;
   const int quad = warp & 3;

@@ -170,9 +170,38 @@ def test_too_few_scale_slots_is_caught():
 
 
 
-def test_other_stage_and_buffer_counts():
+
+def _slots_needed(stages, acc, group=4):
+    # the producer of a group's first slab is at most STAGES + ACC slabs ahead
+    # of the slowest epilogue warp, which reads a slab's scales before it
+    # releases it: the previous occupant of a slot must end that far back
+    return -(-(stages + acc + group - 1) // group)
+
+
+def test_other_even_stage_counts():
     """The protocol does not depend on the particular 6 stages x 4 buffers:
-    any ACC <= STAGES keeps every invariant (the kernel uses ACC < STAGES)."""
-    for stages, acc in [(5, 4), (4, 4), (8, 2), (3, 2)]:
+    any even stage count with ACC <= STAGES keeps every invariant, given
+    enough scale slots."""
+    assert _slots_needed(6, 4) <= 4  # the kernel's configuration
+    for stages, acc in [(4, 4), (8, 2), (8, 6), (2, 2)]:
         for seed in range(3):
-            simulate(tiles=3, nkb=8, stages=stages, acc=acc, seed=500 + 10 * stages + seed)
+            simulate(tiles=3, nkb=8, stages=stages, acc=acc, slots=_slots_needed(stages, acc),
+                     seed=500 + 10 * stages + seed)
+
+
+def test_slot_count_bound_is_tight():
+    """One slot fewer than the bound admits a schedule that rewrites a slot early."""
+    with pytest.raises(AssertionError, match="scale slot"):
+        for seed in range(200):
+            simulate(tiles=3, nkb=16, stages=8, acc=6, slots=_slots_needed(8, 6) - 1, seed=700 + seed)
+
+
+@pytest.mark.parametrize("stages,acc", [(5, 4), (3, 2)])
+def test_odd_stage_counts_alias(stages, acc):
+    """Two issuers (and two producers) take alternate slabs.  With an odd
+    stage count, slab j + STAGES belongs to the other thread, which can run
+    ahead and pass a parity wait on the phase before its own: the kernel
+    therefore requires an even stage count."""
+    with pytest.raises(AssertionError, match="parity wait passed on an earlier phase"):
+        for seed in range(50):
+            simulate(tiles=3, nkb=8, stages=stages, acc=acc, seed=600 + seed)
