@@ -66,6 +66,10 @@ def _load():
     lib.orc_quant_tensor.argtypes = [P, I64, P, P]
     lib.orc_quant_with_scale.argtypes = [P, I64, ctypes.c_float, P]
     lib.orc_quant_with_scale.restype = ctypes.c_int
+    lib.orc_quant_act_1x128_ue8m0.argtypes = [P, I64, I64, P, P]
+    lib.orc_quant_act_1x128_ue8m0.restype = ctypes.c_int
+    lib.orc_quant_w_128x128_ue8m0.argtypes = [P, I64, I64, I64, P, P]
+    lib.orc_quant_w_128x128_ue8m0.restype = ctypes.c_int
     lib.orc_quant_act_128x1.argtypes = [P, I64, I64, P, P]
     lib.orc_quant_act_128x1.restype = ctypes.c_int
     lib.orc_gemm_1d1d.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
@@ -155,6 +159,29 @@ def quant_act_1x128(x_bf16: np.ndarray):
     s = np.empty((M, K // TILE), dtype=np.float32)
     _check(_load().orc_quant_act_1x128(_ptr(x), M, K, _ptr(q), _ptr(s)), "quant_act_1x128")
     return q, s
+
+
+def quant_act_1x128_ue8m0(x_bf16: np.ndarray):
+    """1x128 tiles with power-of-two (UE8M0) scales -> (q [M,K], s [M,K/128] f32, each 2^e)."""
+    x = _bf16(x_bf16)
+    M, K = x.shape
+    q = np.empty((M, K), dtype=np.uint8)
+    s = np.empty((M, K // TILE), dtype=np.float32)
+    _check(_load().orc_quant_act_1x128_ue8m0(_ptr(x), M, K, _ptr(q), _ptr(s)), "quant_act_1x128_ue8m0")
+    return q, s
+
+
+def quant_w_128x128_ue8m0(w_bf16: np.ndarray):
+    """128x128 blocks with power-of-two (UE8M0) scales, [N,K] or [G,N,K]."""
+    w = _bf16(w_bf16)
+    squeeze = w.ndim == 2
+    if squeeze:
+        w = w[None]
+    G, N, K = w.shape
+    q = np.empty((G, N, K), dtype=np.uint8)
+    s = np.empty((G, N // TILE, K // TILE), dtype=np.float32)
+    _check(_load().orc_quant_w_128x128_ue8m0(_ptr(w), G, N, K, _ptr(q), _ptr(s)), "quant_w_128x128_ue8m0")
+    return (q[0], s[0]) if squeeze else (q, s)
 
 
 def quant_act_128x1(x_bf16: np.ndarray):

@@ -232,6 +232,66 @@ int orc_quant_tensor(const uint16_t* x, int64_t n, uint8_t* q, float* s_out) {
   return 0;
 }
 
+/* Power-of-two (UE8M0) group scales: the microscaling direction the first
+ * page names for Blackwell ([P1], fine-grained quantization in step with
+ * microscaling formats).  s = 2^e with e the smallest integer such that
+ * 448 * 2^e >= amax (so |x / s| <= 448 and no code saturates), clamped to the
+ * E8M0 range [-127, 127]; amax == 0 gives s = 1.  With amax = m 2^p,
+ * m in [0.5, 1) (frexp), 448 = 0.875 * 2^9 gives e = p - 9 when m <= 0.875
+ * and p - 8 otherwise.  Division by a power of two is exact, so the codes
+ * are E4M3_RNE(x * 2^-e). */
+static int ue8m0_exponent(float amax) {
+  if (amax == 0.0f) return 0;
+  int p;
+  const float m = frexpf(amax, &p);
+  int e = m <= 0.875f ? p - 9 : p - 8;
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return e;
+}
+
+int orc_quant_act_1x128_ue8m0(const uint16_t* x, int64_t M, int64_t K, uint8_t* q, float* s) {
+  if (M < 0 || K < 0 || K % ORC_TILE) return -1;
+  const int64_t nkb = K / ORC_TILE;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t kb = 0; kb < nkb; ++kb) {
+      const uint16_t* xt = x + m * K + kb * ORC_TILE;
+      float amax = 0.0f;
+      for (int j = 0; j < ORC_TILE; ++j) {
+        float a = fabsf(bf16_to_float(xt[j]));
+        if (a > amax) amax = a;
+      }
+      const float sc = ldexpf(1.0f, ue8m0_exponent(amax));
+      s[m * nkb + kb] = sc;
+      for (int j = 0; j < ORC_TILE; ++j) q[m * K + kb * ORC_TILE + j] = orc_e4m3_encode(bf16_to_float(xt[j]) / sc);
+    }
+  }
+  return 0;
+}
+
+int orc_quant_w_128x128_ue8m0(const uint16_t* w, int64_t G, int64_t N, int64_t K, uint8_t* q, float* s) {
+  if (G < 0 || N < 0 || K < 0 || N % ORC_TILE || K % ORC_TILE) return -1;
+  const int64_t nnb = N / ORC_TILE, nkb = K / ORC_TILE;
+#pragma omp parallel for schedule(static)
+  for (int64_t b = 0; b < G * nnb * nkb; ++b) {
+    const int64_t kb = b % nkb, gnb = b / nkb;
+    const uint16_t* wb = w + gnb * ORC_TILE * K + kb * ORC_TILE;
+    uint8_t* qb = q + gnb * ORC_TILE * K + kb * ORC_TILE;
+    float amax = 0.0f;
+    for (int r = 0; r < ORC_TILE; ++r)
+      for (int j = 0; j < ORC_TILE; ++j) {
+        float a = fabsf(bf16_to_float(wb[r * K + j]));
+        if (a > amax) amax = a;
+      }
+    const float sc = ldexpf(1.0f, ue8m0_exponent(amax));
+    s[b] = sc;
+    for (int r = 0; r < ORC_TILE; ++r)
+      for (int j = 0; j < ORC_TILE; ++j) qb[r * K + j] = orc_e4m3_encode(bf16_to_float(wb[r * K + j]) / sc);
+  }
+  return 0;
+}
+
 /* Quantization with a given scale (delayed scaling, which the codingmall page
  * contrasts with online scaling: the scale comes from earlier iterations'
  * maxima, so values beyond 448 * s saturate at +-448).  Used only by the

@@ -9,7 +9,8 @@ push the other values toward FP8's underflow, and that 1x128 / 128x128 groups
 contain that damage (Figure 7 (a)).  The codingmall DeepSeek-V3 FP8 page
 contrasts its online scales (taken from the current values) with delayed
 scaling, which takes the scale from earlier iterations' maxima.  This script
-measures all three on the dense_fprop workload (per-channel log-normal
+measures all three, plus the fine-grained groups with power-of-two (UE8M0)
+scales, on the dense_fprop workload (per-channel log-normal
 activations with +-200 outliers, N(0, 0.02) weights): the error of the
 block-scaled product against the exact product of the unquantized bf16
 inputs, on a seeded sample of rows.
@@ -30,7 +31,8 @@ import time
 
 import numpy as np
 
-from . import TILE, gemm_blockscaled, quant_act_1x128, quant_tensor, quant_w_128x128, quant_with_scale, e4m3_decode_table
+from . import (TILE, e4m3_decode_table, gemm_blockscaled, quant_act_1x128, quant_act_1x128_ue8m0, quant_tensor,
+               quant_w_128x128, quant_w_128x128_ue8m0, quant_with_scale)
 
 
 def _f64(bits: np.ndarray) -> np.ndarray:
@@ -71,6 +73,13 @@ def study(a_bits: np.ndarray, b_bits: np.ndarray, rows: np.ndarray) -> list[dict
     out.append(dict(name="fine-grained 1x128 / 128x128, online",
                     act_err=_dequant_rel_rms(a_bits, qa, np.repeat(sa, TILE, axis=1)),
                     saturated=0, **_errors(gemm_blockscaled(qa, sa, qb, sb, rows), ref)))
+
+    # fine-grained groups with power-of-two (UE8M0) scales, the microscaling variant
+    qa2, sa2 = quant_act_1x128_ue8m0(a_bits)
+    qb2, sb2 = quant_w_128x128_ue8m0(b_bits)
+    out.append(dict(name="fine-grained 1x128 / 128x128, power-of-two (UE8M0) scales",
+                    act_err=_dequant_rel_rms(a_bits, qa2, np.repeat(sa2, TILE, axis=1)),
+                    saturated=0, **_errors(gemm_blockscaled(qa2, sa2, qb2, sb2, rows), ref)))
 
     # per-tensor, online
     qa_t, s_a = quant_tensor(a_bits)

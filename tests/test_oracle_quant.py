@@ -260,3 +260,65 @@ def test_scaling_study_orders_the_schemes(orc):
     assert fine["act_err"] < tensor["act_err"] and fine["fro_rel"] < tensor["fro_rel"]
     assert spike_delayed["fro_rel"] > 3 * spike_fine["fro_rel"]
     assert spike_fine["fro_rel"] < 1.1 * fine["fro_rel"]
+
+
+# --------------------------------------------------------------------------- power-of-two (UE8M0) scales
+@pytest.mark.parametrize("amax,expect", [
+    (448.0, 1.0),                 # 448 * 2^0 >= 448, and 448 * 2^-1 < 448
+    (450.0, 2.0),                 # the next bf16 above 448
+    (1.0, 2.0 ** -8),             # 448 / 256 = 1.75 >= 1 > 0.875 = 448 / 512
+    (224.0, 0.5),                 # exactly 448 * 2^-1
+    (0.0, 1.0),
+    (float(np.float32(3.3895313892515355e38)), 2.0 ** 120),   # largest bf16
+    (2.0 ** -133, 2.0 ** -127),   # smallest bf16 subnormal: exponent clamped to the E8M0 range
+])
+def test_ue8m0_scale_hand_cases(orc, amax, expect):
+    x = np.zeros((1, 128), dtype=np.float32)
+    x[0, 17] = amax
+    x[0, 40] = -amax / 3
+    q, s = orc.quant_act_1x128_ue8m0(bf16_bits(x))
+    assert s[0, 0] == np.float32(expect)
+    if amax > 0:
+        assert orc.e4m3_decode(q[0, 17]) * float(s[0, 0]) <= amax * 1.0625  # within an E4M3 step, never clipped
+
+
+def test_ue8m0_scales_are_the_least_power_of_two_cover(orc):
+    d = tiny_dense()
+    for quant, per_group in ((orc.quant_act_1x128_ue8m0, "act"), (orc.quant_w_128x128_ue8m0, "w")):
+        src = d.a if per_group == "act" else d.b
+        q, s = quant(src)
+        f = bf16_to_f32(src).astype(np.float64)
+        if per_group == "act":
+            amax = np.abs(f).reshape(f.shape[0], -1, 128).max(axis=2)
+        else:
+            n, k = f.shape
+            amax = np.abs(f).reshape(n // 128, 128, k // 128, 128).max(axis=(1, 3))
+        s64 = s.astype(np.float64)
+        mant, _ = np.frexp(s64)
+        assert np.all(mant == 0.5), "every scale is a power of two"
+        assert np.all(448.0 * s64 >= amax)
+        assert np.all((224.0 * s64 < amax) | (amax == 0))
+        # no saturation: every code is exactly the RNE code of x / s (an exact quotient)
+        reps = np.repeat(s64, 128, axis=1) if per_group == "act" else np.repeat(np.repeat(s64, 128, 0), 128, 1)
+        expect = orc.e4m3_encode_array((f / reps).astype(np.float32))
+        assert np.array_equal(q, expect.reshape(q.shape))
+
+
+def test_ue8m0_vs_fp32_scales(orc):
+    """The power-of-two scale is the fp32 scale rounded up to a power of two."""
+    d = tiny_dense()
+    _, s2 = orc.quant_act_1x128_ue8m0(d.a)
+    _, s32 = orc.quant_act_1x128(d.a)
+    assert np.all(s2 >= s32) and np.all(s2 < 2 * s32)
+
+
+def test_ue8m0_all_ones_gemm_is_exact(orc):
+    """All-ones operands: every scale is 2^-8, every code is 256 (0x78), and the
+    block-scaled product is exactly K (no rounding anywhere)."""
+    M, N, K = 4, 256, 640
+    a = np.full((M, K), 0x3F80, dtype=np.uint16)
+    b = np.full((N, K), 0x3F80, dtype=np.uint16)
+    qa, sa = orc.quant_act_1x128_ue8m0(a)
+    qb, sb = orc.quant_w_128x128_ue8m0(b)
+    assert np.all(qa == 0x78) and np.all(sa == 2.0 ** -8) and np.all(sb == 2.0 ** -8)
+    assert np.all(orc.gemm_blockscaled(qa, sa, qb, sb) == float(K))
