@@ -70,6 +70,10 @@ def _load():
     lib.orc_quant_act_1x128_ue8m0.restype = ctypes.c_int
     lib.orc_quant_w_128x128_ue8m0.argtypes = [P, I64, I64, I64, P, P]
     lib.orc_quant_w_128x128_ue8m0.restype = ctypes.c_int
+    lib.orc_round_bf16.argtypes = [P, I64, P]
+    lib.orc_round_bf16.restype = None
+    lib.orc_swiglu_bf16.argtypes = [P, I64, I64, P]
+    lib.orc_swiglu_bf16.restype = ctypes.c_int
     lib.orc_quant_act_128x1.argtypes = [P, I64, I64, P, P]
     lib.orc_quant_act_128x1.restype = ctypes.c_int
     lib.orc_gemm_1d1d.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
@@ -276,6 +280,43 @@ def dgrad(q_dy, s_dy, q_w, s_w, rows=None) -> np.ndarray:
     """dX [M,K] = dY W from 1x128-quantized dY [M,N] and 128x128-quantized
     W [N,K]: the forward GEMM with W's codes and block scales transposed."""
     return gemm_blockscaled(q_dy, s_dy, np.ascontiguousarray(q_w.T), np.ascontiguousarray(s_w.T), rows)
+
+
+def round_bf16(v: np.ndarray) -> np.ndarray:
+    """float64 values -> bf16 bit patterns, one round-to-nearest-even step."""
+    x = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(x.shape, dtype=np.uint16)
+    _load().orc_round_bf16(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def masked_moe_chain(a_bits, b1_bits, b2_bits, masked_m) -> np.ndarray:
+    """The masked MoE decode as one chain: 1x128 quantization of A [E,cap,K1], masked
+    GEMM1 with 128x128-quantized B1 [E,2I,K1], bf16 rounding of its output,
+    SwiGLU, 1x128 requantization, masked GEMM2 with B2 [E,N2,I].  Returns the
+    float64 GEMM2 output [E,cap,N2]; rows at or past masked_m[e] are NaN."""
+    E, cap, K1 = a_bits.shape
+    qa, sa = quant_act_1x128(a_bits.reshape(E * cap, K1))
+    qb1, sb1 = quant_w_128x128(b1_bits)
+    c1 = grouped_masked(qa.reshape(E, cap, K1), sa.reshape(E, cap, K1 // TILE), qb1, sb1, masked_m)
+    c1 = np.where(np.isnan(c1), 0.0, c1)  # rows past the count never reach GEMM2's valid rows
+    h = swiglu_bf16(round_bf16(c1))
+    inter = h.shape[-1]
+    qh, sh = quant_act_1x128(h.reshape(E * cap, inter))
+    qb2, sb2 = quant_w_128x128(b2_bits)
+    return grouped_masked(qh.reshape(E, cap, inter), sh.reshape(E, cap, inter // TILE), qb2, sb2, masked_m)
+
+
+def swiglu_bf16(c1_bf16: np.ndarray) -> np.ndarray:
+    """[.., 2I] bf16 bits ([gate | up]) -> [.., I] bf16 bits of silu(gate) * up (double, one rounding)."""
+    c1 = _bf16(c1_bf16)
+    inter = c1.shape[-1] // 2
+    if c1.shape[-1] != 2 * inter:
+        raise ValueError("oracle: the last dimension must be even ([gate | up])")
+    rows = c1.size // (2 * inter) if inter else 0
+    h = np.empty(c1.shape[:-1] + (inter,), dtype=np.uint16)
+    _check(_load().orc_swiglu_bf16(_ptr(c1), rows, inter, _ptr(h)), "swiglu_bf16")
+    return h
 
 
 def grouped_contiguous(qa, sa, qb, sb, m_indices, rows=None, out=None) -> np.ndarray:

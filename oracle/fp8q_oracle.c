@@ -303,6 +303,52 @@ int orc_quant_with_scale(const uint16_t* x, int64_t n, float s, uint8_t* q) {
   return 0;
 }
 
+/* Round a double to the nearest bf16 (ties to even) in one step, without an
+ * intermediate float (which could round twice).  Finite inputs only; values
+ * beyond the bf16 range become +-inf. */
+static uint16_t double_to_bf16_rne(double v) {
+  if (v == 0.0) return signbit(v) ? 0x8000 : 0x0000;
+  const uint16_t sign = v < 0 ? 0x8000 : 0x0000;
+  double a = fabs(v);
+  int e;
+  (void)frexp(a, &e);  /* a = m 2^e, m in [0.5, 1) */
+  /* bf16 normal: 8 significant bits (1 + 7), exponents 2^-126 .. 2^127 */
+  int ulp_exp = e - 8;      /* weight of the last kept bit for a normal */
+  if (e - 1 < -126) ulp_exp = -126 - 7;  /* subnormal spacing 2^-133 */
+  double q = ldexp(a, -ulp_exp);  /* value in units of the last kept bit (exact) */
+  double r = floor(q);
+  double frac = q - r;
+  if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) == 1.0)) r += 1.0;
+  double y = ldexp(r, ulp_exp);
+  if (y > 3.3895313892515355e38) return sign | 0x7F80;  /* overflow: inf */
+  float f = (float)y;  /* exact: y has at most 8 significant bits */
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  return sign | (uint16_t)(u >> 16);
+}
+
+/* A double array rounded once to bf16 bit patterns (RNE). */
+void orc_round_bf16(const double* v, int64_t n, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = double_to_bf16_rne(v[i]);
+}
+
+/* SwiGLU between the two MoE GEMMs (not on the pages: the configurations'
+ * GEMM1 width N = 4096 = 2 x 2048 = GEMM2's K implies it): c1 holds
+ * [gate | up] halves of each row, h = silu(gate) * up with silu(g) =
+ * g / (1 + exp(-g)), computed in double from the bf16 inputs and rounded once
+ * to bf16.  rows x (2 inter) in, rows x inter out. */
+int orc_swiglu_bf16(const uint16_t* c1, int64_t rows, int64_t inter, uint16_t* h) {
+  if (rows < 0 || inter < 0) return -1;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t i = 0; i < inter; ++i) {
+      const double g = bf16_to_float(c1[r * 2 * inter + i]);
+      const double u = bf16_to_float(c1[r * 2 * inter + inter + i]);
+      h[r * inter + i] = double_to_bf16_rne(g / (1.0 + exp(-g)) * u);
+    }
+  return 0;
+}
+
 /* ---------------------------------------------------------------------------
  * Block-scaled GEMM, C = A * B^T with per-slab promotion ([P1] Figure 7 (b);
  * [P3] increased accumulation precision):
