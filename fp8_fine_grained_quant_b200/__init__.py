@@ -11,6 +11,7 @@ Names and semantics match the C entry points:
 * :func:`fp8_quant_act_1x128`  -- bf16 [M,K] -> E4M3 [M,K] + f32 scales [M,K/128]
 * :func:`fp8_quant_w_128x128`  -- bf16 [N,K] or [G,N,K] -> E4M3 + f32 scales [..,N/128,K/128]
 * :func:`fp8_quant_act_128x1`  -- bf16 [M,K] -> E4M3 [M,K] + f32 scales [ceil(M/128),K] (token-axis tiles)
+* :func:`fp8_quant_act_1x128_ue8m0`, :func:`fp8_quant_w_128x128_ue8m0` -- the same groups, power-of-two scales
 * :func:`fp8_transpose_w_128x128` -- block-quantized W [..,N,K] -> W^T [..,K,N] (codes and block scales)
 * :func:`fp8_gemm_blockscaled` -- C = A * B^T (bf16) with per-128-slab promotion
 * :func:`fp8_grouped_gemm_contiguous` -- MoE grouped GEMM, contiguous layout
@@ -25,6 +26,7 @@ import torch
 
 __all__ = [
     "fp8_quant_act_1x128", "fp8_quant_w_128x128", "fp8_quant_act_128x1", "fp8_transpose_w_128x128",
+    "fp8_quant_act_1x128_ue8m0", "fp8_quant_w_128x128_ue8m0",
     "fp8_gemm_blockscaled", "fp8_grouped_gemm_contiguous",
     "fp8_grouped_gemm_masked", "fp8_gemm_unpromoted_diag", "get_device_error", "set_wait_timeout_ns",
     "selftest_wait_timeout", "launch_count", "status_string", "Fp8qError", "lib", "LIB_PATH", "EXPORTS",
@@ -42,6 +44,8 @@ EXPORTS = {
     "fp8_quant_act_1x128": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
     "fp8_quant_w_128x128": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "fp8_quant_act_128x1": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
+    "fp8_quant_act_1x128_ue8m0": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
+    "fp8_quant_w_128x128_ue8m0": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "fp8_transpose_w_128x128": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P]),
     "fp8_gemm_blockscaled": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "fp8_grouped_gemm_contiguous": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
@@ -118,7 +122,8 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
-def fp8_quant_act_1x128(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None, stream=None):
+def fp8_quant_act_1x128(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None, stream=None,
+                        _entry: str = "fp8_quant_act_1x128"):
     """Online 1x128 activation quantization.  Returns (q [M,K] float8_e4m3fn, s [M,K/128] f32)."""
     _dev(x, "x", _BF16, (2,))
     M, K = x.shape
@@ -131,11 +136,12 @@ def fp8_quant_act_1x128(x: torch.Tensor, q: torch.Tensor | None = None, s: torch
     if q.numel() != M * K or s.numel() != M * (K // TILE):
         raise ValueError("output sizes do not match x")
     with torch.cuda.device(x.device):
-        _check(lib().fp8_quant_act_1x128(_p(x), M, K, _p(q), _p(s), _stream(stream, x.device)), "fp8_quant_act_1x128")
+        _check(getattr(lib(), _entry)(_p(x), M, K, _p(q), _p(s), _stream(stream, x.device)), _entry)
     return q, s
 
 
-def fp8_quant_w_128x128(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None, stream=None):
+def fp8_quant_w_128x128(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None, stream=None,
+                        _entry: str = "fp8_quant_w_128x128"):
     """Online 128x128 weight quantization of [N,K] or [G,N,K] bf16."""
     _dev(w, "w", _BF16, (2, 3))
     G, N, K = (1,) + tuple(w.shape) if w.dim() == 2 else tuple(w.shape)
@@ -149,9 +155,18 @@ def fp8_quant_w_128x128(w: torch.Tensor, q: torch.Tensor | None = None, s: torch
     if q.numel() != G * N * K or s.numel() != G * (N // TILE) * (K // TILE):
         raise ValueError("output sizes do not match w")
     with torch.cuda.device(w.device):
-        _check(lib().fp8_quant_w_128x128(_p(w), G, N, K, _p(q), _p(s), _stream(stream, w.device)),
-               "fp8_quant_w_128x128")
+        _check(getattr(lib(), _entry)(_p(w), G, N, K, _p(q), _p(s), _stream(stream, w.device)), _entry)
     return q, s
+
+
+def fp8_quant_act_1x128_ue8m0(x, q=None, s=None, stream=None):
+    """1x128 activation quantization with power-of-two (UE8M0) scales."""
+    return fp8_quant_act_1x128(x, q, s, stream, _entry="fp8_quant_act_1x128_ue8m0")
+
+
+def fp8_quant_w_128x128_ue8m0(w, q=None, s=None, stream=None):
+    """128x128 weight quantization with power-of-two (UE8M0) scales."""
+    return fp8_quant_w_128x128(w, q, s, stream, _entry="fp8_quant_w_128x128_ue8m0")
 
 
 def fp8_quant_act_128x1(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None, stream=None):

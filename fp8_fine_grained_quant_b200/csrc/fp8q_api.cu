@@ -246,9 +246,8 @@ __global__ void wait_selftest_kernel(uint32_t* status, uint64_t timeout_ns) {
 
 using namespace fp8q;
 
-extern "C" {
-
-int fp8_quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
+template <bool kPow2>
+static int quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
   if (M < 0 || K < 0 || K % 128) return FP8Q_ERR_SHAPE;
   if (M == 0 || K == 0) return FP8Q_OK;
   if (!x_bf16 || !q || !s) return FP8Q_ERR_NULL;
@@ -262,15 +261,16 @@ int fp8_quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, fl
   int64_t grid = (tiles + per_cta - 1) / per_cta;
   const int64_t cap = static_cast<int64_t>(dev->num_sms) * 10;  // two full waves of 5 resident CTAs per SM
   if (grid > cap) grid = cap;
-  quant_act_1x128_kernel<kUnroll><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+  quant_act_1x128_kernel<kUnroll, kPow2><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
       static_cast<const uint8_t*>(x_bf16), q, s, tiles);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FP8Q_OK;
 }
 
-int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, uint8_t* q, float* s,
-                        cudaStream_t stream) {
+template <bool kPow2>
+static int quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, uint8_t* q, float* s,
+                           cudaStream_t stream) {
   if (G < 0 || N < 0 || K < 0 || N % 128 || K % 128) return FP8Q_ERR_SHAPE;
   if (G == 0 || N == 0 || K == 0) return FP8Q_OK;
   if (!w_bf16 || !q || !s) return FP8Q_ERR_NULL;
@@ -281,11 +281,31 @@ int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, uin
   const int64_t blocks = G * (N / 128) * (K / 128);
   const int64_t cap = static_cast<int64_t>(dev->num_sms) * 64;
   const int64_t grid = blocks < cap ? blocks : cap;
-  quant_w_128x128_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(static_cast<const uint8_t*>(w_bf16), q, s,
+  quant_w_128x128_kernel<kPow2><<<static_cast<unsigned>(grid), 256, 0, stream>>>(static_cast<const uint8_t*>(w_bf16), q, s,
                                                                            K, blocks);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FP8Q_OK;
+}
+
+extern "C" {
+
+int fp8_quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
+  return quant_act_1x128<false>(x_bf16, M, K, q, s, stream);
+}
+
+int fp8_quant_act_1x128_ue8m0(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
+  return quant_act_1x128<true>(x_bf16, M, K, q, s, stream);
+}
+
+int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, uint8_t* q, float* s,
+                        cudaStream_t stream) {
+  return quant_w_128x128<false>(w_bf16, G, N, K, q, s, stream);
+}
+
+int fp8_quant_w_128x128_ue8m0(const void* w_bf16, int64_t G, int64_t N, int64_t K, uint8_t* q, float* s,
+                              cudaStream_t stream) {
+  return quant_w_128x128<true>(w_bf16, G, N, K, q, s, stream);
 }
 
 int fp8_quant_act_128x1(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {

@@ -112,6 +112,32 @@ __device__ __forceinline__ void zero8(uint32_t (&w)[8]) {
   for (int i = 0; i < 8; ++i) w[i] = 0u;
 }
 
+// Power-of-two (UE8M0) group scales, the microscaling form the first page
+// names for Blackwell: s = 2^e with e the least integer such that
+// 448 * 2^e >= amax (so no code saturates), clamped to E8M0's [-127, 127];
+// amax == 0 gives 1.  With amax = 1.f * 2^(E-127) (E the biased exponent),
+// 448 = 1.75 * 2^8 gives e = E - 135 when 1.f <= 1.75 and E - 134 otherwise;
+// a subnormal amax clamps to e = -127.  Returns 2^-e (the exact multiplier).
+__device__ __forceinline__ float pow2_scale(float amax, float* inv) {
+  const uint32_t b = __float_as_uint(amax);
+  const int E = static_cast<int>(b >> 23);
+  int e = E == 0 ? -127 : ((b & 0x7FFFFFu) <= 0x600000u ? E - 135 : E - 134);
+  if (amax == 0.0f) e = 0;
+  e = e < -127 ? -127 : (e > 127 ? 127 : e);
+  *inv = e <= 126 ? __uint_as_float(static_cast<uint32_t>(127 - e) << 23) : 0x1p-127f;  // 2^-e
+  return e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23) : 0x1p-127f;
+}
+
+// 16 bf16 -> 16 codes of x * 2^-e (exact products: one conversion each).
+__device__ __forceinline__ uint4 quantize16_pow2(const uint32_t (&w)[8], float inv) {
+  const uint64_t inv2 = pack_f32x2(inv);
+  uint32_t c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    c[i] = e4m3x4_from_f32x2(mul_f32x2(bf16x2_to_f32x2(w[2 * i]), inv2), mul_f32x2(bf16x2_to_f32x2(w[2 * i + 1]), inv2));
+  return make_uint4(c[0], c[1], c[2], c[3]);
+}
+
 // ---------------------------------------------------------------------------
 // 1x128 activation tiles.  A tile is 128 bf16 = 256 contiguous bytes; eight
 // lanes (32 bytes each) own one tile per step, so a warp covers four tiles.
@@ -119,7 +145,7 @@ __device__ __forceinline__ void zero8(uint32_t (&w)[8]) {
 // s[M, K/128].  Each lane group handles kUnroll tiles per iteration (loads
 // issued together) in a grid-stride loop; five CTAs fit per SM.
 // ---------------------------------------------------------------------------
-template <int kUnroll>
+template <int kUnroll, bool kPow2>
 __global__ void __launch_bounds__(256, 5) quant_act_1x128_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
                                                               float* __restrict__ s, int64_t num_tiles) {
   const int sub = threadIdx.x & 7;
@@ -143,11 +169,20 @@ __global__ void __launch_bounds__(256, 5) quant_act_1x128_kernel(const uint8_t* 
       float amax = abs_max16(v[u]);
 #pragma unroll
       for (int off = 4; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-      const float sc = group_scale(amax);
-      const RecipPair rp = recip_pair(sc);
-      if (t < num_tiles) {
-        *reinterpret_cast<uint4*>(q + t * 128 + sub * 16) = quantize16(v[u], sc, rp, sc < kMinFastScale);
-        if (sub == 0) s[t] = sc;
+      if constexpr (kPow2) {
+        float inv;
+        const float sc = pow2_scale(amax, &inv);
+        if (t < num_tiles) {
+          *reinterpret_cast<uint4*>(q + t * 128 + sub * 16) = quantize16_pow2(v[u], inv);
+          if (sub == 0) s[t] = sc;
+        }
+      } else {
+        const float sc = group_scale(amax);
+        const RecipPair rp = recip_pair(sc);
+        if (t < num_tiles) {
+          *reinterpret_cast<uint4*>(q + t * 128 + sub * 16) = quantize16(v[u], sc, rp, sc < kMinFastScale);
+          if (sub == 0) s[t] = sc;
+        }
       }
     }
   }
@@ -161,6 +196,7 @@ __global__ void __launch_bounds__(256, 5) quant_act_1x128_kernel(const uint8_t* 
 // local memory).  Block b = (g * N/128 + nb) * K/128 + kb, also the index of
 // its scale in s[G, N/128, K/128].  Grid-stride over blocks.
 // ---------------------------------------------------------------------------
+template <bool kPow2>
 __global__ void __launch_bounds__(256, 4) quant_w_128x128_kernel(const uint8_t* __restrict__ w,
                                                                  uint8_t* __restrict__ q, float* __restrict__ s,
                                                                  int64_t K, int64_t num_blocks) {
@@ -187,13 +223,22 @@ __global__ void __launch_bounds__(256, 4) quant_w_128x128_kernel(const uint8_t* 
     amax = warp_max[half][0];
 #pragma unroll
     for (int i = 1; i < 8; ++i) amax = fmaxf(amax, warp_max[half][i]);
-    const float sc = group_scale(amax);
-    const RecipPair rp = recip_pair(sc);
-    const bool exact_only = sc < kMinFastScale;
     uint8_t* dst = q + row0 * K + kb * 128 + sub * 16;
+    float sc;
+    if constexpr (kPow2) {
+      float inv;
+      sc = pow2_scale(amax, &inv);
 #pragma unroll
-    for (int p = 0; p < 4; ++p)
-      *reinterpret_cast<uint4*>(dst + (p * 32 + rsub) * K) = quantize16(v[p], sc, rp, exact_only);
+      for (int p = 0; p < 4; ++p)
+        *reinterpret_cast<uint4*>(dst + (p * 32 + rsub) * K) = quantize16_pow2(v[p], inv);
+    } else {
+      sc = group_scale(amax);
+      const RecipPair rp = recip_pair(sc);
+      const bool exact_only = sc < kMinFastScale;
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        *reinterpret_cast<uint4*>(dst + (p * 32 + rsub) * K) = quantize16(v[p], sc, rp, exact_only);
+    }
     if (tid == 0) s[b] = sc;
   }
 }

@@ -89,6 +89,22 @@ FP8Q_API int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64
                         cudaStream_t stream);
 
 /*
+ * The same two quantizers with power-of-two (UE8M0) group scales: the
+ * microscaling form the first page names for Blackwell ("The Insider Secrets
+ * Of Deepseek Discovered", fine-grained quantization in step with
+ * microscaling formats).  s = 2^e with e the least integer such that
+ * 448 * 2^e >= amax, clamped to [-127, 127] (amax == 0: s = 1), so no code
+ * saturates and q = E4M3_RNE(x * 2^-e) exactly.  Scales are written as
+ * float32 powers of two, in the same layouts as above, so the GEMMs accept
+ * them unchanged.  Same shapes, alignment and errors as the entry points
+ * above.
+ */
+FP8Q_API int fp8_quant_act_1x128_ue8m0(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s,
+                                       cudaStream_t stream);
+FP8Q_API int fp8_quant_w_128x128_ue8m0(const void* w_bf16, int64_t G, int64_t N, int64_t K, uint8_t* q, float* s,
+                                       cudaStream_t stream);
+
+/*
  * Activation quantization along the token axis, 128x1 tiles (for the weight
  * gradient dW = dY^T X, which contracts over tokens; "The Insider Secrets Of
  * Deepseek Discovered", Figure 6: Fprop, Dgrad and Wgrad all run in FP8).

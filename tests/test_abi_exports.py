@@ -157,3 +157,14 @@ def test_quant_act_128x1_validation(args, expect):
 ])
 def test_transpose_w_validation(args, expect):
     assert _call("fp8_transpose_w_128x128", *args) == expect
+
+
+@pytest.mark.parametrize("name,args,expect", [
+    ("fp8_quant_act_1x128_ue8m0", (A16, 4, 100, A16, A16, None), fq.ERR_SHAPE),
+    ("fp8_quant_act_1x128_ue8m0", (A16_ONLY, 4, 128, A16, A16, None), fq.ERR_ALIGN),
+    ("fp8_quant_act_1x128_ue8m0", (A16, 0, 128, A16, A16, None), fq.OK),
+    ("fp8_quant_w_128x128_ue8m0", (A16, 1, 100, 128, A16, A16, None), fq.ERR_SHAPE),
+    ("fp8_quant_w_128x128_ue8m0", (None, 1, 128, 128, A16, A16, None), fq.ERR_NULL),
+])
+def test_ue8m0_quant_validation(name, args, expect):
+    assert _call(name, *args) == expect

@@ -224,3 +224,37 @@ def test_every_16th_bf16_amax_w(dev):
         blocks[i, 1:] = wl.bf16_bits(rows)
     w = blocks.reshape(nb * TILE, TILE)   # G = 1, N = 128 * nb, K = 128
     assert_w_exact(w, dev)
+
+
+# --------------------------------------------------------------------------- power-of-two (UE8M0) scales
+@pytest.mark.parametrize("M,K", [(300, 384), (1, 128), (4096, 7168)])
+def test_ue8m0_act_matches_oracle(dev, M, K):
+    rng = np.random.default_rng(M + K)
+    x = wl.bf16_bits((rng.standard_normal((M, K)) * np.exp(rng.standard_normal(K))).astype(np.float32))
+    x[0, :] = 0
+    q, s = fq.fp8_quant_act_1x128_ue8m0(to_torch_bf16(x, dev))
+    torch.cuda.synchronize(dev)
+    oq, os_ = oracle.quant_act_1x128_ue8m0(x)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+    assert np.array_equal(bytes_of(q).reshape(M, K), oq)
+
+
+def test_ue8m0_every_bf16_amax(dev):
+    x = _tiles_with_every_amax()
+    x2 = x.reshape(255, 128 * TILE)
+    q, s = fq.fp8_quant_act_1x128_ue8m0(to_torch_bf16(x2, dev))
+    torch.cuda.synchronize(dev)
+    oq, os_ = oracle.quant_act_1x128_ue8m0(x2)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+    assert np.array_equal(bytes_of(q).reshape(oq.shape), oq)
+
+
+@pytest.mark.parametrize("G,N,K", [(1, 256, 384), (3, 128, 256)])
+def test_ue8m0_w_matches_oracle(dev, G, N, K):
+    rng = np.random.default_rng(G + N + K)
+    w = wl.bf16_bits((0.02 * rng.standard_normal((G, N, K))).astype(np.float32))
+    q, s = fq.fp8_quant_w_128x128_ue8m0(to_torch_bf16(w, dev))
+    torch.cuda.synchronize(dev)
+    oq, os_ = oracle.quant_w_128x128_ue8m0(w)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+    assert np.array_equal(bytes_of(q).reshape(oq.shape), oq)
