@@ -9,6 +9,7 @@ import re
 from pathlib import Path
 
 import pytest
+import torch
 
 import fp8_fine_grained_quant_b200 as fq
 
@@ -168,3 +169,18 @@ def test_transpose_w_validation(args, expect):
 ])
 def test_ue8m0_quant_validation(name, args, expect):
     assert _call(name, *args) == expect
+
+
+@pytest.mark.parametrize("call", [
+    lambda: fq.fp8_quant_act_1x128(torch.zeros((4, 128), dtype=torch.bfloat16)),
+    lambda: fq.fp8_quant_w_128x128(torch.zeros((128, 128), dtype=torch.bfloat16)),
+    lambda: fq.fp8_quant_act_128x1(torch.zeros((4, 128), dtype=torch.bfloat16)),
+    lambda: fq.fp8_quant_act_1x128_ue8m0(torch.zeros((4, 128), dtype=torch.bfloat16)),
+    lambda: fq.fp8_gemm_blockscaled(torch.zeros((4, 128), dtype=torch.uint8), torch.ones((4, 1)),
+                                    torch.zeros((128, 128), dtype=torch.uint8), torch.ones((1, 1))),
+    lambda: fq.fp8_transpose_w_128x128(torch.zeros((128, 128), dtype=torch.uint8), torch.ones((1, 1))),
+])
+def test_no_cpu_fallback(call):
+    """Host tensors are refused before anything runs: there is no CPU path."""
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        call()
