@@ -11,6 +11,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "fp8q.h"
 #include "fp8q_gemm.cuh"
 #include "fp8q_ptx.cuh"
@@ -246,6 +248,19 @@ __global__ void wait_selftest_kernel(uint32_t* status, uint64_t timeout_ns) {
 
 using namespace fp8q;
 
+// An NVTX range named after the entry point around each call that launches
+// work, so profilers show the library's calls on the host timeline (a no-op
+// when no tool is attached).
+namespace {
+struct ApiRange {
+  explicit ApiRange(const char* name) { nvtxRangePushA(name); }
+  ~ApiRange() { nvtxRangePop(); }
+  ApiRange(const ApiRange&) = delete;
+  ApiRange& operator=(const ApiRange&) = delete;
+};
+}  // namespace
+#define FP8Q_API_RANGE() ApiRange fp8q_api_range_(__func__)
+
 template <bool kPow2>
 static int quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
   if (M < 0 || K < 0 || K % 128) return FP8Q_ERR_SHAPE;
@@ -291,24 +306,29 @@ static int quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, 
 extern "C" {
 
 int fp8_quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
+  FP8Q_API_RANGE();
   return quant_act_1x128<false>(x_bf16, M, K, q, s, stream);
 }
 
 int fp8_quant_act_1x128_ue8m0(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
+  FP8Q_API_RANGE();
   return quant_act_1x128<true>(x_bf16, M, K, q, s, stream);
 }
 
 int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, uint8_t* q, float* s,
                         cudaStream_t stream) {
+  FP8Q_API_RANGE();
   return quant_w_128x128<false>(w_bf16, G, N, K, q, s, stream);
 }
 
 int fp8_quant_w_128x128_ue8m0(const void* w_bf16, int64_t G, int64_t N, int64_t K, uint8_t* q, float* s,
                               cudaStream_t stream) {
+  FP8Q_API_RANGE();
   return quant_w_128x128<true>(w_bf16, G, N, K, q, s, stream);
 }
 
 int fp8_quant_act_128x1(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
+  FP8Q_API_RANGE();
   if (M < 0 || K < 0 || K % 128) return FP8Q_ERR_SHAPE;
   if (M == 0 || K == 0) return FP8Q_OK;
   if (!x_bf16 || !q || !s) return FP8Q_ERR_NULL;
@@ -328,6 +348,7 @@ int fp8_quant_act_128x1(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, fl
 
 int fp8_transpose_w_128x128(const uint8_t* q, const float* s, int64_t G, int64_t N, int64_t K, uint8_t* qt,
                             float* st, cudaStream_t stream) {
+  FP8Q_API_RANGE();
   if (G < 0 || N < 0 || K < 0 || N % 128 || K % 128) return FP8Q_ERR_SHAPE;
   if (G == 0 || N == 0 || K == 0) return FP8Q_OK;
   if (!q || !s || !qt || !st) return FP8Q_ERR_NULL;
@@ -357,17 +378,20 @@ static int dense_common(const uint8_t* qa, const float* sa, const uint8_t* qb, c
 
 int fp8_gemm_blockscaled(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, void* c_bf16,
                          int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+  FP8Q_API_RANGE();
   return dense_common(qa, sa, qb, sb, c_bf16, M, N, K, 1, stream);
 }
 
 int fp8_gemm_unpromoted_diag(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb, void* c_bf16,
                              int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+  FP8Q_API_RANGE();
   return dense_common(qa, sa, qb, sb, c_bf16, M, N, K, 0, stream);
 }
 
 int fp8_grouped_gemm_contiguous(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb,
                                 const int32_t* m_indices, void* c_bf16, int64_t M_tot, int64_t N, int64_t K,
                                 int64_t E, cudaStream_t stream) {
+  FP8Q_API_RANGE();
   if (M_tot < 0 || N < 0 || E < 0 || K < 128 || K % 128 || N % 128 || M_tot % 128 || M_tot >= kMaxRows ||
       K >= kMaxRows || E * N >= kMaxRows)
     return FP8Q_ERR_SHAPE;
@@ -384,6 +408,7 @@ int fp8_grouped_gemm_contiguous(const uint8_t* qa, const float* sa, const uint8_
 int fp8_grouped_gemm_masked(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb,
                             const int32_t* masked_m, void* c_bf16, int64_t E, int64_t cap, int64_t N, int64_t K,
                             int64_t expected_m, cudaStream_t stream) {
+  FP8Q_API_RANGE();
   if (E < 0 || cap < 0 || N < 0 || K < 128 || K % 128 || N % 128 || cap % 128 || E > kMaxMaskedExperts ||
       E * cap >= kMaxRows || E * N >= kMaxRows || K >= kMaxRows || expected_m < 0)
     return FP8Q_ERR_SHAPE;
@@ -428,6 +453,7 @@ int fp8q_set_wait_timeout_ns(uint64_t timeout_ns) {
 }
 
 int fp8q_selftest_wait_timeout(uint64_t timeout_ns, cudaStream_t stream) {
+  FP8Q_API_RANGE();
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);
   if (rc) return rc;
