@@ -98,11 +98,13 @@ def _stream(stream, device) -> int:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def _dev(t: torch.Tensor, name: str, dtypes, ndim=None) -> torch.Tensor:
+def _tensor(t, name: str, dtypes, ndim=None):
+    """Type, dtype, rank and layout of one argument (the device is checked
+    once for all arguments by :func:`_device_of`)."""
+    if t is None:
+        return None
     if not isinstance(t, torch.Tensor):
         raise TypeError("%s must be a torch.Tensor" % name)
-    if not t.is_cuda:
-        raise ValueError("%s must be a CUDA tensor" % name)
     if t.dtype not in dtypes:
         raise TypeError("%s: dtype %s not in %s" % (name, t.dtype, dtypes))
     if ndim is not None and t.dim() not in ndim:
@@ -110,6 +112,28 @@ def _dev(t: torch.Tensor, name: str, dtypes, ndim=None) -> torch.Tensor:
     if not t.is_contiguous():
         raise ValueError("%s must be contiguous" % name)
     return t
+
+
+def _numel(t, n: int, name: str):
+    """A caller-supplied buffer must hold exactly the elements the call reads
+    or writes: the C library trusts the sizes it is given."""
+    if t is not None and t.numel() != n:
+        raise ValueError("%s holds %d elements, the call needs %d" % (name, t.numel(), n))
+
+
+def _device_of(**tensors) -> torch.device:
+    """All tensors are CUDA tensors on one device (there is no CPU path)."""
+    dev = None
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("%s must be a CUDA tensor" % name)
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("%s is on %s, the other arguments on %s" % (name, t.device, dev))
+    return dev
 
 
 _FP8 = (torch.float8_e4m3fn, torch.uint8)
@@ -122,40 +146,50 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
+def _multiple(v: int, name: str):
+    if v % TILE:
+        raise ValueError("%s = %d is not a multiple of %d" % (name, v, TILE))
+
+
 def fp8_quant_act_1x128(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None, stream=None,
                         _entry: str = "fp8_quant_act_1x128"):
     """Online 1x128 activation quantization.  Returns (q [M,K] float8_e4m3fn, s [M,K/128] f32)."""
-    _dev(x, "x", _BF16, (2,))
+    _tensor(x, "x", _BF16, (2,))
     M, K = x.shape
+    _multiple(K, "K")
+    _tensor(q, "q", _FP8)
+    _tensor(s, "s", _F32)
+    _numel(q, M * K, "q")
+    _numel(s, M * (K // TILE), "s")
+    dev = _device_of(x=x, q=q, s=s)
     if q is None:
-        q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+        q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev)
     if s is None:
-        s = torch.empty((M, K // TILE), dtype=torch.float32, device=x.device)
-    _dev(q, "q", _FP8)
-    _dev(s, "s", _F32)
-    if q.numel() != M * K or s.numel() != M * (K // TILE):
-        raise ValueError("output sizes do not match x")
-    with torch.cuda.device(x.device):
-        _check(getattr(lib(), _entry)(_p(x), M, K, _p(q), _p(s), _stream(stream, x.device)), _entry)
+        s = torch.empty((M, K // TILE), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(getattr(lib(), _entry)(_p(x), M, K, _p(q), _p(s), _stream(stream, dev)), _entry)
     return q, s
 
 
 def fp8_quant_w_128x128(w: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None, stream=None,
                         _entry: str = "fp8_quant_w_128x128"):
     """Online 128x128 weight quantization of [N,K] or [G,N,K] bf16."""
-    _dev(w, "w", _BF16, (2, 3))
+    _tensor(w, "w", _BF16, (2, 3))
     G, N, K = (1,) + tuple(w.shape) if w.dim() == 2 else tuple(w.shape)
+    _multiple(N, "N")
+    _multiple(K, "K")
     lead = tuple(w.shape[:-2])
+    _tensor(q, "q", _FP8)
+    _tensor(s, "s", _F32)
+    _numel(q, G * N * K, "q")
+    _numel(s, G * (N // TILE) * (K // TILE), "s")
+    dev = _device_of(w=w, q=q, s=s)
     if q is None:
-        q = torch.empty(tuple(w.shape), dtype=torch.float8_e4m3fn, device=w.device)
+        q = torch.empty(tuple(w.shape), dtype=torch.float8_e4m3fn, device=dev)
     if s is None:
-        s = torch.empty(lead + (N // TILE, K // TILE), dtype=torch.float32, device=w.device)
-    _dev(q, "q", _FP8)
-    _dev(s, "s", _F32)
-    if q.numel() != G * N * K or s.numel() != G * (N // TILE) * (K // TILE):
-        raise ValueError("output sizes do not match w")
-    with torch.cuda.device(w.device):
-        _check(getattr(lib(), _entry)(_p(w), G, N, K, _p(q), _p(s), _stream(stream, w.device)), _entry)
+        s = torch.empty(lead + (N // TILE, K // TILE), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(getattr(lib(), _entry)(_p(w), G, N, K, _p(q), _p(s), _stream(stream, dev)), _entry)
     return q, s
 
 
@@ -171,19 +205,21 @@ def fp8_quant_w_128x128_ue8m0(w, q=None, s=None, stream=None):
 
 def fp8_quant_act_128x1(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.Tensor | None = None, stream=None):
     """Token-axis (128x1) quantization.  Returns (q [M,K] float8_e4m3fn, s [ceil(M/128),K] f32)."""
-    _dev(x, "x", _BF16, (2,))
+    _tensor(x, "x", _BF16, (2,))
     M, K = x.shape
+    _multiple(K, "K")
     nmb = (M + TILE - 1) // TILE
+    _tensor(q, "q", _FP8)
+    _tensor(s, "s", _F32)
+    _numel(q, M * K, "q")
+    _numel(s, nmb * K, "s")
+    dev = _device_of(x=x, q=q, s=s)
     if q is None:
-        q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+        q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev)
     if s is None:
-        s = torch.empty((nmb, K), dtype=torch.float32, device=x.device)
-    _dev(q, "q", _FP8)
-    _dev(s, "s", _F32)
-    if q.numel() != M * K or s.numel() != nmb * K:
-        raise ValueError("output sizes do not match x")
-    with torch.cuda.device(x.device):
-        _check(lib().fp8_quant_act_128x1(_p(x), M, K, _p(q), _p(s), _stream(stream, x.device)), "fp8_quant_act_128x1")
+        s = torch.empty((nmb, K), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().fp8_quant_act_128x1(_p(x), M, K, _p(q), _p(s), _stream(stream, dev)), "fp8_quant_act_128x1")
     return q, s
 
 
@@ -191,97 +227,127 @@ def fp8_transpose_w_128x128(q: torch.Tensor, s: torch.Tensor, qt: torch.Tensor |
                             st: torch.Tensor | None = None, stream=None):
     """Block-quantized W [N,K] or [G,N,K] (codes + [..,N/128,K/128] scales) -> W^T codes [..,K,N] and
     scales [..,K/128,N/128].  With them, fp8_gemm_blockscaled(q_dy, s_dy, qt, st) is dX = dY W."""
-    _dev(q, "q", _FP8, (2, 3))
-    _dev(s, "s", _F32)
+    _tensor(q, "q", _FP8, (2, 3))
+    _tensor(s, "s", _F32)
     G, N, K = (1,) + tuple(q.shape) if q.dim() == 2 else tuple(q.shape)
+    _multiple(N, "N")
+    _multiple(K, "K")
     lead = tuple(q.shape[:-2])
-    if s.numel() != G * (N // TILE) * (K // TILE):
-        raise ValueError("scale size does not match q")
+    _numel(s, G * (N // TILE) * (K // TILE), "s")
+    _tensor(qt, "qt", _FP8)
+    _tensor(st, "st", _F32)
+    _numel(qt, G * N * K, "qt")
+    _numel(st, G * (N // TILE) * (K // TILE), "st")
+    dev = _device_of(q=q, s=s, qt=qt, st=st)
     if qt is None:
-        qt = torch.empty(lead + (K, N), dtype=torch.float8_e4m3fn, device=q.device)
+        qt = torch.empty(lead + (K, N), dtype=torch.float8_e4m3fn, device=dev)
     if st is None:
-        st = torch.empty(lead + (K // TILE, N // TILE), dtype=torch.float32, device=q.device)
-    _dev(qt, "qt", _FP8)
-    _dev(st, "st", _F32)
-    if qt.numel() != G * N * K or st.numel() != G * (N // TILE) * (K // TILE):
-        raise ValueError("output sizes do not match q")
-    with torch.cuda.device(q.device):
-        _check(lib().fp8_transpose_w_128x128(_p(q), _p(s), G, N, K, _p(qt), _p(st), _stream(stream, q.device)),
+        st = torch.empty(lead + (K // TILE, N // TILE), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().fp8_transpose_w_128x128(_p(q), _p(s), G, N, K, _p(qt), _p(st), _stream(stream, dev)),
                "fp8_transpose_w_128x128")
     return qt, st
 
 
-def _gemm_operands(qa, sa, qb, sb):
-    _dev(qa, "qa", _FP8)
-    _dev(sa, "sa", _F32)
-    _dev(qb, "qb", _FP8)
-    _dev(sb, "sb", _F32)
+def _dense_operands(qa, sa, qb, sb, out):
+    """Shapes of C = A * B^T: qa [M,K], sa [M,K/128], qb [N,K], sb [N/128,K/128], out [M,N]."""
+    _tensor(qa, "qa", _FP8, (2,))
+    _tensor(sa, "sa", _F32)
+    _tensor(qb, "qb", _FP8, (2,))
+    _tensor(sb, "sb", _F32)
+    _tensor(out, "out", _BF16)
+    M, K = qa.shape
+    N = qb.shape[0]
+    if qb.shape[1] != K:
+        raise ValueError("qa and qb differ in K (%d, %d)" % (K, qb.shape[1]))
+    _multiple(N, "N")
+    _multiple(K, "K")
+    _numel(sa, M * (K // TILE), "sa")
+    _numel(sb, (N // TILE) * (K // TILE), "sb")
+    _numel(out, M * N, "out")
+    return M, N, K, _device_of(qa=qa, sa=sa, qb=qb, sb=sb, out=out)
 
 
 def fp8_gemm_blockscaled(qa, sa, qb, sb, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """C[M,N] (bf16) = A * B^T from 1x128-quantized A and 128x128-quantized B."""
-    _gemm_operands(qa, sa, qb, sb)
-    M, K = qa.shape
-    N = qb.shape[0]
-    if tuple(qb.shape) != (N, K) or sa.numel() != M * (K // TILE) or sb.numel() != (N // TILE) * (K // TILE):
-        raise ValueError("operand shapes do not agree")
+    M, N, K, dev = _dense_operands(qa, sa, qb, sb, out)
     if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=qa.device)
-    _dev(out, "out", _BF16)
-    if out.numel() != M * N:
-        raise ValueError("out must hold M*N elements")
-    with torch.cuda.device(qa.device):
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
         _check(lib().fp8_gemm_blockscaled(_p(qa), _p(sa), _p(qb), _p(sb), _p(out), M, N, K,
-                                          _stream(stream, qa.device)), "fp8_gemm_blockscaled")
+                                          _stream(stream, dev)), "fp8_gemm_blockscaled")
     return out
 
 
 def fp8_gemm_unpromoted_diag(qa, sa, qb, sb, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Diagnostic: all of K accumulated in the tensor cores, scaled once (per-tensor scales only)."""
-    _gemm_operands(qa, sa, qb, sb)
-    M, K = qa.shape
-    N = qb.shape[0]
+    M, N, K, dev = _dense_operands(qa, sa, qb, sb, out)
     if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=qa.device)
-    _dev(out, "out", _BF16)
-    with torch.cuda.device(qa.device):
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
         _check(lib().fp8_gemm_unpromoted_diag(_p(qa), _p(sa), _p(qb), _p(sb), _p(out), M, N, K,
-                                              _stream(stream, qa.device)), "fp8_gemm_unpromoted_diag")
+                                              _stream(stream, dev)), "fp8_gemm_unpromoted_diag")
     return out
 
 
 def fp8_grouped_gemm_contiguous(qa, sa, qb, sb, m_indices, out: torch.Tensor | None = None, stream=None):
-    """Contiguous-layout grouped GEMM: C[M_tot,N]; block b uses expert m_indices[b]."""
-    _gemm_operands(qa, sa, qb, sb)
-    _dev(m_indices, "m_indices", _I32)
+    """Contiguous-layout grouped GEMM: C[M_tot,N]; block b uses expert m_indices[b].
+
+    qa [M_tot,K], sa [M_tot,K/128], qb [E,N,K], sb [E,N/128,K/128], m_indices int32 [M_tot/128]."""
+    _tensor(qa, "qa", _FP8, (2,))
+    _tensor(sa, "sa", _F32)
+    _tensor(qb, "qb", _FP8, (3,))
+    _tensor(sb, "sb", _F32)
+    _tensor(m_indices, "m_indices", _I32)
+    _tensor(out, "out", _BF16)
     M_tot, K = qa.shape
     E, N, K2 = qb.shape
-    if K2 != K or m_indices.numel() != M_tot // TILE:
-        raise ValueError("operand shapes do not agree")
+    if K2 != K:
+        raise ValueError("qa and qb differ in K (%d, %d)" % (K, K2))
+    _multiple(M_tot, "M_tot")
+    _multiple(N, "N")
+    _multiple(K, "K")
+    _numel(sa, M_tot * (K // TILE), "sa")
+    _numel(sb, E * (N // TILE) * (K // TILE), "sb")
+    _numel(m_indices, M_tot // TILE, "m_indices")
+    _numel(out, M_tot * N, "out")
+    dev = _device_of(qa=qa, sa=sa, qb=qb, sb=sb, m_indices=m_indices, out=out)
     if out is None:
-        out = torch.empty((M_tot, N), dtype=torch.bfloat16, device=qa.device)
-    _dev(out, "out", _BF16)
-    with torch.cuda.device(qa.device):
+        out = torch.empty((M_tot, N), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
         _check(lib().fp8_grouped_gemm_contiguous(_p(qa), _p(sa), _p(qb), _p(sb), _p(m_indices), _p(out), M_tot, N, K,
-                                                 E, _stream(stream, qa.device)), "fp8_grouped_gemm_contiguous")
+                                                 E, _stream(stream, dev)), "fp8_grouped_gemm_contiguous")
     return out
 
 
 def fp8_grouped_gemm_masked(qa, sa, qb, sb, masked_m, expected_m: int = 0, out: torch.Tensor | None = None,
                             stream=None):
-    """Masked-layout grouped GEMM: C[E,cap,N]; rows >= masked_m[e] are left unwritten."""
-    _gemm_operands(qa, sa, qb, sb)
-    _dev(masked_m, "masked_m", _I32)
+    """Masked-layout grouped GEMM: C[E,cap,N]; rows >= masked_m[e] are left unwritten.
+
+    qa [E,cap,K], sa [E,cap,K/128], qb [E,N,K], sb [E,N/128,K/128], masked_m int32 [E]."""
+    _tensor(qa, "qa", _FP8, (3,))
+    _tensor(sa, "sa", _F32)
+    _tensor(qb, "qb", _FP8, (3,))
+    _tensor(sb, "sb", _F32)
+    _tensor(masked_m, "masked_m", _I32)
+    _tensor(out, "out", _BF16)
     E, cap, K = qa.shape
     E2, N, K2 = qb.shape
-    if E2 != E or K2 != K or masked_m.numel() != E:
-        raise ValueError("operand shapes do not agree")
+    if E2 != E or K2 != K:
+        raise ValueError("qa [E=%d, K=%d] and qb [E=%d, K=%d] do not agree" % (E, K, E2, K2))
+    _multiple(cap, "cap")
+    _multiple(N, "N")
+    _multiple(K, "K")
+    _numel(sa, E * cap * (K // TILE), "sa")
+    _numel(sb, E * (N // TILE) * (K // TILE), "sb")
+    _numel(masked_m, E, "masked_m")
+    _numel(out, E * cap * N, "out")
+    dev = _device_of(qa=qa, sa=sa, qb=qb, sb=sb, masked_m=masked_m, out=out)
     if out is None:
-        out = torch.empty((E, cap, N), dtype=torch.bfloat16, device=qa.device)
-    _dev(out, "out", _BF16)
-    with torch.cuda.device(qa.device):
+        out = torch.empty((E, cap, N), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
         _check(lib().fp8_grouped_gemm_masked(_p(qa), _p(sa), _p(qb), _p(sb), _p(masked_m), _p(out), E, cap, N, K,
-                                             int(expected_m), _stream(stream, qa.device)), "fp8_grouped_gemm_masked")
+                                             int(expected_m), _stream(stream, dev)), "fp8_grouped_gemm_masked")
     return out
 
 
