@@ -31,7 +31,8 @@ std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<uint64_t> g_launches{0};
 
 struct DeviceInfo {
-  bool ready = false;
+  // set (release) once every other field is final; read (acquire) without the lock
+  std::atomic<bool> ready{false};
   bool supported = false;
   int num_sms = 0;
   uint32_t* status = nullptr;  // device address of g_device_status
@@ -56,9 +57,9 @@ int device_info(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8Q_ERR_CUDA;
   DeviceInfo& d = g_dev[dev];
-  if (!d.ready) {
+  if (!d.ready.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lock(g_dev_mu);
-    if (!d.ready) {
+    if (!d.ready.load(std::memory_order_relaxed)) {
       int major = 0, minor = 0, sms = 0;
       if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
           cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
@@ -79,7 +80,7 @@ int device_info(DeviceInfo** out) {
         if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kMasked, true, false>();
         if (e != cudaSuccess) return FP8Q_ERR_CUDA;
       }
-      d.ready = true;
+      d.ready.store(true, std::memory_order_release);
     }
   }
   if (!d.supported) return FP8Q_ERR_UNSUPPORTED;
@@ -263,7 +264,7 @@ struct ApiRange {
 
 template <bool kPow2>
 static int quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
-  if (M < 0 || K < 0 || K % 128) return FP8Q_ERR_SHAPE;
+  if (M < 0 || K < 0 || K % 128 || M >= kMaxRows || K >= kMaxRows) return FP8Q_ERR_SHAPE;
   if (M == 0 || K == 0) return FP8Q_OK;
   if (!x_bf16 || !q || !s) return FP8Q_ERR_NULL;
   if (!aligned(x_bf16, 32) || !aligned(q, 16) || !aligned(s, 4)) return FP8Q_ERR_ALIGN;
@@ -286,7 +287,9 @@ static int quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q,
 template <bool kPow2>
 static int quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, uint8_t* q, float* s,
                            cudaStream_t stream) {
-  if (G < 0 || N < 0 || K < 0 || N % 128 || K % 128) return FP8Q_ERR_SHAPE;
+  if (G < 0 || N < 0 || K < 0 || N % 128 || K % 128 || G >= kMaxRows || N >= kMaxRows || G * N >= kMaxRows ||
+      K >= kMaxRows)
+    return FP8Q_ERR_SHAPE;
   if (G == 0 || N == 0 || K == 0) return FP8Q_OK;
   if (!w_bf16 || !q || !s) return FP8Q_ERR_NULL;
   if (!aligned(w_bf16, 32) || !aligned(q, 16) || !aligned(s, 4)) return FP8Q_ERR_ALIGN;
@@ -329,7 +332,7 @@ int fp8_quant_w_128x128_ue8m0(const void* w_bf16, int64_t G, int64_t N, int64_t 
 
 int fp8_quant_act_128x1(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
   FP8Q_API_RANGE();
-  if (M < 0 || K < 0 || K % 128) return FP8Q_ERR_SHAPE;
+  if (M < 0 || K < 0 || K % 128 || M >= kMaxRows || K >= kMaxRows) return FP8Q_ERR_SHAPE;
   if (M == 0 || K == 0) return FP8Q_OK;
   if (!x_bf16 || !q || !s) return FP8Q_ERR_NULL;
   if (!aligned(x_bf16, 16) || !aligned(q, 16) || !aligned(s, 16)) return FP8Q_ERR_ALIGN;
@@ -349,7 +352,9 @@ int fp8_quant_act_128x1(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, fl
 int fp8_transpose_w_128x128(const uint8_t* q, const float* s, int64_t G, int64_t N, int64_t K, uint8_t* qt,
                             float* st, cudaStream_t stream) {
   FP8Q_API_RANGE();
-  if (G < 0 || N < 0 || K < 0 || N % 128 || K % 128) return FP8Q_ERR_SHAPE;
+  if (G < 0 || N < 0 || K < 0 || N % 128 || K % 128 || G >= kMaxRows || N >= kMaxRows || G * N >= kMaxRows ||
+      K >= kMaxRows)
+    return FP8Q_ERR_SHAPE;
   if (G == 0 || N == 0 || K == 0) return FP8Q_OK;
   if (!q || !s || !qt || !st) return FP8Q_ERR_NULL;
   if (!aligned(q, 16) || !aligned(qt, 16) || !aligned(s, 4) || !aligned(st, 4)) return FP8Q_ERR_ALIGN;

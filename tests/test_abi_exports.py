@@ -184,3 +184,22 @@ def test_no_cpu_fallback(call):
     """Host tensors are refused before anything runs: there is no CPU path."""
     with pytest.raises(ValueError, match="CUDA tensor"):
         call()
+
+
+BIG = 1 << 31
+
+
+@pytest.mark.parametrize("name,args", [
+    ("fp8_quant_act_1x128", (A16, BIG, 128, A16, A16, None)),
+    ("fp8_quant_act_1x128", (A16, 4, BIG, A16, A16, None)),
+    ("fp8_quant_act_1x128_ue8m0", (A16, BIG, 128, A16, A16, None)),
+    ("fp8_quant_w_128x128", (A16, 1 << 24, 1 << 8, 128, A16, A16, None)),   # G*N = 2^32 stacked rows
+    ("fp8_quant_w_128x128", (A16, 1, 128, BIG, A16, A16, None)),
+    ("fp8_quant_w_128x128_ue8m0", (A16, BIG, 128, 128, A16, A16, None)),
+    ("fp8_quant_act_128x1", (A16, BIG, 128, A16, A16, None)),
+    ("fp8_transpose_w_128x128", (A16, A16, 1 << 24, 1 << 8, 128, A16, A16, None)),
+])
+def test_sizes_beyond_the_limits_are_refused(name, args):
+    """Row and column counts of 2^31 or more (and stacked counts that reach
+    it) are refused before any index arithmetic could overflow."""
+    assert _call(name, *args) == fq.ERR_SHAPE
