@@ -4,9 +4,12 @@ Tolerance (written here, from the target): max |C - C_ref| <= 1e-2 * rms(C_ref)
 and max relative error <= 2e-3 over elements with |C_ref| >= 0.1 * rms(C_ref)
 (see parity.py).  The oracle quantizes the same bf16 inputs itself; nothing it
 compares against comes from the GPU.  Small shapes are compared in full
-(several tiles, ragged tails); full-size workloads on a seeded row sample that
-covers every 128-row tile (first and last row of each), every expert and all
-N columns.
+(several tiles, ragged tails), among them shapes with more than twice as many
+output tiles as the B200 has SMs, so every persistent CTA carries its state
+(accumulator reset, scale-ring slot, barrier phases) over several tiles.
+Full-size workloads are compared on a seeded row sample that reaches every
+32-row quad of every 128-row tile (the rows of each epilogue warp), every
+expert and all N columns.
 """
 import numpy as np
 import pytest
@@ -104,9 +107,27 @@ def test_dense_workloads_sampled(dev, name):
     (qa, sa, qb, sb), (oqa, osa, oqb, osb) = _quantize_both(d.a, d.b, dev)
     c = fq.fp8_gemm_blockscaled(qa, sa, qb, sb)
     _finish(dev)
-    rows = wl.parity_rows(np.random.default_rng(77), d.M, per_tile=2)
+    rows = wl.quad_rows(np.random.default_rng(77), d.M)
     ref = oracle.gemm_blockscaled(oqa, osa, oqb, osb, rows=rows)
     assert_gemm_close(bf16_bits_of(c)[rows], ref, name)
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (1024, 5120, 512),   # 320 tiles: one scale group per tile, the scale ring's slot moves on every tile
+    (2048, 2560, 2048),  # 320 tiles, four scale groups per tile
+    (1000, 4864, 1664),  # 304 tiles, ragged M; K % 512 != 0: scales loaded from global memory
+])
+def test_dense_many_tiles_full(dev, M, N, K):
+    """More than two tiles per SM, every element compared: each CTA's second
+    and later tiles, in every epilogue warp."""
+    rng = np.random.default_rng(M + 5 * N + 11 * K)
+    a = rng.standard_normal((M, K)).astype(np.float32) * np.exp(rng.standard_normal(K)).astype(np.float32)
+    b = (0.02 * rng.standard_normal((N, K))).astype(np.float32)
+    (qa, sa, qb, sb), (oqa, osa, oqb, osb) = _quantize_both(wl.bf16_bits(a), wl.bf16_bits(b), dev)
+    c = fq.fp8_gemm_blockscaled(qa, sa, qb, sb)
+    _finish(dev)
+    ref = oracle.gemm_blockscaled(oqa, osa, oqb, osb)
+    assert_gemm_close(bf16_bits_of(c), ref, "dense %dx%dx%d" % (M, N, K))
 
 
 def test_all_ones_closed_form(dev):
@@ -136,18 +157,26 @@ def test_output_rows_beyond_m_untouched(dev):
 
 
 # ------------------------------------------------------------------ contiguous
-def _contiguous_case(dev, d, rows_per_block=2):
+def _contiguous_case(dev, d, all_rows=False):
     (qa, sa, qb, sb), (oqa, osa, oqb, osb) = _quantize_both(d.a, d.b, dev)
     mi = torch.from_numpy(d.m_indices).to(dev)
     c = fq.fp8_grouped_gemm_contiguous(qa, sa, qb.view(d.b.shape), sb, mi)
     _finish(dev)
-    rows = wl.parity_rows(np.random.default_rng(3), d.M_tot, per_tile=rows_per_block)
+    rows = np.arange(d.M_tot) if all_rows else wl.quad_rows(np.random.default_rng(3), d.M_tot)
     ref = oracle.grouped_contiguous(oqa, osa, oqb, osb, d.m_indices, rows=rows)
     assert_gemm_close(bf16_bits_of(c)[rows], ref, d.name)
 
 
 def test_contiguous_small(dev):
-    _contiguous_case(dev, wl.moe_contiguous(tokens=96, topk=4, E=6, N=384, K=512, seed=21), rows_per_block=128)
+    _contiguous_case(dev, wl.moe_contiguous(tokens=96, topk=4, E=6, N=384, K=512, seed=21), all_rows=True)
+
+
+@pytest.mark.parametrize("K", [512, 2048])
+def test_contiguous_many_tiles_full(dev, K):
+    """Over 300 tiles of mixed experts, every element compared."""
+    d = wl.moe_contiguous(tokens=512, topk=6, E=8, N=2560, K=K, seed=40 + K)
+    assert (d.M_tot // TILE) * (d.N // TILE) > 2 * 148
+    _contiguous_case(dev, d, all_rows=True)
 
 
 def test_contiguous_full(dev):
@@ -170,7 +199,7 @@ def test_contiguous_skips_out_of_range_blocks(dev):
 
 
 # ------------------------------------------------------------------ masked
-def _masked_case(dev, a, b, masked_m, rows_per_expert=None):
+def _masked_case(dev, a, b, masked_m, sampled=False):
     E, cap, K = a.shape
     N = b.shape[1]
     (qa, sa, qb, sb), (oqa, osa, oqb, osb) = _quantize_both(a, b, dev)
@@ -187,16 +216,16 @@ def _masked_case(dev, a, b, masked_m, rows_per_expert=None):
                            + [np.zeros(0, np.int64)])
     invalid = np.setdiff1d(np.arange(E * cap), valid)
     assert np.all(got[invalid] == 0xC0A0), "rows at or past masked_m must stay untouched"  # bf16 -5.0
-    if rows_per_expert is None:
+    if not sampled:
         rows = valid
     else:
+        # every 32-row quad of every valid tile of every expert
         rng = np.random.default_rng(11)
         rows = []
         for e in range(E):
             m = min(cap, max(0, int(masked_m[e])))
             if m:
-                pick = {0, m - 1} | set(rng.choice(m, size=min(m, rows_per_expert), replace=False).tolist())
-                rows.extend(e * cap + r for r in sorted(pick))
+                rows.extend(e * cap + wl.quad_rows(rng, m))
         rows = np.asarray(rows, dtype=np.int64)
     if rows.size:
         ref = oracle.grouped_masked(oqa3, osa3, oqb, osb, np.asarray(masked_m, np.int32), rows=rows)
@@ -225,7 +254,21 @@ def test_masked_out_of_range_counts_clamped(dev):
     _masked_case(dev, a, b, [-4, 500, 77])
 
 
+def test_masked_many_tiles_full(dev):
+    """Over 300 tiles (counts spanning 0..cap), every valid element compared
+    and every other row checked untouched."""
+    rng = np.random.default_rng(34)
+    E, cap, N, K = 12, 256, 2560, 1024
+    masked_m = rng.integers(0, cap, size=E, endpoint=True)
+    masked_m[:3] = [cap, 129, 0]
+    tiles = sum((int(m) + TILE - 1) // TILE for m in masked_m) * (N // TILE)
+    assert tiles > 2 * 148
+    a = wl.bf16_bits(rng.standard_normal((E, cap, K)).astype(np.float32))
+    b = wl.bf16_bits((0.02 * rng.standard_normal((E, N, K))).astype(np.float32))
+    _masked_case(dev, a, b, masked_m)
+
+
 def test_masked_full_both_gemms(dev):
     d = wl.moe_masked()
-    _masked_case(dev, d.a, d.b, d.masked_m, rows_per_expert=4)
-    _masked_case(dev, d.a2, d.b2, d.masked_m, rows_per_expert=4)
+    _masked_case(dev, d.a, d.b, d.masked_m, sampled=True)
+    _masked_case(dev, d.a2, d.b2, d.masked_m, sampled=True)

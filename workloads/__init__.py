@@ -238,6 +238,23 @@ def parity_rows(rng: np.random.Generator, M: int, per_tile: int = 2, tile: int =
     return np.asarray(rows, dtype=np.int64)
 
 
+def quad_rows(rng: np.random.Generator, M: int, tile: int = TILE, quad: int = 32) -> np.ndarray:
+    """Seeded sample of row indices that reaches every 32-row quad of every
+    128-row tile: the tile's first and last row, plus one seeded row inside
+    each quad that holds valid rows (a ragged last tile only has the quads
+    below M).  The GEMM's epilogue assigns each quad of a tile to its own
+    warps, so every warp's rows are compared on every tile."""
+    rows = []
+    for t0 in range(0, M, tile):
+        t1 = min(M, t0 + tile)
+        pick = {t0, t1 - 1}
+        for q0 in range(t0, t1, quad):
+            q1 = min(t1, q0 + quad)
+            pick.add(int(rng.integers(q0, q1)))
+        rows.extend(sorted(pick))
+    return np.asarray(rows, dtype=np.int64)
+
+
 CONFIGS = {
     "tiny_dense": tiny_dense,
     "dense_fprop": dense_fprop,
