@@ -155,6 +155,10 @@ def make_workload(name: str):
         # the activation-gradient GEMM of the dense_fprop layer: dY takes the
         # shape and distribution of the forward activations, W is the weight
         return wl.dense_fprop()
+    if name == "moe_masked_chain":
+        # the masked decode as one chain: GEMM2's activation is the SwiGLU of
+        # GEMM1's output, requantized (its own A2 draw is not used)
+        return wl.moe_masked()
     return wl.CONFIGS[name]()
 
 
@@ -170,8 +174,8 @@ def describe(name: str, d) -> dict:
                                                                                  d.N, d.K),
                 "E": d.E, "M_tot": d.M_tot, "valid_rows": int(d.counts.sum()), "N": d.N, "K": d.K,
                 "seed": d.meta["seed"]}
-    return {"workload": "moe_masked E=%d cap=%d valid=%d (N,K)=(%d,%d)+(%d,%d)" % (
-        d.E, d.cap, int(d.masked_m.sum()), d.b.shape[1], d.b.shape[2], d.b2.shape[1], d.b2.shape[2]),
+    return {"workload": "%s E=%d cap=%d valid=%d (N,K)=(%d,%d)+(%d,%d)" % (
+        name, d.E, d.cap, int(d.masked_m.sum()), d.b.shape[1], d.b.shape[2], d.b2.shape[1], d.b2.shape[2]),
         "E": d.E, "cap": d.cap, "valid_rows": int(d.masked_m.sum()), "seed": d.meta["seed"]}
 
 
@@ -184,11 +188,12 @@ def build_sets(name, d, dev, nsets, torch, fq):
     sets = []
     for _ in range(nsets):
         s = {}
-        if name == "moe_masked":
+        if name in ("moe_masked", "moe_masked_chain"):
             E, cap, K = d.a.shape
             s["a"] = _to_dev_bf16(torch, d.a.reshape(E * cap, K), dev)
             s["b"] = _to_dev_bf16(torch, d.b, dev)
-            s["a2"] = _to_dev_bf16(torch, d.a2.reshape(E * cap, -1), dev)
+            if name == "moe_masked":
+                s["a2"] = _to_dev_bf16(torch, d.a2.reshape(E * cap, -1), dev)
             s["b2"] = _to_dev_bf16(torch, d.b2, dev)
             s["mm"] = torch.from_numpy(d.masked_m).to(dev)
         else:
@@ -228,6 +233,13 @@ def kernel_plan(name, d):
     N, K2, N2 = d.b.shape[1], d.a2.shape[2], d.b2.shape[1]
     active = int((d.masked_m > 0).sum())
     valid = int(d.masked_m.sum())
+    if name == "moe_masked_chain":
+        # GEMM1's valid rows in (gate | up, bf16), h's codes and scales out
+        swiglu = valid * N * 2 + valid * K2 + valid * (K2 // TILE) * 4
+        return [("quant_act_1x128", qa_bytes(E * cap, K), 0.0), ("quant_w_128x128", qw_bytes(E, N, K), 0.0),
+                ("grouped_gemm_masked", gemm_bytes(valid, N, K, active), d.flops(False)),
+                ("swiglu_quant_1x128", swiglu, 0.0), ("quant_w_128x128#2", qw_bytes(E, N2, K2), 0.0),
+                ("grouped_gemm_masked#2", gemm_bytes(valid, N2, K2, active), d.flops(True))]
     return [("quant_act_1x128", qa_bytes(E * cap, K), 0.0), ("quant_w_128x128", qw_bytes(E, N, K), 0.0),
             ("grouped_gemm_masked", gemm_bytes(valid, N, K, active), d.flops(False)),
             ("quant_act_1x128#2", qa_bytes(E * cap, K2), 0.0), ("quant_w_128x128#2", qw_bytes(E, N2, K2), 0.0),
@@ -241,6 +253,22 @@ def launch_step(name, d, s, fq, events=None):
         if events is not None:
             events[i][which].record()
 
+    if name == "moe_masked_chain":
+        E, cap, K = d.a.shape
+        rec(0, 0); qa, sa = fq.fp8_quant_act_1x128(s["a"], s.get("qa"), s.get("sa")); rec(0, 1)
+        rec(1, 0); qb, sb = fq.fp8_quant_w_128x128(s["b"], s.get("qb"), s.get("sb")); rec(1, 1)
+        rec(2, 0)
+        c = fq.fp8_grouped_gemm_masked(qa.view(E, cap, K), sa.view(E, cap, K // TILE), qb, sb, s["mm"],
+                                       expected_m=int(d.masked_m.mean()), out=s.get("c"))
+        rec(2, 1)
+        rec(3, 0); qh, sh = fq.fp8_swiglu_quant_1x128(c, s["mm"], s.get("qh"), s.get("sh")); rec(3, 1)
+        rec(4, 0); qb2, sb2 = fq.fp8_quant_w_128x128(s["b2"], s.get("qb2"), s.get("sb2")); rec(4, 1)
+        rec(5, 0)
+        c2 = fq.fp8_grouped_gemm_masked(qh, sh, qb2, sb2, s["mm"], expected_m=int(d.masked_m.mean()),
+                                        out=s.get("c2"))
+        rec(5, 1)
+        s.update(qa=qa, sa=sa, qb=qb, sb=sb, c=c, qh=qh, sh=sh, qb2=qb2, sb2=sb2, c2=c2)
+        return c2
     if name == "moe_masked":
         E, cap, K = d.a.shape
         rec(0, 0); qa, sa = fq.fp8_quant_act_1x128(s["a"], s.get("qa"), s.get("sa")); rec(0, 1)
@@ -276,7 +304,7 @@ def launch_step(name, d, s, fq, events=None):
 
 
 def step_flops(name, d):
-    if name == "moe_masked":
+    if name in ("moe_masked", "moe_masked_chain"):
         return d.flops(False) + d.flops(True)
     return d.flops
 
@@ -288,7 +316,7 @@ def oracle_sample_step(name, d, rows: int, nblocks: int):
     weight blocks, and the GEMM outputs rows x (128 * nblocks).  Returns
     (seconds, flops of the sample)."""
     import oracle
-    if name == "moe_masked":
+    if name in ("moe_masked", "moe_masked_chain"):
         a, b = d.a[0], d.b[0]
     elif name == "moe_contiguous":
         a, b = d.a, d.b[int(d.m_indices[0])]
@@ -498,9 +526,9 @@ def run_e2e(args, name, d, dev, torch, fq, world):
     """Same step through the public API from pinned host buffers: H2D copy of
     the bf16 inputs, the three kernels, D2H copy of the bf16 result."""
     host = {}
-    keys = ["a", "b"] + (["a2", "b2"] if name == "moe_masked" else [])
+    keys = ["a", "b"] + (["a2", "b2"] if name == "moe_masked" else ["b2"] if name == "moe_masked_chain" else [])
     src = {"a": d.a, "b": d.b}
-    if name == "moe_masked":
+    if name in ("moe_masked", "moe_masked_chain"):
         src.update(a2=d.a2, b2=d.b2)
     for k in keys:
         arr = np.ascontiguousarray(src[k]).view(np.int16)
@@ -559,7 +587,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dense_fprop",
-                    choices=["tiny_dense", "dense_fprop", "long_k", "moe_contiguous", "moe_masked", "dense_dgrad"])
+                    choices=["tiny_dense", "dense_fprop", "long_k", "moe_contiguous", "moe_masked", "dense_dgrad",
+                             "moe_masked_chain"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

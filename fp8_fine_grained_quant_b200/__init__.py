@@ -13,6 +13,7 @@ Names and semantics match the C entry points:
 * :func:`fp8_quant_act_128x1`  -- bf16 [M,K] -> E4M3 [M,K] + f32 scales [ceil(M/128),K] (token-axis tiles)
 * :func:`fp8_quant_act_1x128_ue8m0`, :func:`fp8_quant_w_128x128_ue8m0` -- the same groups, power-of-two scales
 * :func:`fp8_transpose_w_128x128` -- block-quantized W [..,N,K] -> W^T [..,K,N] (codes and block scales)
+* :func:`fp8_swiglu_quant_1x128` -- GEMM1 output [.., 2I] bf16 -> SwiGLU -> 1x128 E4M3 [.., I] + scales
 * :func:`fp8_gemm_blockscaled` -- C = A * B^T (bf16) with per-128-slab promotion
 * :func:`fp8_grouped_gemm_contiguous` -- MoE grouped GEMM, contiguous layout
 * :func:`fp8_grouped_gemm_masked`     -- MoE grouped GEMM, masked layout
@@ -26,6 +27,7 @@ import torch
 
 __all__ = [
     "fp8_quant_act_1x128", "fp8_quant_w_128x128", "fp8_quant_act_128x1", "fp8_transpose_w_128x128",
+    "fp8_swiglu_quant_1x128",
     "fp8_quant_act_1x128_ue8m0", "fp8_quant_w_128x128_ue8m0",
     "fp8_gemm_blockscaled", "fp8_grouped_gemm_contiguous",
     "fp8_grouped_gemm_masked", "fp8_gemm_unpromoted_diag", "get_device_error", "set_wait_timeout_ns",
@@ -47,6 +49,7 @@ EXPORTS = {
     "fp8_quant_act_1x128_ue8m0": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
     "fp8_quant_w_128x128_ue8m0": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "fp8_transpose_w_128x128": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P]),
+    "fp8_swiglu_quant_1x128": (ctypes.c_int, [_P, _I64, _I64, _P, _I64, _P, _P, _P]),
     "fp8_gemm_blockscaled": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "fp8_grouped_gemm_contiguous": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "fp8_grouped_gemm_masked": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P]),
@@ -247,6 +250,41 @@ def fp8_transpose_w_128x128(q: torch.Tensor, s: torch.Tensor, qt: torch.Tensor |
         _check(lib().fp8_transpose_w_128x128(_p(q), _p(s), G, N, K, _p(qt), _p(st), _stream(stream, dev)),
                "fp8_transpose_w_128x128")
     return qt, st
+
+
+def fp8_swiglu_quant_1x128(c1: torch.Tensor, masked_m: torch.Tensor | None = None, qh: torch.Tensor | None = None,
+                           sh: torch.Tensor | None = None, stream=None):
+    """SwiGLU of GEMM1's [gate | up] output fused with its 1x128 requantization.
+    c1 [rows, 2I] or [E, cap, 2I] bf16 -> (qh [.., I] float8_e4m3fn, sh [.., I/128] f32).  With
+    masked_m (int32 [E], c1 3-D), rows at or past masked_m[e] are left unwritten."""
+    _tensor(c1, "c1", _BF16, (2, 3))
+    _tensor(masked_m, "masked_m", _I32)
+    if c1.shape[-1] % (2 * TILE):
+        raise ValueError("c1's last dim %d is not 2 x a multiple of %d" % (c1.shape[-1], TILE))
+    inter = c1.shape[-1] // 2
+    lead = tuple(c1.shape[:-1])
+    rows = 1
+    for d in lead:
+        rows *= d
+    cap = 0
+    if masked_m is not None:
+        if c1.dim() != 3:
+            raise ValueError("masked_m needs c1 as [E, cap, 2I]")
+        cap = c1.shape[1]
+        _numel(masked_m, c1.shape[0], "masked_m")
+    _tensor(qh, "qh", _FP8)
+    _tensor(sh, "sh", _F32)
+    _numel(qh, rows * inter, "qh")
+    _numel(sh, rows * (inter // TILE), "sh")
+    dev = _device_of(c1=c1, masked_m=masked_m, qh=qh, sh=sh)
+    if qh is None:
+        qh = torch.empty(lead + (inter,), dtype=torch.float8_e4m3fn, device=dev)
+    if sh is None:
+        sh = torch.empty(lead + (inter // TILE,), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().fp8_swiglu_quant_1x128(_p(c1), rows, inter, _p(masked_m), cap, _p(qh), _p(sh),
+                                            _stream(stream, dev)), "fp8_swiglu_quant_1x128")
+    return qh, sh
 
 
 def _dense_operands(qa, sa, qb, sb, out):

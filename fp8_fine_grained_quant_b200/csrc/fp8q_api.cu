@@ -349,6 +349,29 @@ int fp8_quant_act_128x1(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, fl
   return FP8Q_OK;
 }
 
+int fp8_swiglu_quant_1x128(const void* c1_bf16, int64_t rows, int64_t inter, const int32_t* masked_m, int64_t cap,
+                           uint8_t* qh, float* sh, cudaStream_t stream) {
+  FP8Q_API_RANGE();
+  if (rows < 0 || inter < 0 || inter % 128 || rows >= kMaxRows || inter >= kMaxRows / 2) return FP8Q_ERR_SHAPE;
+  if (masked_m && (cap <= 0 || rows % cap)) return FP8Q_ERR_SHAPE;
+  if (rows == 0 || inter == 0) return FP8Q_OK;
+  if (!c1_bf16 || !qh || !sh) return FP8Q_ERR_NULL;
+  if (!aligned(c1_bf16, 32) || !aligned(qh, 16) || !aligned(sh, 4) || (masked_m && !aligned(masked_m, 4)))
+    return FP8Q_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  const int64_t tiles = rows * (inter / 128);
+  int64_t grid = (tiles + 31) / 32;  // 32 tiles per CTA pass
+  const int64_t cap_grid = static_cast<int64_t>(dev->num_sms) * 8;
+  if (grid > cap_grid) grid = cap_grid;
+  swiglu_quant_1x128_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+      static_cast<const uint8_t*>(c1_bf16), qh, sh, inter, tiles, masked_m, masked_m ? cap : 1);
+  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
 int fp8_transpose_w_128x128(const uint8_t* q, const float* s, int64_t G, int64_t N, int64_t K, uint8_t* qt,
                             float* st, cudaStream_t stream) {
   FP8Q_API_RANGE();

@@ -402,4 +402,94 @@ __global__ void __launch_bounds__(256) transpose_w_128x128_kernel(const uint8_t*
   }
 }
 
+// ---------------------------------------------------------------------------
+// SwiGLU between the two MoE GEMMs, fused with the 1x128 requantization of its
+// output.  Each row of GEMM1's bf16 output is [gate | up] (inter columns each);
+// the next GEMM's activation is h = silu(gate) * up, silu(g) = g / (1 +
+// exp(-g)), rounded once to bf16, then quantized per 1x128 tile exactly as
+// quant_act_1x128_kernel does.  (The SwiGLU is not on the pages: the MoE
+// configurations' GEMM1 width, twice GEMM2's depth, implies it.)
+//
+// h is the correctly rounded bf16 of the expression.  The FP32 evaluation
+// (expf within 2 ulp, three rounded operations: relative error below 2^-21)
+// is bracketed by h (1 -+ 2^-20); when both ends round to the same bf16, that
+// is the result (rounding is monotone).  Otherwise -- a value within ~2^-20 of
+// a bf16 rounding midpoint, or outside the range where the bound holds -- the
+// expression is evaluated in double and rounded to bf16 through round-to-odd
+// FP32 (16 spare bits, so the two steps round once).
+// ---------------------------------------------------------------------------
+__device__ __noinline__ uint32_t swiglu_bf16_exact(float g, float u) {
+  const double hd = static_cast<double>(g) / (1.0 + exp(-static_cast<double>(g))) * static_cast<double>(u);
+  float f = __double2float_rz(hd);
+  if (isfinite(hd) && static_cast<double>(f) != hd) f = __uint_as_float(__float_as_uint(f) | 1u);
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ uint32_t swiglu_bf16(float g, float u) {
+  const float e = expf(-g);
+  const float h = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, e)), u);
+  const float a = fabsf(h);
+  if (isfinite(e) && a >= 0x1p-100f && a <= 0x1p+120f) {
+    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(h, 1.0f - 0x1p-20f)));
+    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(h, 1.0f + 0x1p-20f)));
+    if (lo == hi) return lo;
+  }
+  return swiglu_bf16_exact(g, u);
+}
+
+// Eight words of bf16 pairs (gate) and (up) -> eight words of bf16 pairs of h.
+__device__ __forceinline__ void swiglu16(const uint32_t (&gw)[8], const uint32_t (&uw)[8], uint32_t (&hw)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t h0 = swiglu_bf16(__uint_as_float(gw[i] << 16), __uint_as_float(uw[i] << 16));
+    const uint32_t h1 = swiglu_bf16(__uint_as_float(gw[i] & 0xFFFF0000u), __uint_as_float(uw[i] & 0xFFFF0000u));
+    hw[i] = h0 | (h1 << 16);
+  }
+}
+
+// c1 [rows, 2 * inter] bf16 -> qh [rows, inter] E4M3 codes, sh [rows, inter/128]
+// scales.  Tile t = row * (inter/128) + kb, as in quant_act_1x128_kernel.  With
+// masked_m, row = e * cap + r is valid when r < clamp(masked_m[e], 0, cap);
+// other rows are neither read nor written.
+__global__ void __launch_bounds__(256, 4) swiglu_quant_1x128_kernel(const uint8_t* __restrict__ c1,
+                                                                    uint8_t* __restrict__ qh, float* __restrict__ sh,
+                                                                    int64_t inter, int64_t num_tiles,
+                                                                    const int32_t* __restrict__ masked_m,
+                                                                    int64_t cap) {
+  const int sub = threadIdx.x & 7;
+  const int64_t grp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 3;
+  const int64_t ngrp = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 3;
+  const int64_t per_row = inter >> 7;
+  // same trip count for every lane of a warp (the shuffles need all 32)
+  for (int64_t t = grp; t - grp < num_tiles; t += ngrp) {
+    bool valid = t < num_tiles;
+    const int64_t row = valid ? t / per_row : 0, kb = valid ? t - row * per_row : 0;
+    if (valid && masked_m != nullptr) {
+      const int64_t e = row / cap;
+      int64_t m = masked_m[e];
+      m = m < 0 ? 0 : (m > cap ? cap : m);
+      valid = row - e * cap < m;
+    }
+    uint32_t hw[8];
+    if (valid) {
+      uint32_t gw[8], uw[8];
+      const uint8_t* src = c1 + ((row * 2 * inter) + kb * 128 + sub * 16) * 2;
+      ld_nc_v8(src, gw);
+      ld_nc_v8(src + inter * 2, uw);
+      swiglu16(gw, uw, hw);
+    } else {
+      zero8(hw);
+    }
+    float amax = abs_max16(hw);
+#pragma unroll
+    for (int off = 4; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+    const float sc = group_scale(amax);
+    const RecipPair rp = recip_pair(sc);
+    if (valid) {
+      *reinterpret_cast<uint4*>(qh + t * 128 + sub * 16) = quantize16(hw, sc, rp, sc < kMinFastScale);
+      if (sub == 0) sh[t] = sc;
+    }
+  }
+}
+
 }  // namespace fp8q

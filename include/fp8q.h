@@ -123,6 +123,25 @@ FP8Q_API int fp8_quant_w_128x128_ue8m0(const void* w_bf16, int64_t G, int64_t N,
 FP8Q_API int fp8_quant_act_128x1(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream);
 
 /*
+ * SwiGLU between the two MoE GEMMs fused with the 1x128 requantization of its
+ * output (the chained MoE decode; the SwiGLU is not on the pages: the MoE
+ * configurations' GEMM1 width, twice GEMM2's depth, implies it):
+ *   h[r, i] = bf16_rne( g / (1 + exp(-g)) * u ),  g = c1[r, i], u = c1[r, inter + i]
+ * (the correctly rounded bf16 of the real-valued expression), then qh, sh =
+ * the fp8_quant_act_1x128 quantization of h.
+ *   c1_bf16  : [rows, 2*inter] bf16 (GEMM1's output, [gate | up] halves), read only.
+ *   masked_m : NULL (every row valid), or the masked layout's [rows/cap] int32
+ *              counts: row e*cap + r is valid when r < clamp(masked_m[e], 0, cap);
+ *              invalid rows of qh and sh are left unwritten (their c1 rows are
+ *              not read).
+ *   qh       : [rows, inter] E4M3, sh : [rows, inter/128] f32, written.
+ * inter a multiple of 128; with masked_m, cap > 0 divides rows.  c1 32-byte,
+ * qh 16-byte, sh and masked_m 4-byte aligned.
+ */
+FP8Q_API int fp8_swiglu_quant_1x128(const void* c1_bf16, int64_t rows, int64_t inter, const int32_t* masked_m,
+                                    int64_t cap, uint8_t* qh, float* sh, cudaStream_t stream);
+
+/*
  * Transposition of 128x128-block-quantized weights (for the activation
  * gradient dX = dY W, the Dgrad GEMM of the same Figure 6): a 128x128 block
  * of W^T has the same amax, scale and codes as W's block, transposed.

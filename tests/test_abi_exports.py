@@ -203,3 +203,17 @@ def test_sizes_beyond_the_limits_are_refused(name, args):
     """Row and column counts of 2^31 or more (and stacked counts that reach
     it) are refused before any index arithmetic could overflow."""
     assert _call(name, *args) == fq.ERR_SHAPE
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((A16, 4, 100, None, 0, A16, A16, None), fq.ERR_SHAPE),      # inter not a multiple of 128
+    ((A16, -1, 128, None, 0, A16, A16, None), fq.ERR_SHAPE),
+    ((A16, 300, 128, A16, 256, A16, A16, None), fq.ERR_SHAPE),   # masked: cap does not divide rows
+    ((A16, 256, 128, A16, 0, A16, A16, None), fq.ERR_SHAPE),
+    ((A16, 0, 128, None, 0, A16, A16, None), fq.OK),
+    ((None, 4, 128, None, 0, A16, A16, None), fq.ERR_NULL),
+    ((A16_ONLY, 4, 128, None, 0, A16, A16, None), fq.ERR_ALIGN),  # bf16 input: 32 bytes
+    ((A16, 256, 128, A1, 128, A16, A16, None), fq.ERR_ALIGN),
+])
+def test_swiglu_quant_validation(args, expect):
+    assert _call("fp8_swiglu_quant_1x128", *args) == expect

@@ -174,3 +174,19 @@ def test_one_device_for_all_arguments():
     assert fq._device_of(a=d0, b=None, c=d0) == torch.device("cuda", 0)
     with pytest.raises(ValueError, match="c is on cuda:1"):
         fq._device_of(a=d0, b=d0, c=d1)
+
+
+def test_swiglu_quant_buffers():
+    c1 = z(2, 128, 512, dtype=bf16)
+    with pytest.raises(ValueError, match="not 2 x a multiple"):
+        fq.fp8_swiglu_quant_1x128(z(4, 384, dtype=bf16))
+    with pytest.raises(ValueError, match="masked_m needs c1"):
+        fq.fp8_swiglu_quant_1x128(z(256, 512, dtype=bf16), masked_m=z(2, dtype=i32))
+    with pytest.raises(ValueError, match="masked_m holds 3"):
+        fq.fp8_swiglu_quant_1x128(c1, masked_m=z(3, dtype=i32))
+    with pytest.raises(ValueError, match="qh holds 100"):
+        fq.fp8_swiglu_quant_1x128(c1, qh=z(100))
+    with pytest.raises(ValueError, match="sh holds 7"):
+        fq.fp8_swiglu_quant_1x128(c1, sh=z(7, dtype=f32))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fq.fp8_swiglu_quant_1x128(c1, masked_m=z(2, dtype=i32))
