@@ -169,6 +169,9 @@ def describe(name: str, d) -> dict:
     if name == "dense_dgrad":
         return {"workload": "dense_dgrad dX[M,K] = dY[M,N] W[N,K] M=%d N=%d K=%d" % (d.M, d.N, d.K), "M": d.M,
                 "N": d.N, "K": d.K, "seed": d.meta["seed"]}
+    if name == "dense_wgrad":
+        return {"workload": "dense_wgrad dW[N,K] = dY[M,N]^T X[M,K] M=%d N=%d K=%d" % (d.M, d.N, d.K), "M": d.M,
+                "N": d.N, "K": d.K, "seed": d.meta["seed"]}
     if name == "moe_contiguous":
         return {"workload": "moe_contiguous E=%d M_tot=%d (valid %d) N=%d K=%d" % (d.E, d.M_tot, int(d.counts.sum()),
                                                                                  d.N, d.K),
@@ -196,6 +199,9 @@ def build_sets(name, d, dev, nsets, torch, fq):
                 s["a2"] = _to_dev_bf16(torch, d.a2.reshape(E * cap, -1), dev)
             s["b2"] = _to_dev_bf16(torch, d.b2, dev)
             s["mm"] = torch.from_numpy(d.masked_m).to(dev)
+        elif name == "dense_wgrad":
+            s["dy"] = _to_dev_bf16(torch, d.dy, dev)
+            s["x"] = _to_dev_bf16(torch, d.x, dev)
         else:
             s["a"] = _to_dev_bf16(torch, d.a, dev)
             s["b"] = _to_dev_bf16(torch, d.b, dev)
@@ -226,6 +232,17 @@ def kernel_plan(name, d):
         return [("quant_act_1x128", qa_bytes(M, Nout), 0.0), ("quant_w_128x128", qw_bytes(1, Nout, K), 0.0),
                 ("transpose_w_128x128", 2 * Nout * K + 2 * 4 * (Nout // TILE) * (K // TILE), 0.0),
                 ("gemm_dgrad", gemm_bytes(M, K, Nout), 2.0 * M * Nout * K)]
+    if name == "dense_wgrad":
+        # both operands quantized along tokens, codes written token-contiguous
+        M, N, K = d.M, d.N, d.K
+        Mp = -(-M // (4 * TILE)) * (4 * TILE)  # tokens in whole groups of four slabs
+
+        def qt_bytes(C):
+            return M * C * 2 + C * Mp + (Mp // TILE) * C * 4
+
+        gemm = N * Mp + K * Mp + (Mp // TILE) * (N + K) * 4 + N * K * 2
+        return [("quant_act_128x1_t", qt_bytes(N), 0.0), ("quant_act_128x1_t#2", qt_bytes(K), 0.0),
+                ("gemm_wgrad", gemm, 2.0 * M * N * K)]
     if name == "moe_contiguous":
         return [("quant_act_1x128", qa_bytes(d.M_tot, d.K), 0.0), ("quant_w_128x128", qw_bytes(d.E, d.N, d.K), 0.0),
                 ("grouped_gemm_contiguous", gemm_bytes(d.M_tot, d.N, d.K, d.E), d.flops)]
@@ -286,6 +303,12 @@ def launch_step(name, d, s, fq, events=None):
         rec(5, 1)
         s.update(qa=qa, sa=sa, qb=qb, sb=sb, c=c, qa2=qa2, sa2=sa2, qb2=qb2, sb2=sb2, c2=c2)
         return c2
+    if name == "dense_wgrad":
+        rec(0, 0); q_dy, s_dy = fq.fp8_quant_act_128x1_t(s["dy"], s.get("q_dy"), s.get("s_dy")); rec(0, 1)
+        rec(1, 0); q_x, s_x = fq.fp8_quant_act_128x1_t(s["x"], s.get("q_x"), s.get("s_x")); rec(1, 1)
+        rec(2, 0); c = fq.fp8_gemm_wgrad(q_dy, s_dy, q_x, s_x, out=s.get("c")); rec(2, 1)
+        s.update(q_dy=q_dy, s_dy=s_dy, q_x=q_x, s_x=s_x, c=c)
+        return c
     rec(0, 0); qa, sa = fq.fp8_quant_act_1x128(s["a"], s.get("qa"), s.get("sa")); rec(0, 1)
     rec(1, 0); qb, sb = fq.fp8_quant_w_128x128(s["b"], s.get("qb"), s.get("sb")); rec(1, 1)
     if name == "dense_dgrad":
@@ -316,6 +339,16 @@ def oracle_sample_step(name, d, rows: int, nblocks: int):
     weight blocks, and the GEMM outputs rows x (128 * nblocks).  Returns
     (seconds, flops of the sample)."""
     import oracle
+    if name == "dense_wgrad":
+        # `rows` output channels of dY and `nblocks` x 128 of X, over every token
+        dy = np.ascontiguousarray(d.dy[:, :rows])
+        x = np.ascontiguousarray(d.x[:, :TILE * nblocks])
+        t0 = time.perf_counter()
+        q_dy, s_dy = oracle.quant_act_128x1(dy)
+        q_x, s_x = oracle.quant_act_128x1(x)
+        oracle.wgrad(q_dy, s_dy, q_x, s_x)
+        dt = time.perf_counter() - t0
+        return dt, 2.0 * rows * TILE * nblocks * d.M
     if name in ("moe_masked", "moe_masked_chain"):
         a, b = d.a[0], d.b[0]
     elif name == "moe_contiguous":
@@ -333,11 +366,23 @@ def oracle_sample_step(name, d, rows: int, nblocks: int):
     return dt, 2.0 * rows * TILE * nblocks * K
 
 
+def sample_description(name, d, rows: int, nb: int) -> str:
+    if name == "dense_wgrad":
+        return ("token-axis quantization of %d dY channels and %d X channels over %d tokens, float64 weight-"
+                "gradient GEMM of the %d x %d outputs they determine" % (rows, TILE * nb, d.M, rows, TILE * nb))
+    return ("1x128 quantization of %d rows of A, 128x128 quantization of %d weight block-rows (%d x %d), "
+            "float64 GEMM of the %d x %d outputs they determine (K=%d)" % (
+                rows, nb, TILE * nb, d.a.shape[-1], rows, TILE * nb, d.a.shape[-1]))
+
+
 def cpu_sample_size(name, d, budget_s: float):
     """Rows x weight blocks whose oracle step takes about budget_s."""
     rows, nb = 8, 1
-    nb_max = (d.b.shape[-2]) // TILE
-    rows_max = d.a.shape[-2]
+    if name == "dense_wgrad":
+        nb_max, rows_max = d.K // TILE, d.N
+    else:
+        nb_max = (d.b.shape[-2]) // TILE
+        rows_max = d.a.shape[-2]
     # a step's cost is not proportional to rows x blocks at small sizes
     # (fixed costs dominate), so grow the sample in a few measured rounds
     for _ in range(5):
@@ -368,9 +413,7 @@ def run_reference(args, name):
         flops += f
     total = sum(times)
     value = flops / total / 1e12
-    sample = ("per step: 1x128 quantization of %d rows of A, 128x128 quantization of %d weight block-rows "
-              "(%d x %d), GEMM of %d x %d outputs over K=%d" % (rows, nb, TILE * nb, d.a.shape[-1], rows, TILE * nb,
-                                                               d.a.shape[-1]))
+    sample = "per step: " + sample_description(name, d, rows, nb)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
@@ -526,10 +569,13 @@ def run_e2e(args, name, d, dev, torch, fq, world):
     """Same step through the public API from pinned host buffers: H2D copy of
     the bf16 inputs, the three kernels, D2H copy of the bf16 result."""
     host = {}
-    keys = ["a", "b"] + (["a2", "b2"] if name == "moe_masked" else ["b2"] if name == "moe_masked_chain" else [])
-    src = {"a": d.a, "b": d.b}
-    if name in ("moe_masked", "moe_masked_chain"):
-        src.update(a2=d.a2, b2=d.b2)
+    if name == "dense_wgrad":
+        keys, src = ["dy", "x"], {"dy": d.dy, "x": d.x}
+    else:
+        keys = ["a", "b"] + (["a2", "b2"] if name == "moe_masked" else ["b2"] if name == "moe_masked_chain" else [])
+        src = {"a": d.a, "b": d.b}
+        if name in ("moe_masked", "moe_masked_chain"):
+            src.update(a2=d.a2, b2=d.b2)
     for k in keys:
         arr = np.ascontiguousarray(src[k]).view(np.int16)
         host[k] = torch.from_numpy(arr).pin_memory()
@@ -575,9 +621,7 @@ def cpu_baseline(name, d):
         fl += f
     value = fl / sum(dts) / 1e12
     return {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": "3 oracle steps, each: 1x128 quantization of %d rows of A, 128x128 quantization of %d weight "
-                      "block-rows, float64 GEMM of the %d x %d outputs they determine (K=%d); %.1f s total" % (
-                          rows, nb, rows, TILE * nb, d.a.shape[-1], sum(dts))}
+            "sample": "3 oracle steps, each: %s; %.1f s total" % (sample_description(name, d, rows, nb), sum(dts))}
 
 
 def main(argv=None):
@@ -588,7 +632,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dense_fprop",
                     choices=["tiny_dense", "dense_fprop", "long_k", "moe_contiguous", "moe_masked", "dense_dgrad",
-                             "moe_masked_chain"])
+                             "moe_masked_chain", "dense_wgrad"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

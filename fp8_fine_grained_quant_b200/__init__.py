@@ -11,12 +11,14 @@ Names and semantics match the C entry points:
 * :func:`fp8_quant_act_1x128`  -- bf16 [M,K] -> E4M3 [M,K] + f32 scales [M,K/128]
 * :func:`fp8_quant_w_128x128`  -- bf16 [N,K] or [G,N,K] -> E4M3 + f32 scales [..,N/128,K/128]
 * :func:`fp8_quant_act_128x1`  -- bf16 [M,K] -> E4M3 [M,K] + f32 scales [ceil(M/128),K] (token-axis tiles)
+* :func:`fp8_quant_act_128x1_t` -- the same groups, codes token-contiguous: E4M3 [K,Mp] (tokens padded to Mp)
 * :func:`fp8_quant_act_1x128_ue8m0`, :func:`fp8_quant_w_128x128_ue8m0` -- the same groups, power-of-two scales
 * :func:`fp8_transpose_w_128x128` -- block-quantized W [..,N,K] -> W^T [..,K,N] (codes and block scales)
 * :func:`fp8_swiglu_quant_1x128` -- GEMM1 output [.., 2I] bf16 -> SwiGLU -> 1x128 E4M3 [.., I] + scales
 * :func:`fp8_gemm_blockscaled` -- C = A * B^T (bf16) with per-128-slab promotion
 * :func:`fp8_grouped_gemm_contiguous` -- MoE grouped GEMM, contiguous layout
 * :func:`fp8_grouped_gemm_masked`     -- MoE grouped GEMM, masked layout
+* :func:`fp8_gemm_wgrad`       -- dW [N,K] = dY^T X over tokens, both operands token-axis quantized
 """
 from __future__ import annotations
 
@@ -26,8 +28,8 @@ from pathlib import Path
 import torch
 
 __all__ = [
-    "fp8_quant_act_1x128", "fp8_quant_w_128x128", "fp8_quant_act_128x1", "fp8_transpose_w_128x128",
-    "fp8_swiglu_quant_1x128",
+    "fp8_quant_act_1x128", "fp8_quant_w_128x128", "fp8_quant_act_128x1", "fp8_quant_act_128x1_t",
+    "fp8_transpose_w_128x128", "fp8_gemm_wgrad", "fp8_swiglu_quant_1x128",
     "fp8_quant_act_1x128_ue8m0", "fp8_quant_w_128x128_ue8m0",
     "fp8_gemm_blockscaled", "fp8_grouped_gemm_contiguous",
     "fp8_grouped_gemm_masked", "fp8_gemm_unpromoted_diag", "get_device_error", "set_wait_timeout_ns",
@@ -46,6 +48,7 @@ EXPORTS = {
     "fp8_quant_act_1x128": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
     "fp8_quant_w_128x128": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "fp8_quant_act_128x1": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
+    "fp8_quant_act_128x1_t": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "fp8_quant_act_1x128_ue8m0": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
     "fp8_quant_w_128x128_ue8m0": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "fp8_transpose_w_128x128": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P]),
@@ -54,6 +57,7 @@ EXPORTS = {
     "fp8_grouped_gemm_contiguous": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "fp8_grouped_gemm_masked": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P]),
     "fp8_gemm_unpromoted_diag": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "fp8_gemm_wgrad": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "fp8q_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fp8q_get_device_error": (ctypes.c_int, [_P]),
     "fp8q_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_uint64]),
@@ -226,6 +230,37 @@ def fp8_quant_act_128x1(x: torch.Tensor, q: torch.Tensor | None = None, s: torch
     return q, s
 
 
+WGRAD_TOKEN_GROUP = 4 * TILE  # fp8_gemm_wgrad contracts over whole groups of four 128-token slabs
+
+
+def fp8_quant_act_128x1_t(x: torch.Tensor, qt: torch.Tensor | None = None, s: torch.Tensor | None = None,
+                          Mp: int | None = None, stream=None):
+    """Token-axis (128x1) quantization with token-contiguous codes, the operand layout of
+    :func:`fp8_gemm_wgrad`.  Returns (qt [K, Mp] float8_e4m3fn, s [Mp/128, K] f32) for tokens padded
+    to Mp (default: M rounded up to 512, what fp8_gemm_wgrad takes); padding tokens get code 0."""
+    _tensor(x, "x", _BF16, (2,))
+    M, K = x.shape
+    _multiple(K, "K")
+    if Mp is None:
+        Mp = -(-M // WGRAD_TOKEN_GROUP) * WGRAD_TOKEN_GROUP
+    _multiple(Mp, "Mp")
+    if Mp < M:
+        raise ValueError("Mp = %d is below the token count %d" % (Mp, M))
+    _tensor(qt, "qt", _FP8)
+    _tensor(s, "s", _F32)
+    _numel(qt, K * Mp, "qt")
+    _numel(s, (Mp // TILE) * K, "s")
+    dev = _device_of(x=x, qt=qt, s=s)
+    if qt is None:
+        qt = torch.empty((K, Mp), dtype=torch.float8_e4m3fn, device=dev)
+    if s is None:
+        s = torch.empty((Mp // TILE, K), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().fp8_quant_act_128x1_t(_p(x), M, K, Mp, _p(qt), _p(s), _stream(stream, dev)),
+               "fp8_quant_act_128x1_t")
+    return qt, s
+
+
 def fp8_transpose_w_128x128(q: torch.Tensor, s: torch.Tensor, qt: torch.Tensor | None = None,
                             st: torch.Tensor | None = None, stream=None):
     """Block-quantized W [N,K] or [G,N,K] (codes + [..,N/128,K/128] scales) -> W^T codes [..,K,N] and
@@ -325,6 +360,35 @@ def fp8_gemm_unpromoted_diag(qa, sa, qb, sb, out: torch.Tensor | None = None, st
     with torch.cuda.device(dev):
         _check(lib().fp8_gemm_unpromoted_diag(_p(qa), _p(sa), _p(qb), _p(sb), _p(out), M, N, K,
                                               _stream(stream, dev)), "fp8_gemm_unpromoted_diag")
+    return out
+
+
+def fp8_gemm_wgrad(q_dy_t, s_dy, q_x_t, s_x, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """dW [N, K] (bf16) = dY^T X from the token-contiguous quantizations of dY [M, N] and
+    X [M, K] (:func:`fp8_quant_act_128x1_t`): q_dy_t [N, Mp], s_dy [Mp/128, N], q_x_t [K, Mp],
+    s_x [Mp/128, K]."""
+    _tensor(q_dy_t, "q_dy_t", _FP8, (2,))
+    _tensor(s_dy, "s_dy", _F32)
+    _tensor(q_x_t, "q_x_t", _FP8, (2,))
+    _tensor(s_x, "s_x", _F32)
+    _tensor(out, "out", _BF16)
+    N, Mp = q_dy_t.shape
+    K = q_x_t.shape[0]
+    if q_x_t.shape[1] != Mp:
+        raise ValueError("q_dy_t and q_x_t differ in tokens (%d, %d)" % (Mp, q_x_t.shape[1]))
+    _multiple(N, "N")
+    _multiple(K, "K")
+    if Mp % WGRAD_TOKEN_GROUP or Mp == 0:
+        raise ValueError("Mp = %d is not a positive multiple of %d" % (Mp, WGRAD_TOKEN_GROUP))
+    _numel(s_dy, (Mp // TILE) * N, "s_dy")
+    _numel(s_x, (Mp // TILE) * K, "s_x")
+    _numel(out, N * K, "out")
+    dev = _device_of(q_dy_t=q_dy_t, s_dy=s_dy, q_x_t=q_x_t, s_x=s_x, out=out)
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().fp8_gemm_wgrad(_p(q_dy_t), _p(s_dy), _p(q_x_t), _p(s_x), _p(out), N, K, Mp,
+                                    _stream(stream, dev)), "fp8_gemm_wgrad")
     return out
 
 

@@ -42,10 +42,11 @@ std::mutex g_dev_mu;
 
 // Per-device set-up, done once: SM count, arch check, status-word address,
 // and the dynamic shared-memory opt-in of every GEMM instantiation.
-template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales>
+template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D = false>
 cudaError_t opt_in_smem() {
-  return cudaFuncSetAttribute(gemm_blockscaled_kernel<BN, STAGES, S, kPromote, kTmaScales>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, GemmSmem<BN, STAGES>::kDynamicBytes);
+  return cudaFuncSetAttribute(gemm_blockscaled_kernel<BN, STAGES, S, kPromote, kTmaScales, k1D1D>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              GemmSmem<BN, STAGES, k1D1D>::kDynamicBytes);
 }
 
 // Output tile 128 x kTileN: 64 FP32 accumulators per epilogue thread, four
@@ -78,6 +79,7 @@ int device_info(DeviceInfo** out) {
         if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kContiguous, true, false>();
         if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kMasked, true, true>();
         if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kMasked, true, false>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kDense, true, true, true>();
         if (e != cudaSuccess) return FP8Q_ERR_CUDA;
       }
       d.ready.store(true, std::memory_order_release);
@@ -138,6 +140,23 @@ int make_scale_map(CUtensorMap* map, const float* base, uint64_t rows, uint64_t 
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
+// Slab-major scale tensor [nkb, rows] f32 (one row per 128-deep slab) with a
+// box of 4 slabs x box_rows: the per-row scales of both weight-gradient
+// operands.  rows % 4 == 0 and a 16-byte-aligned base; slabs past nkb read as
+// zero.
+int make_row_scale_map(CUtensorMap* map, const float* base, uint64_t rows, uint64_t nkb, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FP8Q_ERR_CUDA;
+  const cuuint64_t dims[2] = {rows, nkb};
+  const cuuint64_t strides[1] = {rows * 4};
+  const cuuint32_t box[2] = {box_rows, 4};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- GEMM launch
 struct GemmCall {
   const uint8_t* qa;
@@ -155,7 +174,7 @@ struct GemmCall {
   int promote;
 };
 
-template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales>
+template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D = false>
 int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
   CUtensorMap ma, mb, msa, msb;
   std::memset(&msa, 0, sizeof msa);
@@ -164,7 +183,13 @@ int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
   if (rc) return rc;
   rc = make_operand_map(&mb, g.qb, static_cast<uint64_t>(g.E * g.N), static_cast<uint64_t>(g.K), BN);
   if (rc) return rc;
-  if constexpr (kTmaScales) {
+  if constexpr (k1D1D) {
+    const uint64_t nkb = static_cast<uint64_t>(g.K / kSlabK);
+    rc = make_row_scale_map(&msa, g.sa, static_cast<uint64_t>(g.a_rows), nkb, kBlockM);
+    if (rc) return rc;
+    rc = make_row_scale_map(&msb, g.sb, static_cast<uint64_t>(g.N), nkb, BN);
+    if (rc) return rc;
+  } else if constexpr (kTmaScales) {
     const uint64_t nkb = static_cast<uint64_t>(g.K / kSlabK);
     rc = make_scale_map(&msa, g.sa, static_cast<uint64_t>(g.a_rows), nkb, kBlockM);
     if (rc) return rc;
@@ -192,10 +217,11 @@ int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
   std::memset(&cfg, 0, sizeof cfg);
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = GemmSmem<BN, STAGES>::kDynamicBytes;
+  cfg.dynamicSmemBytes = GemmSmem<BN, STAGES, k1D1D>::kDynamicBytes;
   cfg.stream = stream;
   cudaError_t e =
-      cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<BN, STAGES, S, kPromote, kTmaScales>, ma, mb, msa, msb, a);
+      cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<BN, STAGES, S, kPromote, kTmaScales, k1D1D>, ma, mb, msa, msb,
+                         a);
   if (e != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FP8Q_OK;
@@ -342,7 +368,7 @@ int fp8_quant_act_128x1(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, fl
   const int64_t blocks = ((M + 127) / 128) * (K / 128);
   const int64_t cap = static_cast<int64_t>(dev->num_sms) * 16;
   const int64_t grid = blocks < cap ? blocks : cap;
-  quant_act_128x1_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(static_cast<const uint8_t*>(x_bf16), q, s,
+  quant_act_128x1_kernel<2><<<static_cast<unsigned>(grid), 256, 0, stream>>>(static_cast<const uint8_t*>(x_bf16), q, s,
                                                                            M, K, blocks);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -367,6 +393,26 @@ int fp8_swiglu_quant_1x128(const void* c1_bf16, int64_t rows, int64_t inter, con
   if (grid > cap_grid) grid = cap_grid;
   swiglu_quant_1x128_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(
       static_cast<const uint8_t*>(c1_bf16), qh, sh, inter, tiles, masked_m, masked_m ? cap : 1);
+  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
+int fp8_quant_act_128x1_t(const void* x_bf16, int64_t M, int64_t K, int64_t Mp, uint8_t* qt, float* s,
+                          cudaStream_t stream) {
+  FP8Q_API_RANGE();
+  if (M < 0 || K < 0 || K % 128 || Mp < M || Mp % 128 || Mp >= kMaxRows || K >= kMaxRows) return FP8Q_ERR_SHAPE;
+  if (Mp == 0 || K == 0) return FP8Q_OK;
+  if (!x_bf16 || !qt || !s) return FP8Q_ERR_NULL;
+  if (!aligned(x_bf16, 16) || !aligned(qt, 16) || !aligned(s, 16)) return FP8Q_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  const int64_t blocks = (Mp / 128) * (K / 128);
+  const int64_t cap = static_cast<int64_t>(dev->num_sms) * 16;
+  const int64_t grid = blocks < cap ? blocks : cap;
+  quant_act_128x1_t_kernel<2><<<static_cast<unsigned>(grid), 256, 0, stream>>>(static_cast<const uint8_t*>(x_bf16), qt,
+                                                                             s, M, K, Mp, blocks);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FP8Q_OK;
@@ -447,6 +493,27 @@ int fp8_grouped_gemm_masked(const uint8_t* qa, const float* sa, const uint8_t* q
   if (!aligned(masked_m, 4)) return FP8Q_ERR_ALIGN;
   GemmCall g{qa, sa, qb, sb, c_bf16, nullptr, masked_m, E * cap, cap, N, K, E, cap / kBlockM, expected_m, 1};
   return run_gemm<Sched::kMasked>(g, stream);
+}
+
+int fp8_gemm_wgrad(const uint8_t* q_dy_t, const float* s_dy, const uint8_t* q_x_t, const float* s_x, void* dw_bf16,
+                   int64_t N, int64_t K, int64_t Mp, cudaStream_t stream) {
+  FP8Q_API_RANGE();
+  // the contraction runs over Mp tokens in whole groups of four 128-token
+  // slabs: the per-row scales of both operands are staged a group at a time
+  if (N < 0 || K < 0 || Mp < 512 || N % 128 || K % 128 || Mp % 512 || N >= kMaxRows || K >= kMaxRows ||
+      Mp >= kMaxRows)
+    return FP8Q_ERR_SHAPE;
+  if (N == 0 || K == 0) return FP8Q_OK;
+  if (!q_dy_t || !s_dy || !q_x_t || !s_x || !dw_bf16) return FP8Q_ERR_NULL;
+  if (!aligned(q_dy_t, 16) || !aligned(q_x_t, 16) || !aligned(dw_bf16, 16) || !aligned(s_dy, 16) ||
+      !aligned(s_x, 16))
+    return FP8Q_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  // C [N, K] = A [N, Mp] * B [K, Mp]^T: GEMM rows N, columns K, depth Mp
+  GemmCall g{q_dy_t, s_dy, q_x_t, s_x, dw_bf16, nullptr, nullptr, N, N, K, Mp, 1, N / kBlockM, 0, 1};
+  return launch_gemm<kTileN, kStages128, Sched::kDense, true, true, true>(g, *dev, stream);
 }
 
 const char* fp8q_status_string(int status) {

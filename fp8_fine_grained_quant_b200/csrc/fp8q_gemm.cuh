@@ -73,7 +73,7 @@ struct Tile {
   int32_t rows;   // valid rows in this tile (<= 128)
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool k1D1D = false>
 struct GemmSmem {
   static constexpr uint32_t kABytes = kBlockM * kSlabK;  // 16 KB
   static constexpr uint32_t kBBytes = BN * kSlabK;
@@ -90,16 +90,19 @@ struct GemmSmem {
   static constexpr uint32_t kOffPrefix = (kOffMisc + 16 + 15) / 16 * 16;
   // Scale ring (TMA-staged scales): per group of kScaleGroup slabs, the 128
   // tile rows' activation scales as a [128][kScaleGroup] f32 box and the
-  // weight block's kScaleGroup scales.
+  // weight block's kScaleGroup scales.  With per-row scales on both operands
+  // (k1D1D, the weight-gradient GEMM) both boxes are slab-major,
+  // [kScaleGroup][128] and [kScaleGroup][BN].
   static constexpr int kScaleGroup = 4;
   static constexpr int kScaleSlots = 4;
   static constexpr uint32_t kSaSlotBytes = kBlockM * kScaleGroup * 4;  // 2 KB
-  static constexpr uint32_t kSbSlotBytes = kScaleGroup * 4;             // 16 B
-  static constexpr uint32_t kSbSlotStride = 128;                        // TMA destinations 128-byte aligned
+  static constexpr uint32_t kSbSlotBytes = k1D1D ? BN * kScaleGroup * 4 : kScaleGroup * 4;
+  static constexpr uint32_t kSbSlotStride = k1D1D ? kSbSlotBytes : 128;  // TMA destinations 128-byte aligned
   static constexpr uint32_t kOffSa = (kOffPrefix + 4 * (kMaxMaskedExperts + 1) + 127) / 128 * 128;
   static constexpr uint32_t kOffSb = kOffSa + kScaleSlots * kSaSlotBytes;
   static constexpr uint32_t kBytes = kOffSb + kScaleSlots * kSbSlotStride;
   static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack for 1024-byte alignment
+  static_assert(kDynamicBytes <= 227u * 1024u, "shared memory per CTA");
 };
 
 // ----------------------------------------------------------------- scheduler
@@ -215,13 +218,13 @@ struct Bars {
 };
 
 // TMA producer `who` of two: loads the slabs j with j % 2 == who.
-template <int BN, int STAGES, Sched S, bool kTmaScales>
+template <int BN, int STAGES, Sched S, bool kTmaScales, bool k1D1D>
 __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensorMap* tma_b,
                                         const CUtensorMap* tma_sa, const CUtensorMap* tma_sb, const GemmArgs& args,
                                         const int32_t* prefix, uint32_t s_base,
                                         Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
                                         int32_t total, uint32_t who) {
-  using L = GemmSmem<BN, STAGES>;
+  using L = GemmSmem<BN, STAGES, k1D1D>;
   const int nnb = args.N / 128;
   int stage = 0;
   uint32_t phase = 0, j = 0;
@@ -240,11 +243,18 @@ __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensor
         tma_load_2d(s_base + L::kOffA + stage * L::kABytes, tma_a, bars.full(stage), kb * kSlabK, tile.a_row);
         tma_load_2d(s_base + L::kOffB + stage * L::kBBytes, tma_b, bars.full(stage), kb * kSlabK, tile.b_row);
         if (group_start) {
-          // x = kb is a multiple of 4 f32: a 16-byte-aligned start
           const uint32_t slot = group % L::kScaleSlots;
-          tma_load_2d(s_base + L::kOffSa + slot * L::kSaSlotBytes, tma_sa, bars.full(stage), kb, tile.a_row);
-          tma_load_2d(s_base + L::kOffSb + slot * L::kSbSlotStride, tma_sb, bars.full(stage), kb,
-                      tile.e * nnb + tile.n0 / 128);
+          if constexpr (k1D1D) {
+            // slab-major [nkb, rows] scales: x = the tile's first row, a
+            // multiple of 128 f32 (16-byte aligned); slabs past nkb read as 0
+            tma_load_2d(s_base + L::kOffSa + slot * L::kSaSlotBytes, tma_sa, bars.full(stage), tile.a_row, kb);
+            tma_load_2d(s_base + L::kOffSb + slot * L::kSbSlotStride, tma_sb, bars.full(stage), tile.b_row, kb);
+          } else {
+            // x = kb is a multiple of 4 f32: a 16-byte-aligned start
+            tma_load_2d(s_base + L::kOffSa + slot * L::kSaSlotBytes, tma_sa, bars.full(stage), kb, tile.a_row);
+            tma_load_2d(s_base + L::kOffSb + slot * L::kSbSlotStride, tma_sb, bars.full(stage), kb,
+                        tile.e * nnb + tile.n0 / 128);
+          }
         }
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -329,11 +339,11 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
 // back as soon as the values are in registers, then applies
 // acc += (sa * sb) * partial.  The completion probe of the next slab is issued
 // before this slab's work and read after it.
-template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales>
+template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D>
 __device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, const int32_t* prefix,
                                          Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
                                          int32_t total, uint32_t tmem_base, int warp, int lane) {
-  using L = GemmSmem<BN, STAGES>;
+  using L = GemmSmem<BN, STAGES, k1D1D>;
   constexpr int kCols = BN / 2;
   constexpr int kGroup = kCols < 64 ? kCols : 64;
   constexpr int kGroups = kCols / kGroup;
@@ -346,6 +356,9 @@ __device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, 
                 "two threads take alternate slabs per role; with an even stage count each waits only on its "
                 "own stages, so no parity wait can pass on an earlier phase");
   static_assert(kPromote || !kTmaScales, "staged scales serve the per-slab promotion only");
+  // k1D1D also needs whole scale groups (nkb % 4 == 0, checked by the host):
+  // the slot bound above counts four slabs per group
+  static_assert(!k1D1D || (kTmaScales && S == Sched::kDense), "per-row B scales come staged, dense layout only");
   constexpr bool promote = kPromote;
   const int quad = warp & 3;
   const int half = (warp - 4) >> 2;
@@ -383,12 +396,18 @@ __device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, 
         if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
       }
       float sa_smem = 0.0f, sb_smem = 0.0f;
+      uint32_t sb_cols = 0;  // k1D1D: shared address of this half's column scales for the slab
       if constexpr (kTmaScales) {
         // this slab's scales, staged with its group's first stage
         const uint32_t slot = group % L::kScaleSlots;
         const uint32_t k = static_cast<uint32_t>(it % L::kScaleGroup);
-        sa_smem = lds_f32(s_base + L::kOffSa + slot * L::kSaSlotBytes + r * (L::kScaleGroup * 4) + k * 4);
-        sb_smem = lds_f32(s_base + L::kOffSb + slot * L::kSbSlotStride + k * 4);
+        if constexpr (k1D1D) {
+          sa_smem = lds_f32(s_base + L::kOffSa + slot * L::kSaSlotBytes + k * (kBlockM * 4) + r * 4);
+          sb_cols = s_base + L::kOffSb + slot * L::kSbSlotStride + k * (BN * 4) + half * (kCols * 4);
+        } else {
+          sa_smem = lds_f32(s_base + L::kOffSa + slot * L::kSaSlotBytes + r * (L::kScaleGroup * 4) + k * 4);
+          sb_smem = lds_f32(s_base + L::kOffSb + slot * L::kSbSlotStride + k * 4);
+        }
         if (k == L::kScaleGroup - 1) ++group;
       }
       tc_fence_after();
@@ -432,8 +451,21 @@ __device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, 
             }
           }
         }
+        if constexpr (k1D1D) {
+          // acc += (sa_r * sb_c) * partial, column by column: the B scales of
+          // 4 columns per (broadcast) shared load
+          const uint64_t sa2 = pack_f32x2(sa_smem);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ffma2(acc[g * 32 + i], v[i], scale2);
+          for (int i = 0; i < 32; i += 2) {
+            uint64_t sb01, sb23;
+            lds_v2_b64(sb_cols + (g * kGroup + 2 * i) * 4, sb01, sb23);
+            ffma2(acc[g * 32 + i], v[i], mul_f32x2(sa2, sb01));
+            ffma2(acc[g * 32 + i + 1], v[i + 1], mul_f32x2(sa2, sb23));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ffma2(acc[g * 32 + i], v[i], scale2);
+        }
       }
       ready = __all_sync(0xFFFFFFFFu, next_done);
       if (promote) {
@@ -462,12 +494,12 @@ __device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, 
 }
 
 // ----------------------------------------------------------------- kernel
-template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales>
+template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                             const __grid_constant__ CUtensorMap tma_sa, const __grid_constant__ CUtensorMap tma_sb,
                             const GemmArgs args) {
-  using L = GemmSmem<BN, STAGES>;
+  using L = GemmSmem<BN, STAGES, k1D1D>;
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "UMMA N for M=128 must be a multiple of 16 in [16,256]");
 
   extern __shared__ uint8_t smem_raw[];
@@ -528,7 +560,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t n_mma = promote ? 2u : 1u;
     if (lane == 0) {
       if (warp == 0 || warp == 3)
-        produce<BN, STAGES, S, kTmaScales>(&tma_a, &tma_b, &tma_sa, &tma_sb, args, prefix, s_base, bars, wc, total,
+        produce<BN, STAGES, S, kTmaScales, k1D1D>(&tma_a, &tma_b, &tma_sa, &tma_sb, args, prefix, s_base, bars, wc, total,
                                            warp == 0 ? 0u : 1u);
       else if (static_cast<uint32_t>(warp - 1) < n_mma)
         issue_mma<BN, STAGES, S, kPromote>(args, prefix, s_base, bars, wc, total, tmem_base, warp - 1, n_mma);
@@ -537,7 +569,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // all TMEM slab buffers start free: every lane releases them for the first slabs
     if (promote)
       for (int b = 0; b < L::kAccBufs; ++b) mbar_arrive(bars.full(b));
-    epilogue<BN, STAGES, S, kPromote, kTmaScales>(s_base, args, prefix, bars, wc, total, tmem_base, warp, lane);
+    epilogue<BN, STAGES, S, kPromote, kTmaScales, k1D1D>(s_base, args, prefix, bars, wc, total, tmem_base, warp, lane);
   }
 
   __syncwarp();

@@ -108,6 +108,11 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
   return v;
 }
 
+// 16 bytes of shared memory as two packed FP32 pairs; addr 16-byte aligned.
+__device__ __forceinline__ void lds_v2_b64(uint32_t addr, uint64_t& a, uint64_t& b) {
+  asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr) : "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -273,7 +273,9 @@ __device__ __noinline__ uint2 quantize8_cols_exact(uint32_t w0, uint32_t w1, uin
   return make_uint2(c[0], c[1]);
 }
 
-__global__ void __launch_bounds__(256) quant_act_128x1_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
+// kMinBlocks: CTAs per SM the register budget is fitted to (2: 128 registers).
+template <int kMinBlocks = 2>
+__global__ void __launch_bounds__(256, kMinBlocks) quant_act_128x1_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
                                                               float* __restrict__ s, int64_t M, int64_t K,
                                                               int64_t num_blocks) {
   __shared__ float col_max[8][16][8];  // [warp][column group][column]
@@ -356,49 +358,189 @@ __global__ void __launch_bounds__(256) quant_act_128x1_kernel(const uint8_t* __r
 }
 
 // ---------------------------------------------------------------------------
+// Token-axis (128x1) quantization with token-contiguous codes, for the weight
+// gradient dW = dY^T X.  Written as C = A * B^T, that GEMM contracts over
+// tokens: A = dY^T [N, Mp] and B = X^T [K, Mp], each row carrying one scale
+// per 128-token slab.  This kernel quantizes x [M, K] (tokens x channels) in
+// the groups of quant_act_128x1_kernel (same scales s [Mp/128, K], which is
+// the slab-major layout the GEMM stages) and writes the codes transposed,
+// qt [K, Mp] for a padded token count Mp >= M (a multiple of 128); tokens
+// past M get code 0 and whole padding groups scale 1.
+//
+// Per 128x128 block a thread owns 8 tokens x 8 channels, as in the untransposed
+// kernel.  Its 8x8 code bytes are transposed in registers (byte permutes) and
+// written to a shared [channel][token] tile whose 8-byte slots are XOR-
+// swizzled by channel / 8 (two wavefronts per warp store); each channel row
+// then leaves as eight coalesced 16-byte stores.
+// ---------------------------------------------------------------------------
+
+// 4x4 byte transpose: w[i] holds row i (byte j = column j); afterwards w[j]
+// holds column j (byte i = row i).
+__device__ __forceinline__ void transpose4x4_bytes(uint32_t& w0, uint32_t& w1, uint32_t& w2, uint32_t& w3) {
+  const uint32_t x0 = __byte_perm(w0, w2, 0x5410), x2 = __byte_perm(w0, w2, 0x7632);
+  const uint32_t x1 = __byte_perm(w1, w3, 0x5410), x3 = __byte_perm(w1, w3, 0x7632);
+  w0 = __byte_perm(x0, x1, 0x6240);
+  w1 = __byte_perm(x0, x1, 0x7351);
+  w2 = __byte_perm(x2, x3, 0x6240);
+  w3 = __byte_perm(x2, x3, 0x7351);
+}
+
+// 8x8 byte transpose of rows (lo[r]: bytes 0-3, hi[r]: bytes 4-7): as 2x2
+// blocks of 4x4, [[A, B], [C, D]]^T = [[A^T, C^T], [B^T, D^T]].
+__device__ __forceinline__ void transpose8x8_bytes(uint32_t (&lo)[8], uint32_t (&hi)[8]) {
+  transpose4x4_bytes(lo[0], lo[1], lo[2], lo[3]);  // A
+  transpose4x4_bytes(lo[4], lo[5], lo[6], lo[7]);  // C
+  transpose4x4_bytes(hi[0], hi[1], hi[2], hi[3]);  // B
+  transpose4x4_bytes(hi[4], hi[5], hi[6], hi[7]);  // D
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t b = hi[i];  // B^T row i becomes row 4 + i, low half
+    hi[i] = lo[4 + i];         // C^T row i: row i, high half
+    lo[4 + i] = b;
+  }
+}
+
+// kMinBlocks: CTAs per SM the register budget is fitted to (2: 128 registers).
+template <int kMinBlocks = 2>
+__global__ void __launch_bounds__(256, kMinBlocks) quant_act_128x1_t_kernel(const uint8_t* __restrict__ x,
+                                                                uint8_t* __restrict__ qt, float* __restrict__ s,
+                                                                int64_t M, int64_t K, int64_t Mp,
+                                                                int64_t num_blocks) {
+  __shared__ float col_max[8][16][8];            // [warp][column group][column]
+  __shared__ __align__(16) uint8_t tile[128 * 128];  // [channel][token], 8-byte slots swizzled
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cg = tid & 15, rg = tid >> 4;
+  const int64_t nkc = K >> 7;
+  for (int64_t b = blockIdx.x; b < num_blocks; b += gridDim.x) {
+    const int64_t mb = b / nkc, kc = b % nkc;
+    const int64_t col0 = kc * 128 + cg * 8;
+    const int64_t row0 = mb * 128 + rg * 8;
+    uint4 v[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int64_t row = row0 + r;
+      v[r] = row < M ? ld_nc_v4(x + (row * K + col0) * 2) : make_uint4(0, 0, 0, 0);
+    }
+    float m[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) m[c] = 0.0f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const uint32_t w[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        m[2 * i] = fmaxf(m[2 * i], fabsf(__uint_as_float(w[i] << 16)));
+        m[2 * i + 1] = fmaxf(m[2 * i + 1], fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) m[c] = fmaxf(m[c], __shfl_xor_sync(0xFFFFFFFFu, m[c], 16));
+    if (lane < 16) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) col_max[warp][cg][c] = m[c];
+    }
+    __syncthreads();
+    float sc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float a = col_max[0][cg][c];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) a = fmaxf(a, col_max[w][cg][c]);
+      sc[c] = group_scale(a);
+    }
+    if (rg == 0) {
+      float* sd = s + mb * K + col0;
+      *reinterpret_cast<float4*>(sd) = make_float4(sc[0], sc[1], sc[2], sc[3]);
+      *reinterpret_cast<float4*>(sd + 4) = make_float4(sc[4], sc[5], sc[6], sc[7]);
+    }
+    uint64_t lo2[4], hi2[4];
+    bool exact_only = false;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float r0 = __frcp_rn(sc[2 * i]), r1 = __frcp_rn(sc[2 * i + 1]);
+      asm("mov.b64 %0, {%1, %2};" : "=l"(lo2[i]) : "f"(__fmul_rn(r0, 1.0f - 0x1p-20f)), "f"(__fmul_rn(r1, 1.0f - 0x1p-20f)));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[i]) : "f"(__fmul_rn(r0, 1.0f + 0x1p-20f)), "f"(__fmul_rn(r1, 1.0f + 0x1p-20f)));
+      exact_only |= sc[2 * i] < kMinFastScale || sc[2 * i + 1] < kMinFastScale;
+    }
+    // codes of the 8 tokens (zero rows past M give code 0)
+    uint32_t clo[8], chi[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const uint32_t w[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+      uint32_t lo[2], hi[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint64_t x0 = bf16x2_to_f32x2(w[2 * h]), x1 = bf16x2_to_f32x2(w[2 * h + 1]);
+        lo[h] = e4m3x4_from_f32x2(mul_f32x2(x0, lo2[2 * h]), mul_f32x2(x1, lo2[2 * h + 1]));
+        hi[h] = e4m3x4_from_f32x2(mul_f32x2(x0, hi2[2 * h]), mul_f32x2(x1, hi2[2 * h + 1]));
+      }
+      uint2 out = make_uint2(lo[0], lo[1]);
+      if (exact_only || ((lo[0] ^ hi[0]) | (lo[1] ^ hi[1])) != 0u)
+        out = quantize8_cols_exact(w[0], w[1], w[2], w[3], sc[0], sc[1], sc[2], sc[3], sc[4], sc[5], sc[6], sc[7]);
+      clo[r] = out.x;
+      chi[r] = out.y;
+    }
+    transpose8x8_bytes(clo, chi);  // now channel c: tokens 0-3 in clo[c], 4-7 in chi[c]
+    // channel row cg*8 + c, logical 8-byte slot rg, physical slot rg ^ cg
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      *reinterpret_cast<uint2*>(tile + (cg * 8 + c) * 128 + ((rg ^ cg) << 3)) = make_uint2(clo[c], chi[c]);
+    __syncthreads();
+    uint8_t* dst = qt + (kc * 128) * Mp + mb * 128;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = tid + 256 * i, row = c >> 3, ch = c & 7;
+      const int swz = row >> 3;  // the row's column group, 0..15
+      // logical slots 2ch, 2ch+1 sit in physical 16-byte chunk ch ^ (swz / 2),
+      // their halves swapped when swz is odd
+      uint4 o = *reinterpret_cast<const uint4*>(tile + row * 128 + ((ch ^ (swz >> 1)) << 4));
+      if (swz & 1) o = make_uint4(o.z, o.w, o.x, o.y);
+      *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(row) * Mp + ch * 16) = o;
+    }
+    __syncthreads();  // col_max and the tile are reused by the next block
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Transposition of 128x128-block-quantized weights: codes [G, N, K] -> [G, K, N]
 // and block scales [G, N/128, K/128] -> [G, K/128, N/128].  A 128x128 block of
 // W^T is the transpose of W's block (same amax, same scale, the same codes),
 // so the forward GEMM on the transposed codes computes dY * W (the
-// activation-gradient GEMM).  One 256-thread CTA per block through a padded
-// shared tile; 16-byte loads and stores.
+// activation-gradient GEMM).
+//
+// One 256-thread CTA per block, no shared memory: thread (l = t % 16,
+// j = t / 16) loads the 8x8 bytes at rows 8l.., columns 8j.. (eight 8-byte
+// loads; the two warps reading a 32-byte sector share it through L1),
+// transposes them in registers and stores eight 8-byte pieces, rows 8j..,
+// columns 8l.. of the output: each warp store writes two full 128-byte rows.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ uint2 ldg_u2(const uint8_t* p) {
+  return __ldg(reinterpret_cast<const uint2*>(p));
+}
+
 __global__ void __launch_bounds__(256) transpose_w_128x128_kernel(const uint8_t* __restrict__ qw,
                                                                   const float* __restrict__ sw,
                                                                   uint8_t* __restrict__ qt, float* __restrict__ st,
                                                                   int64_t N, int64_t K, int64_t num_blocks) {
-  constexpr int kPitch = 128 + 16;  // bytes per shared row (keeps 16-byte alignment)
-  __shared__ __align__(16) uint8_t tile[128 * kPitch];
   const int tid = threadIdx.x;
+  const int l = tid & 15, j = tid >> 4;
   const int64_t nkb = K >> 7, nnb = N >> 7;
   for (int64_t b = blockIdx.x; b < num_blocks; b += gridDim.x) {
     const int64_t g = b / (nnb * nkb), rem = b % (nnb * nkb);
     const int64_t nb = rem / nkb, kb = rem % nkb;
-    const uint8_t* src = qw + (g * N + nb * 128) * K + kb * 128;
-    // 128 rows x 8 chunks of 16 bytes: thread t loads chunks t, t+256, t+512, t+768
+    const uint8_t* src = qw + (g * N + nb * 128 + 8 * l) * K + kb * 128 + 8 * j;
+    uint32_t lo[8], hi[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int c = tid + 256 * i, row = c >> 3, ch = c & 7;
-      *reinterpret_cast<uint4*>(tile + row * kPitch + ch * 16) =
-          ld_nc_v4(src + static_cast<int64_t>(row) * K + ch * 16);
+    for (int r = 0; r < 8; ++r) {
+      const uint2 v = ldg_u2(src + static_cast<int64_t>(r) * K);
+      lo[r] = v.x;
+      hi[r] = v.y;
     }
-    __syncthreads();
-    uint8_t* dst = qt + (g * K + kb * 128) * N + nb * 128;
+    transpose8x8_bytes(lo, hi);  // lo[c], hi[c]: column 8j + c, rows 8l .. 8l + 7
+    uint8_t* dst = qt + (g * K + kb * 128 + 8 * j) * N + nb * 128 + 8 * l;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int c = tid + 256 * i, orow = c >> 3, ch = c & 7;  // output row = input column
-      uint32_t wv[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        uint32_t acc = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc |= static_cast<uint32_t>(tile[(ch * 16 + w * 4 + j) * kPitch + orow]) << (8 * j);
-        wv[w] = acc;
-      }
-      *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(orow) * N + ch * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-    }
+    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint2*>(dst + static_cast<int64_t>(c) * N) = make_uint2(lo[c], hi[c]);
     if (tid == 0) st[(g * nkb + kb) * nnb + nb] = sw[(g * nnb + nb) * nkb + kb];
-    __syncthreads();  // the tile is reused by the next block
   }
 }
 

@@ -142,6 +142,22 @@ FP8Q_API int fp8_swiglu_quant_1x128(const void* c1_bf16, int64_t rows, int64_t i
                                     int64_t cap, uint8_t* qh, float* sh, cudaStream_t stream);
 
 /*
+ * The same token-axis quantization with the codes written token-contiguous,
+ * the operand layout of the weight-gradient GEMM fp8_gemm_wgrad:
+ *   x_bf16 : [M, K] bf16 (tokens x channels), read only.
+ *   Mp     : padded token count, a multiple of 128 with Mp >= M
+ *            (fp8_gemm_wgrad takes multiples of 512).
+ *   qt     : [K, Mp] E4M3 codes, written; qt[k, m] is the code of x[m, k],
+ *            and 0 for m >= M.
+ *   s      : [Mp/128, K] float32, written; rows below ceil(M/128) are the
+ *            scales of fp8_quant_act_128x1, the rows of groups made only of
+ *            padding are 1 (the zero-group rule).
+ * K a multiple of 128; any M >= 0.  x, qt and s 16-byte aligned.
+ */
+FP8Q_API int fp8_quant_act_128x1_t(const void* x_bf16, int64_t M, int64_t K, int64_t Mp, uint8_t* qt, float* s,
+                                   cudaStream_t stream);
+
+/*
  * Transposition of 128x128-block-quantized weights (for the activation
  * gradient dX = dY W, the Dgrad GEMM of the same Figure 6): a 128x128 block
  * of W^T has the same amax, scale and codes as W's block, transposed.
@@ -204,6 +220,22 @@ FP8Q_API int fp8_grouped_gemm_contiguous(const uint8_t* qa, const float* sa, con
 FP8Q_API int fp8_grouped_gemm_masked(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb,
                             const int32_t* masked_m, void* c_bf16, int64_t E, int64_t cap, int64_t N, int64_t K,
                             int64_t expected_m, cudaStream_t stream);
+
+/*
+ * Weight-gradient GEMM dW = dY^T X over tokens ("The Insider Secrets Of
+ * Deepseek Discovered", Figure 6, Wgrad in FP8), with both operands
+ * quantized along tokens (fp8_quant_act_128x1_t of dY [M, N] and of X [M, K]):
+ *   dW[n,k] = bf16_rne( sum_mb s_dy[mb,n] * s_x[mb,k] * sum_{m in slab mb} dY[m,n] * X[m,k] )
+ * with the same per-slab FP32 promotion as fp8_gemm_blockscaled, each slab's
+ * partial scaled by one A-row scale and one scale per output column.
+ *   q_dy_t : [N, Mp] E4M3, s_dy : [Mp/128, N] f32
+ *   q_x_t  : [K, Mp] E4M3, s_x  : [Mp/128, K] f32
+ *   dw_bf16: [N, K] bf16, written.
+ * N, K multiples of 128; Mp a multiple of 512 (whole groups of four token
+ * slabs), Mp >= 512.  Every pointer 16-byte aligned.
+ */
+FP8Q_API int fp8_gemm_wgrad(const uint8_t* q_dy_t, const float* s_dy, const uint8_t* q_x_t, const float* s_x,
+                            void* dw_bf16, int64_t N, int64_t K, int64_t Mp, cudaStream_t stream);
 
 /*
  * Accumulation diagnostic ("The Insider Secrets Of Deepseek Discovered": the

@@ -217,3 +217,30 @@ def test_sizes_beyond_the_limits_are_refused(name, args):
 ])
 def test_swiglu_quant_validation(args, expect):
     assert _call("fp8_swiglu_quant_1x128", *args) == expect
+@pytest.mark.parametrize("args,expect", [
+    ((A16, 4, 100, 128, A16, A16, None), fq.ERR_SHAPE),
+    ((A16, -1, 128, 128, A16, A16, None), fq.ERR_SHAPE),
+    ((A16, 200, 128, 128, A16, A16, None), fq.ERR_SHAPE),   # padded count below the tokens
+    ((A16, 4, 128, 200, A16, A16, None), fq.ERR_SHAPE),     # padded count not a multiple of 128
+    ((A16, 0, 128, 0, A16, A16, None), fq.OK),
+    ((None, 4, 128, 128, A16, A16, None), fq.ERR_NULL),
+    ((A16, 4, 128, 128, A16_ONLY + 4, A16, None), fq.ERR_ALIGN),
+    ((A16, 4, 128, 512, A16, A4, None), fq.ERR_ALIGN),
+])
+def test_quant_act_128x1_t_validation(args, expect):
+    assert _call("fp8_quant_act_128x1_t", *args) == expect
+
+
+@pytest.mark.parametrize("nkm,ptrs,expect", [
+    ((256, 256, 100), (A16,) * 5, fq.ERR_SHAPE),    # tokens not a multiple of 128
+    ((256, 256, 384), (A16,) * 5, fq.ERR_SHAPE),    # nor of a group of four slabs
+    ((256, 256, 0), (A16,) * 5, fq.ERR_SHAPE),      # at least one group
+    ((200, 256, 512), (A16,) * 5, fq.ERR_SHAPE),
+    ((256, 200, 512), (A16,) * 5, fq.ERR_SHAPE),
+    ((0, 256, 512), (A16,) * 5, fq.OK),
+    ((256, 256, 512), (A16, None, A16, A16, A16), fq.ERR_NULL),
+    ((256, 256, 512), (A16, A4, A16, A16, A16), fq.ERR_ALIGN),   # row scales are staged in 16-byte boxes
+    ((256, 256, 512), (A16, A16, A16, A16, A1), fq.ERR_ALIGN),
+])
+def test_wgrad_validation(nkm, ptrs, expect):
+    assert _call("fp8_gemm_wgrad", *ptrs, *nkm, None) == expect

@@ -96,3 +96,72 @@ def test_dgrad_through_the_forward_gemm(dev, M, N, K):
     oq_w, os_w = oracle.quant_w_128x128(w)
     ref = oracle.dgrad(oq_dy, os_dy, oq_w, os_w)
     assert_gemm_close(bf16_bits_of(dx), ref, "dgrad %dx%dx%d" % (M, N, K))
+
+
+def _pad_tokens(x, Mp):
+    return np.pad(x, ((0, Mp - x.shape[0]), (0, 0)))
+
+
+@pytest.mark.parametrize("M,K,pad", [(128, 128, 128), (256, 384, 512), (200, 256, 128), (1, 128, 512),
+                                     (1000, 640, 128), (1000, 640, 512)])
+def test_token_contiguous_quant_matches_oracle(dev, M, K, pad):
+    """Token-axis groups with the codes written token-contiguous: qt[k, m] is
+    the code of x[m, k]; padding tokens (m >= M) get code 0 and groups made
+    only of padding scale 1."""
+    rng = np.random.default_rng(M * 11 + K)
+    x = _bits(rng, (M, K), outliers=max(1, M * K // 5000), chan=True)
+    if M > 10:
+        x[3, :] = 0
+        x[:, 5] = 0
+    Mp = -(-M // pad) * pad
+    qt, s = fq.fp8_quant_act_128x1_t(to_torch_bf16(x, dev), Mp=Mp)
+    torch.cuda.synchronize(dev)
+    assert fq.get_device_error(device=dev) == fq.OK
+    oq, os_ = oracle.quant_act_128x1(_pad_tokens(x, Mp))
+    assert np.array_equal(oq[M:], np.zeros_like(oq[M:]))
+    assert np.all(os_[-(-M // TILE):] == 1.0)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+    assert np.array_equal(bytes_of(qt).reshape(K, Mp), np.ascontiguousarray(oq.T))
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 384), (300, 128, 256), (1024, 512, 640), (128, 128, 128)])
+def test_wgrad_matches_oracle(dev, M, N, K):
+    """dW = dY^T X over tokens, both operands in token-axis groups."""
+    rng = np.random.default_rng(M + 3 * N + 7 * K)
+    dy = _bits(rng, (M, N), outliers=4, chan=True)
+    x = _bits(rng, (M, K), outliers=4, chan=True)
+    q_dy_t, s_dy = fq.fp8_quant_act_128x1_t(to_torch_bf16(dy, dev))
+    q_x_t, s_x = fq.fp8_quant_act_128x1_t(to_torch_bf16(x, dev))
+    dw = fq.fp8_gemm_wgrad(q_dy_t, s_dy, q_x_t, s_x)
+    torch.cuda.synchronize(dev)
+    assert fq.get_device_error(device=dev) == fq.OK
+    # zero tokens up to the padded count change neither a group's amax nor the sums
+    Mp = -(-M // 512) * 512
+    oq_dy, os_dy = oracle.quant_act_128x1(_pad_tokens(dy, Mp))
+    oq_x, os_x = oracle.quant_act_128x1(_pad_tokens(x, Mp))
+    ref = oracle.wgrad(oq_dy, os_dy, oq_x, os_x)
+    assert_gemm_close(bf16_bits_of(dw), ref, "wgrad %dx%dx%d" % (M, N, K))
+
+
+def test_wgrad_full_size_sampled_rows(dev):
+    """The dense_fprop layer's weight gradient: dY and X [4096, 7168], dW
+    [7168, 7168] over 4096 tokens; the first and last row of every 128-row
+    tile of dW against the oracle."""
+    d = wl.dense_fprop()
+    rng = np.random.default_rng(9)
+    dy = _bits(rng, d.a.shape, chan=True)
+    x = d.a
+    q_dy_t, s_dy = fq.fp8_quant_act_128x1_t(to_torch_bf16(dy, dev))
+    q_x_t, s_x = fq.fp8_quant_act_128x1_t(to_torch_bf16(x, dev))
+    dw = fq.fp8_gemm_wgrad(q_dy_t, s_dy, q_x_t, s_x)
+    torch.cuda.synchronize(dev)
+    assert fq.get_device_error(device=dev) == fq.OK
+    N = dy.shape[1]
+    rows = sorted({r for t in range(N // TILE) for r in (t * TILE, t * TILE + TILE - 1)})
+    oq_dy, os_dy = oracle.quant_act_128x1(dy)
+    oq_x, os_x = oracle.quant_act_128x1(x)
+    # the operands themselves are bit-exact (checked on the small shapes above); spot-check them here too
+    assert np.array_equal(s_dy.cpu().numpy().view(np.uint32), os_dy.view(np.uint32))
+    ref = oracle.wgrad(oq_dy, os_dy, oq_x, os_x, rows=rows)
+    got = bf16_bits_of(dw)[rows]
+    assert_gemm_close(got, ref, "wgrad full size, %d sampled rows" % len(rows))

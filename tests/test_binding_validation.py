@@ -190,3 +190,40 @@ def test_swiglu_quant_buffers():
         fq.fp8_swiglu_quant_1x128(c1, sh=z(7, dtype=f32))
     with pytest.raises(ValueError, match="CUDA tensor"):
         fq.fp8_swiglu_quant_1x128(c1, masked_m=z(2, dtype=i32))
+def test_token_contiguous_quantizer_buffers():
+    x = z(200, 256, dtype=bf16)
+    with pytest.raises(ValueError, match="qt holds 51200 elements, the call needs 131072"):
+        fq.fp8_quant_act_128x1_t(x, qt=z(256, 200))       # tokens padded to 512 by default
+    with pytest.raises(ValueError, match="qt holds 51200 elements, the call needs 65536"):
+        fq.fp8_quant_act_128x1_t(x, qt=z(256, 200), Mp=256)
+    with pytest.raises(ValueError, match="s holds 256"):
+        fq.fp8_quant_act_128x1_t(x, s=z(256, dtype=f32))
+    with pytest.raises(ValueError, match="below the token count"):
+        fq.fp8_quant_act_128x1_t(x, Mp=128)
+    with pytest.raises(ValueError, match="Mp = 300"):
+        fq.fp8_quant_act_128x1_t(x, Mp=300)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fq.fp8_quant_act_128x1_t(x)
+
+
+def test_wgrad_buffers():
+    def args(N=256, K=384, Mp=512):
+        return [z(N, Mp), z(Mp // 128, N, dtype=f32), z(K, Mp), z(Mp // 128, K, dtype=f32)]
+    a = args()
+    a[2] = z(384, 384)
+    with pytest.raises(ValueError, match="differ in tokens"):
+        fq.fp8_gemm_wgrad(*a)
+    a = args()
+    a[1] = z(256, 4, dtype=f32).t()
+    with pytest.raises(ValueError, match="s_dy must be contiguous"):
+        fq.fp8_gemm_wgrad(*a)
+    a = args()
+    a[3] = z(3, 384, dtype=f32)
+    with pytest.raises(ValueError, match="s_x holds 1152"):
+        fq.fp8_gemm_wgrad(*a)
+    with pytest.raises(ValueError, match="Mp = 256 is not a positive multiple of 512"):
+        fq.fp8_gemm_wgrad(z(256, 256), z(2, 256, dtype=f32), z(384, 256), z(2, 384, dtype=f32))
+    with pytest.raises(ValueError, match="out holds"):
+        fq.fp8_gemm_wgrad(*args(), out=z(384, 256 + 1, dtype=bf16))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fq.fp8_gemm_wgrad(*args())

@@ -74,34 +74,52 @@ def test_act_128x1_covers_every_element_once(M, K, grid):
 
 
 def transpose_map(G, N, K, grid):
-    """transpose_w_128x128_kernel: block b -> (g, nb, kb); 1024 16-byte chunks
-    per block, 4 per thread; output element (g, k, n) written once."""
+    """transpose_w_128x128_kernel: block b -> (g, nb, kb); thread (l = t % 16,
+    j = t / 16) reads the 8x8 bytes at rows 8l.., columns 8j.. of the block
+    and writes them transposed at output rows 8j.., columns 8l..  Returns the
+    read and write counts and the output as tags of the source elements."""
     nkb, nnb = K // TILE, N // TILE
     blocks = G * nnb * nkb
-    out = np.zeros((G, K, N), dtype=np.int32)
+    out = np.full((G, K, N), -1, dtype=np.int64)
     src = np.zeros((G, N, K), dtype=np.int32)
+    writes = np.zeros((G, K, N), dtype=np.int32)
     st = np.zeros((G, nkb, nnb), dtype=np.int32)
+    tags = np.arange(G * N * K, dtype=np.int64).reshape(G, N, K)
     for bx in range(grid):
         b = bx
         while b < blocks:
             g, rem = b // (nnb * nkb), b % (nnb * nkb)
             nb, kb = rem // nkb, rem % nkb
             for t in range(256):
-                for i in range(4):
-                    c = t + 256 * i
-                    row, ch = c >> 3, c & 7
-                    src[g, nb * 128 + row, kb * 128 + ch * 16: kb * 128 + ch * 16 + 16] += 1
-                    orow = row  # the store loop uses the same chunk numbering on the output side
-                    out[g, kb * 128 + orow, nb * 128 + ch * 16: nb * 128 + ch * 16 + 16] += 1
+                l, j = t & 15, t >> 4
+                r0, c0 = nb * 128 + 8 * l, kb * 128 + 8 * j
+                src[g, r0:r0 + 8, c0:c0 + 8] += 1
+                block = tags[g, r0:r0 + 8, c0:c0 + 8]          # [r][c]
+                o0, oc = kb * 128 + 8 * j, nb * 128 + 8 * l
+                out[g, o0:o0 + 8, oc:oc + 8] = block.T       # lo[c], hi[c] after the register transpose
+                writes[g, o0:o0 + 8, oc:oc + 8] += 1
             st[g, kb, nb] += 1
             b += grid
-    return src, out, st
+    return src, writes, st, out, tags
 
 
 @pytest.mark.parametrize("G,N,K,grid", [(1, 128, 128, 1), (1, 256, 384, 2), (3, 128, 256, 5)])
 def test_transpose_reads_and_writes_every_element_once(G, N, K, grid):
-    src, out, st = transpose_map(G, N, K, grid)
-    assert np.all(src == 1) and np.all(out == 1) and np.all(st == 1)
+    src, writes, st, out, tags = transpose_map(G, N, K, grid)
+    assert np.all(src == 1) and np.all(writes == 1) and np.all(st == 1)
+    assert np.array_equal(out, np.swapaxes(tags, 1, 2))
+
+
+def test_transpose_warp_stores_are_full_rows():
+    """Per store instruction (fixed c) a warp's lanes write 8 bytes each at
+    output columns 8l of rows 8j + c: two rows, 128 contiguous bytes each."""
+    for w in range(8):
+        for c in range(8):
+            rows = {}
+            for t in range(32 * w, 32 * w + 32):
+                l, j = t & 15, t >> 4
+                rows.setdefault(8 * j + c, []).append(8 * l)
+            assert len(rows) == 2 and all(sorted(v) == list(range(0, 128, 8)) for v in rows.values())
 
 
 def test_launch_caps_leave_no_work_behind():
@@ -111,3 +129,103 @@ def test_launch_caps_leave_no_work_behind():
         grid = min(blocks, cap)
         covered = sum(len(range(bx, blocks, grid)) for bx in range(grid))
         assert covered == blocks
+
+
+# ---------------------------------------------------------------- token-contiguous codes
+def byte_perm(x, y, s):
+    """__byte_perm: result byte i is byte (s >> 4i) & 7 of the 8 bytes {x, y} (x low)."""
+    src = [(x >> (8 * i)) & 0xFF for i in range(4)] + [(y >> (8 * i)) & 0xFF for i in range(4)]
+    return sum(src[(s >> (4 * i)) & 7] << (8 * i) for i in range(4))
+
+
+def transpose4x4_bytes(w):
+    x0, x2 = byte_perm(w[0], w[2], 0x5410), byte_perm(w[0], w[2], 0x7632)
+    x1, x3 = byte_perm(w[1], w[3], 0x5410), byte_perm(w[1], w[3], 0x7632)
+    return [byte_perm(x0, x1, 0x6240), byte_perm(x0, x1, 0x7351), byte_perm(x2, x3, 0x6240),
+            byte_perm(x2, x3, 0x7351)]
+
+
+def transpose8x8_bytes(lo, hi):
+    lo, hi = list(lo), list(hi)
+    lo[0:4] = transpose4x4_bytes(lo[0:4])
+    lo[4:8] = transpose4x4_bytes(lo[4:8])
+    hi[0:4] = transpose4x4_bytes(hi[0:4])
+    hi[4:8] = transpose4x4_bytes(hi[4:8])
+    for i in range(4):
+        hi[i], lo[4 + i] = lo[4 + i], hi[i]
+    return lo, hi
+
+
+def test_byte_transpose_8x8():
+    rng = np.random.default_rng(0)
+    for _ in range(50):
+        m = rng.integers(0, 256, size=(8, 8), dtype=np.uint8)
+        words = m.view("<u4").reshape(8, 2)
+        lo, hi = transpose8x8_bytes([int(v) for v in words[:, 0]], [int(v) for v in words[:, 1]])
+        got = np.array([[lo[c], hi[c]] for c in range(8)], dtype="<u4").view(np.uint8).reshape(8, 8)
+        assert np.array_equal(got, m.T)
+
+
+def act_128x1_t_map(M, K, grid, Mp=None):
+    """quant_act_128x1_t_kernel: per 128x128 block, thread (cg = t % 16,
+    rg = t / 16) writes channel rows cg*8+c of the shared tile at physical
+    8-byte slot rg ^ cg; the store loop reads row c >> 3, 16-byte chunk
+    (c & 7) ^ (row >> 4), swapping halves when (row >> 3) is odd, and writes
+    qt[kc*128 + row, mb*128 + 16*(c & 7) ...].  Returns the transposed codes
+    of a matrix of distinct token/channel tags and the write counts."""
+    Mp = Mp or -(-M // 128) * 128
+    nkc = K // 128
+    blocks = (Mp // 128) * nkc
+    # tag of x[m, k] = (m, k) packed; the "code" of a token past M is 0
+    out = np.full((K, Mp), -1, dtype=np.int64)
+    writes = np.zeros((K, Mp), dtype=np.int32)
+    for bx in range(grid):
+        for b in range(bx, blocks, grid):
+            mb, kc = divmod(b, nkc)
+            tile = np.full((128, 16), -1, dtype=object)   # [channel row][physical 8-byte slot] -> 8 token tags
+            for t in range(256):
+                cg, rg = t & 15, t >> 4
+                for c in range(8):
+                    row = cg * 8 + c
+                    toks = []
+                    for r in range(8):
+                        m, k = mb * 128 + rg * 8 + r, kc * 128 + cg * 8 + c
+                        toks.append(m * K + k + 1 if m < M else 0)
+                    slot = rg ^ cg
+                    assert tile[row, slot] == -1
+                    tile[row, slot] = toks
+            for t in range(256):
+                for i in range(4):
+                    c = t + 256 * i
+                    row, ch = c >> 3, c & 7
+                    swz = row >> 3
+                    p = ch ^ (swz >> 1)
+                    halves = [tile[row, 2 * p], tile[row, 2 * p + 1]]
+                    if swz & 1:
+                        halves = halves[::-1]
+                    vals = halves[0] + halves[1]
+                    orow, ocol = kc * 128 + row, mb * 128 + ch * 16
+                    out[orow, ocol:ocol + 16] = vals
+                    writes[orow, ocol:ocol + 16] += 1
+    return out, writes
+
+
+@pytest.mark.parametrize("M,K,grid,Mp", [(128, 128, 1, 128), (200, 256, 3, 256), (300, 128, 2, 512),
+                                         (0, 128, 1, 512)])
+def test_act_128x1_t_writes_the_transpose(M, K, grid, Mp):
+    out, writes = act_128x1_t_map(M, K, grid, Mp)
+    assert np.all(writes == 1)
+    m = np.arange(Mp)[None, :]
+    k = np.arange(K)[:, None]
+    want = np.where(m < M, m * K + k + 1, 0)
+    assert np.array_equal(out, want)
+
+
+def test_act_128x1_t_shared_store_conflicts():
+    """Per warp store (fixed c), the 32 lanes' 8-byte slots cover every
+    8-byte bank slot of the 128-byte rows exactly twice: two wavefronts."""
+    for w in range(8):
+        for c in range(8):
+            slots = [(((t & 15) * 8 + c) * 128 + (((t >> 4) ^ (t & 15)) << 3)) % 128 // 8
+                     for t in range(32 * w, 32 * w + 32)]
+            assert sorted(slots) == sorted(list(range(16)) * 2)

@@ -40,6 +40,8 @@ calls = [
     ("fp8_grouped_gemm_contiguous", (A16, A16, A16, A16, A1, A16, 256, 256, 128, 4, None)),
     ("fp8_grouped_gemm_masked", (A16, A16, A16, A16, A16, A16, 4, 200, 256, 128, 0, None)),
     ("fp8_swiglu_quant_1x128", (A16, 4, 100, None, 0, A16, A16, None)),
+    ("fp8_quant_act_128x1_t", (A16, 4, 100, 128, A16, A16, None)),
+    ("fp8_gemm_wgrad", (A16, A16, A16, A16, A16, 256, 256, 0, None)),
 ]
 out = []
 lib = fq.lib()
@@ -69,7 +71,7 @@ def test_every_entry_point_pushes_and_pops_one_named_range(recorder):
     res = subprocess.run([sys.executable, "-c", CHILD, str(ROOT), str(recorder)], env=env,
                          capture_output=True, text=True, timeout=300, check=True)
     rows = json.loads(res.stdout.strip().splitlines()[-1])
-    assert len(rows) == 11
+    assert len(rows) == 13
     for r in rows:
         assert r["rc"] in (fq.OK, fq.ERR_SHAPE, fq.ERR_NULL, fq.ERR_ALIGN), r
         assert r["log"] == "push %s\npop\n" % r["name"], r

@@ -19,6 +19,9 @@ discuss; all seeds are numpy PCG64):
 * ``moe_masked``      32 experts x capacity 256, valid counts uniform on {0..256}; A [32,256,7168]
                       N(0,1), B1 [32,4096,7168]; second GEMM A2 [32,256,2048] N(0,1), B2
                       [32,7168,2048]; weights N(0,0.02^2); seed 4.
+* ``dense_wgrad``     the weight gradient of the dense_fprop layer, dW = dY^T X over 4096 tokens:
+                      X is dense_fprop's A (seed 1); dY [4096,7168] z[m,n]*exp(g[n]) (per-channel
+                      log-normal, sigma 1), seed 5.
 
 Every generator takes size overrides so the tests can draw the same
 distributions at sizes the oracle finishes in seconds.
@@ -112,6 +115,42 @@ def dense_fprop(seed: int = 1, M: int = 4096, N: int = 7168, K: int = 7168, outl
     del a
     b_bits = _normal_bf16(rng, (N, K), w_std)
     return Dense("dense_fprop", a_bits, b_bits, {"seed": seed, "outliers": n_out})
+
+
+@dataclass
+class Wgrad:
+    name: str
+    dy: np.ndarray  # [M,N] bf16 bits (tokens x output channels)
+    x: np.ndarray   # [M,K] bf16 bits (tokens x input channels)
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def M(self):
+        return self.x.shape[0]
+
+    @property
+    def N(self):
+        return self.dy.shape[1]
+
+    @property
+    def K(self):
+        return self.x.shape[1]
+
+    @property
+    def flops(self):
+        return 2.0 * self.M * self.N * self.K
+
+
+def dense_wgrad(seed: int = 5, M: int = 4096, N: int = 7168, K: int = 7168) -> Wgrad:
+    x = dense_fprop(M=M, N=128, K=K).a
+    rng = np.random.default_rng(seed)
+    chan = np.exp(rng.standard_normal(N, dtype=np.float32)).astype(np.float32)
+    dy = np.empty((M, N), dtype=np.uint16)
+    for r0 in range(0, M, 1024):
+        z = rng.standard_normal((min(M, r0 + 1024) - r0, N), dtype=np.float32)
+        z *= chan[None, :]
+        dy[r0:r0 + z.shape[0]] = bf16_bits(z)
+    return Wgrad("dense_wgrad", dy, x, {"seed": seed, "x_seed": 1})
 
 
 def long_k(seed: int = 2, M: int = 2048, N: int = 2048, K: int = 16384, shift: float = 0.5) -> Dense:
@@ -261,4 +300,5 @@ CONFIGS = {
     "long_k": long_k,
     "moe_contiguous": moe_contiguous,
     "moe_masked": moe_masked,
+    "dense_wgrad": dense_wgrad,
 }
