@@ -149,16 +149,26 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- workloads
-def make_workload(name: str):
+def make_workload(name: str, shard: int = 0, device=None):
+    """The named workload; ``shard`` r > 0 is rank r's part of the batch
+    (row blocks for the dense shapes, experts for the MoE ones; see
+    workloads.row_shard / expert_shard).  ``device`` draws the large MoE
+    tensors on that device instead of the host."""
     import workloads as wl
-    if name == "dense_dgrad":
-        # the activation-gradient GEMM of the dense_fprop layer: dY takes the
-        # shape and distribution of the forward activations, W is the weight
-        return wl.dense_fprop()
-    if name == "moe_masked_chain":
-        # the masked decode as one chain: GEMM2's activation is the SwiGLU of
-        # GEMM1's output, requantized (its own A2 draw is not used)
-        return wl.moe_masked()
+    if name in ("dense_fprop", "dense_dgrad"):
+        # dense_dgrad: the activation-gradient GEMM of the dense_fprop layer;
+        # dY takes the shape and distribution of the forward activations
+        return wl.dense_fprop(shard=shard)
+    if name == "long_k":
+        return wl.long_k(shard=shard)
+    if name == "dense_wgrad":
+        return wl.dense_wgrad(seed=5 + 100 * shard) if shard else wl.dense_wgrad()
+    if name in ("moe_masked", "moe_masked_chain"):
+        # moe_masked_chain: GEMM2's activation is the SwiGLU of GEMM1's output,
+        # requantized (its own A2 draw is not used)
+        return wl.moe_masked(shard=shard, device=device)
+    if name == "moe_contiguous":
+        return wl.moe_contiguous(shard=shard, device=device)
     return wl.CONFIGS[name]()
 
 
@@ -183,7 +193,15 @@ def describe(name: str, d) -> dict:
 
 
 def _to_dev_bf16(torch, bits, dev):
+    """bf16 bit patterns (numpy) or a bf16 tensor already drawn on the device
+    (a copy, so rotating input sets are distinct buffers)."""
+    if isinstance(bits, torch.Tensor):
+        return bits.to(dev).clone()
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def _to_dev_i32(torch, arr, dev):
+    return torch.from_numpy(np.ascontiguousarray(arr, dtype=np.int32)).to(dev)
 
 
 def build_sets(name, d, dev, nsets, torch, fq):
@@ -198,7 +216,7 @@ def build_sets(name, d, dev, nsets, torch, fq):
             if name == "moe_masked":
                 s["a2"] = _to_dev_bf16(torch, d.a2.reshape(E * cap, -1), dev)
             s["b2"] = _to_dev_bf16(torch, d.b2, dev)
-            s["mm"] = torch.from_numpy(d.masked_m).to(dev)
+            s["mm"] = _to_dev_i32(torch, d.masked_m, dev)
         elif name == "dense_wgrad":
             s["dy"] = _to_dev_bf16(torch, d.dy, dev)
             s["x"] = _to_dev_bf16(torch, d.x, dev)
@@ -206,7 +224,7 @@ def build_sets(name, d, dev, nsets, torch, fq):
             s["a"] = _to_dev_bf16(torch, d.a, dev)
             s["b"] = _to_dev_bf16(torch, d.b, dev)
             if name == "moe_contiguous":
-                s["mi"] = torch.from_numpy(d.m_indices).to(dev)
+                s["mi"] = _to_dev_i32(torch, d.m_indices, dev)
         sets.append(s)
     return sets
 
@@ -470,6 +488,109 @@ def gemm_roofline(plan, kernels, peaks, fp8_peak, bf16_peak, sustained, name):
     return roofline
 
 
+def enqueue_ahead(torch, ms: float = 20.0):
+    """A short device-side delay before the timed region, so the host has the
+    first steps' launches queued when the device reaches them: the events
+    then time the kernels, not the host's launch latency.  The delay itself
+    lies before the start event."""
+    torch.cuda._sleep(int(ms * 1e6))  # ~1 cycle per ns at the SM clock: a delay of a few ms to tens of ms
+
+
+def measure(name, d, dev, steps, warmup, world, torch, fq):
+    """Times `steps` steps of the workload (after `warmup` untimed ones) on
+    rotating input sets: the step's elapsed device time (max over ranks),
+    every kernel's per-launch times, the clock record and the launch count."""
+    plan = kernel_plan(name, d)
+    nk = len(plan)
+    per_set_bytes = sum(b for _, b, _ in plan)
+    nsets = max(2, int(np.ceil(2 * 126e6 / max(per_set_bytes, 1))))
+    nsets = min(nsets, 4)
+    sets = build_sets(name, d, dev, nsets, torch, fq)
+    stream = torch.cuda.current_stream(dev)
+
+    for i in range(warmup):
+        launch_step(name, d, sets[i % nsets], fq)
+    torch.cuda.synchronize(dev)
+    if fq.get_device_error(device=dev) != fq.OK:
+        raise RuntimeError("device error during warm-up of %s" % name)
+
+    events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(nk)]
+              for _ in range(steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    launches0 = fq.launch_count()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        enqueue_ahead(torch)
+        t_start.record(stream)
+        for i in range(steps):
+            launch_step(name, d, sets[i % nsets], fq, events[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    launches = fq.launch_count() - launches0
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
+    if fq.get_device_error(device=dev) != fq.OK:
+        raise RuntimeError("device error in the timed region of %s" % name)
+    kernel_ms = [[events[i][k][0].elapsed_time(events[i][k][1]) for i in range(steps)] for k in range(nk)]
+    # per kernel: the max over ranks of its mean launch time
+    kernel_ms = [[max_over_ranks(float(np.mean(ms)), world, dev)] for ms in kernel_ms]
+    del sets
+    return {"plan": plan, "elapsed_ms": elapsed_ms, "kernel_ms": kernel_ms, "clocks": clk.summary(),
+            "launches": int(launches), "nsets": nsets, "per_set_bytes": per_set_bytes}
+
+
+def kernel_table(m, peaks, fp8_peak):
+    kernels = {}
+    for k, (label, nbytes, kflops) in enumerate(m["plan"]):
+        avg_ms = float(np.mean(m["kernel_ms"][k]))
+        ent = {"avg_ms": avg_ms, "bytes": nbytes}
+        if kflops:
+            ent.update(tflops=kflops / avg_ms / 1e9, frac_of_fp8_peak=kflops / avg_ms / 1e9 / fp8_peak)
+        ent.update(gbs=nbytes / avg_ms / 1e6, frac_of_hbm=nbytes / avg_ms / 1e6 / peaks["hbm_gbs"])
+        kernels[label] = ent
+    return kernels
+
+
+def peaks_for(elapsed_ms):
+    """Peaks for a timed region: the burst bf16 figure for a short region,
+    the sustained one for a region of a second or more."""
+    peaks = load_peaks()
+    sustained = elapsed_ms / 1e3 >= SUSTAINED_AFTER_S
+    bf16_peak = peaks["bf16_sustained"] if sustained else peaks["bf16"]
+    return peaks, bf16_peak * FP8_OVER_BF16, bf16_peak, sustained
+
+
+# Secondary workloads the default run times after the headline (their own
+# per-kernel tables, rooflines and clocks under one key of the same line).
+SECONDARY = ("long_k", "moe_contiguous", "moe_masked")
+SECONDARY_STEPS, SECONDARY_WARMUP = 10, 3
+
+
+def secondary_lines(args, dev, world, rank, torch, fq):
+    out = {}
+    for name in SECONDARY:
+        d = make_workload(name, shard=rank, device=dev if name.startswith("moe") else None)
+        m = measure(name, d, dev, SECONDARY_STEPS, SECONDARY_WARMUP, world, torch, fq)
+        peaks, fp8_peak, bf16_peak, sustained = peaks_for(m["elapsed_ms"])
+        kernels = kernel_table(m, peaks, fp8_peak)
+        flops = step_flops(name, d)
+        draws = d.meta.get("draws", "host")
+        out[name] = {
+            "value": world * flops * SECONDARY_STEPS / (m["elapsed_ms"] / 1e3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": m["elapsed_ms"] / SECONDARY_STEPS, "steps": SECONDARY_STEPS, "warmup": SECONDARY_WARMUP,
+            "config": dict(describe(name, d), draws=draws,
+                           l2="inputs rotated over %d buffer sets (%.0f MB each) between steps" % (
+                               m["nsets"], m["per_set_bytes"] / 1e6)),
+            "roofline": gemm_roofline(m["plan"], kernels, peaks, fp8_peak, bf16_peak, sustained, name),
+            "kernels": kernels, "gpu_launches": m["launches"], "clocks": m["clocks"],
+        }
+        del d
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, name):
     import torch
     rank, world, local = dist_env()
@@ -483,45 +604,18 @@ def run_ours(args, name):
     import fp8_fine_grained_quant_b200 as fq
     fq.lib()
 
-    d = make_workload(name)
-    plan = kernel_plan(name, d)
-    nk = len(plan)
+    # rank r runs its shard of a batch `world` times the single-GPU one: row
+    # blocks (dense; B replicated) or experts (MoE); no collective touches
+    # the data, only the barrier and the max-over-ranks of the timings
+    d = make_workload(name, shard=rank)
+    m = measure(name, d, dev, args.steps, args.warmup, world, torch, fq)
     flops = step_flops(name, d)
-    per_set_bytes = sum(b for _, b, _ in plan)
-    nsets = max(2, int(np.ceil(2 * 126e6 / max(per_set_bytes, 1))))
-    nsets = min(nsets, 4)
-    sets = build_sets(name, d, dev, nsets, torch, fq)
-    stream = torch.cuda.current_stream(dev)
-
-    for i in range(args.warmup):
-        launch_step(name, d, sets[i % nsets], fq)
-    torch.cuda.synchronize(dev)
-    if fq.get_device_error(device=dev) != fq.OK:
-        raise RuntimeError("device error during warm-up")
-
-    events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(nk)]
-              for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    launches0 = fq.launch_count()
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index) as clk:
-        t_start.record(stream)
-        for i in range(args.steps):
-            launch_step(name, d, sets[i % nsets], fq, events[i])
-        t_end.record(stream)
-        torch.cuda.synchronize(dev)
-    barrier(world)
-    launches = fq.launch_count() - launches0
-    elapsed_ms = t_start.elapsed_time(t_end)
-    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
-    if fq.get_device_error(device=dev) != fq.OK:
-        raise RuntimeError("device error in the timed region")
-    kernel_ms = [[events[i][k][0].elapsed_time(events[i][k][1]) for i in range(args.steps)] for k in range(nk)]
 
     # ------------------------------------------------------------ e2e (host buffers)
     e2e = run_e2e(args, name, d, dev, torch, fq, world)
+    extra = None
+    if name == "dense_fprop" and not args.no_secondary:
+        extra = secondary_lines(args, dev, world, rank, torch, fq)
 
     if rank != 0:
         if world > 1:
@@ -529,35 +623,28 @@ def run_ours(args, name):
             dist.destroy_process_group()
         return 0
 
-    peaks = load_peaks()
-    timed_s = elapsed_ms / 1e3
-    sustained = timed_s >= SUSTAINED_AFTER_S
-    bf16_peak = peaks["bf16_sustained"] if sustained else peaks["bf16"]
-    fp8_peak = bf16_peak * FP8_OVER_BF16
-    kernels = {}
-    for k, (label, nbytes, kflops) in enumerate(plan):
-        avg_ms = float(np.mean(kernel_ms[k]))
-        ent = {"avg_ms": avg_ms, "bytes": nbytes}
-        if kflops:
-            ent.update(tflops=kflops / avg_ms / 1e9, frac_of_fp8_peak=kflops / avg_ms / 1e9 / fp8_peak)
-        ent.update(gbs=nbytes / avg_ms / 1e6, frac_of_hbm=nbytes / avg_ms / 1e6 / peaks["hbm_gbs"])
-        kernels[label] = ent
-    roofline = gemm_roofline(plan, kernels, peaks, fp8_peak, bf16_peak, sustained, name)
-    value = world * flops * args.steps / (elapsed_ms / 1e3) / 1e12
+    peaks, fp8_peak, bf16_peak, sustained = peaks_for(m["elapsed_ms"])
+    kernels = kernel_table(m, peaks, fp8_peak)
+    roofline = gemm_roofline(m["plan"], kernels, peaks, fp8_peak, bf16_peak, sustained, name)
+    value = world * flops * args.steps / (m["elapsed_ms"] / 1e3) / 1e12
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(name, d)
     line = {
         "metric": METRIC,
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3", "data": "synthetic",
-        "config": dict(describe(name, d), parallelism="replicas" if world > 1 else "single",
+        "ms_per_step": m["elapsed_ms"] / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": dict(describe(name, d),
+                       parallelism=("dp%d: %s shard per rank, no data-path collective" % (
+                           world, "expert" if name.startswith("moe") else "M-row")) if world > 1 else "single",
                        l2="inputs rotated over %d buffer sets (%.0f MB each) between steps" % (
-                           nsets, per_set_bytes / 1e6)),
+                           m["nsets"], m["per_set_bytes"] / 1e6)),
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": int(launches), "clocks": clk.summary(),
+        "gpu_launches": m["launches"], "clocks": m["clocks"],
     }
+    if extra is not None:
+        line["secondary_workloads"] = extra
     print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist
@@ -624,19 +711,39 @@ def cpu_baseline(name, d):
             "sample": "3 oracle steps, each: %s; %.1f s total" % (sample_description(name, d, rows, nb), sum(dts))}
 
 
+def relaunch_under_torchrun(args_list, n: int) -> int:
+    """`bench.py --gpus N` outside a launcher: start N ranks on this node
+    with torch.distributed.run (rendezvous on 127.0.0.1) and return its
+    status; rank 0 prints the line."""
+    import socket
+    import subprocess
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(n),
+           "--master-addr", "127.0.0.1", "--master-port", str(port), str(Path(__file__).resolve())] + list(args_list)
+    return subprocess.call(cmd)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dense_fprop",
                     choices=["tiny_dense", "dense_fprop", "long_k", "moe_contiguous", "moe_masked", "dense_dgrad",
                              "moe_masked_chain", "dense_wgrad"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args(argv)
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="time the named workload only (the default dense_fprop run also times long_k, "
+                         "moe_contiguous and moe_masked)")
+    raw = sys.argv[1:] if argv is None else list(argv)
+    args = ap.parse_args(raw)
     if args.warmup < 3:
         args.warmup = 3
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch_under_torchrun(raw, args.gpus)
     if args.impl == "reference":
         return run_reference(args, args.workload)
     return run_ours(args, args.workload)

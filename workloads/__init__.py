@@ -41,8 +41,9 @@ def bf16_bits(x: np.ndarray) -> np.ndarray:
     Input preparation only: the generators draw in float32 and store bf16.
     Non-finite values are not produced by any generator here."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    u = x.view(np.uint32)
+    # finite inputs: the largest pattern, 0xFF7FFFFF, plus 0x8000 stays below 2^32
+    rounded = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return rounded.astype(np.uint16)
 
 
@@ -101,7 +102,23 @@ def tiny_dense(seed: int = 0, M: int = 128, N: int = 256, K: int = 512, outlier_
 
 
 def dense_fprop(seed: int = 1, M: int = 4096, N: int = 7168, K: int = 7168, outlier_frac: float = 1e-4,
-                outlier_value: float = 200.0, w_std: float = 0.02) -> Dense:
+                outlier_value: float = 200.0, w_std: float = 0.02, shard: int = 0) -> Dense:
+    """``shard`` r > 0 draws the r-th M-row block of a larger token batch: the
+    same layer (per-channel magnitudes and weight B, both from ``seed``), its
+    own tokens (seeded by (seed, r)).  Shard 0 is the single-GPU workload."""
+    if shard:
+        base = dense_fprop(seed, M=TILE, N=N, K=K, outlier_frac=0.0, w_std=w_std)
+        b_bits = dense_fprop(seed, M=M, N=N, K=K, outlier_frac=outlier_frac, outlier_value=outlier_value,
+                             w_std=w_std).b
+        rng = np.random.default_rng([seed, shard])
+        chan = base.meta["chan"]
+        a = rng.standard_normal((M, K), dtype=np.float32)
+        a *= chan[None, :]
+        n_out = int(round(outlier_frac * M * K))
+        idx = rng.choice(M * K, size=n_out, replace=False)
+        signs = np.where(rng.random(n_out) < 0.5, -1.0, 1.0).astype(np.float32)
+        a.reshape(-1)[idx] = np.float32(outlier_value) * signs
+        return Dense("dense_fprop", bf16_bits(a), b_bits, {"seed": seed, "shard": shard, "outliers": n_out})
     rng = np.random.default_rng(seed)
     g = rng.standard_normal(K, dtype=np.float32)
     chan = np.exp(g).astype(np.float32)  # per-channel log-normal magnitude, sigma = 1
@@ -114,7 +131,7 @@ def dense_fprop(seed: int = 1, M: int = 4096, N: int = 7168, K: int = 7168, outl
     a_bits = bf16_bits(a)
     del a
     b_bits = _normal_bf16(rng, (N, K), w_std)
-    return Dense("dense_fprop", a_bits, b_bits, {"seed": seed, "outliers": n_out})
+    return Dense("dense_fprop", a_bits, b_bits, {"seed": seed, "outliers": n_out, "chan": chan})
 
 
 @dataclass
@@ -153,11 +170,14 @@ def dense_wgrad(seed: int = 5, M: int = 4096, N: int = 7168, K: int = 7168) -> W
     return Wgrad("dense_wgrad", dy, x, {"seed": seed, "x_seed": 1})
 
 
-def long_k(seed: int = 2, M: int = 2048, N: int = 2048, K: int = 16384, shift: float = 0.5) -> Dense:
+def long_k(seed: int = 2, M: int = 2048, N: int = 2048, K: int = 16384, shift: float = 0.5, shard: int = 0) -> Dense:
+    """``shard`` r > 0: the r-th M-row block of a larger batch (same B, own rows)."""
     rng = np.random.default_rng(seed)
     a = rng.uniform(-1.0, 1.0, size=(M, K)).astype(np.float32) + np.float32(shift)
     b = rng.uniform(-1.0, 1.0, size=(N, K)).astype(np.float32) + np.float32(shift)
-    return Dense("long_k", bf16_bits(a), bf16_bits(b), {"seed": seed})
+    if shard:
+        a = np.random.default_rng([seed, shard]).uniform(-1.0, 1.0, size=(M, K)).astype(np.float32) + np.float32(shift)
+    return Dense("long_k", bf16_bits(a), bf16_bits(b), {"seed": seed, "shard": shard})
 
 
 @dataclass
@@ -207,23 +227,56 @@ def zipf_topk_counts(rng: np.random.Generator, tokens: int, E: int, topk: int, a
     return np.bincount(chosen.reshape(-1), minlength=E).astype(np.int64)
 
 
+def device_normal_bf16(shape, std: float, seed: int, device):
+    """N(0, std^2) as a bf16 tensor drawn on a CUDA device with torch's seeded
+    Philox generator (float32 draws, rounded to bf16 to nearest even).  The
+    same distribution as the host draws, other values: for timing runs of the
+    large MoE weights, where the host generator would take a minute."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    z = torch.randn(tuple(int(v) for v in shape), generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        z.mul_(std)
+    return z.to(torch.bfloat16)
+
+
 def moe_contiguous(seed: int = 3, tokens: int = 4096, topk: int = 8, E: int = 32, N: int = 4096, K: int = 7168,
-                   alpha: float = 1.1, w_std: float = 0.02) -> Contiguous:
-    rng = np.random.default_rng(seed)
+                   alpha: float = 1.1, w_std: float = 0.02, device=None, shard: int = 0) -> Contiguous:
+    """With ``device`` given, ``a`` and ``b`` are bf16 tensors drawn on that
+    device (device_normal_bf16, seeds derived from ``seed``); the routing
+    (counts, m_indices) is the host draw either way.  ``shard`` r > 0 draws
+    the r-th rank's experts of an expert-parallel layer E times the ranks
+    wide: its own tokens' rows and its own expert weights, seeded by
+    (seed, r)."""
+    rng = np.random.default_rng([seed, shard] if shard else seed)
+    dseed = seed * 1000 + 100000 * shard
     counts = zipf_topk_counts(rng, tokens, E, topk, alpha)
     padded = (counts + TILE - 1) // TILE * TILE
     M_tot = int(padded.sum())
-    a = np.zeros((M_tot, K), dtype=np.uint16)
     m_indices = np.empty(M_tot // TILE, dtype=np.int32)
+    if device is not None:
+        import torch
+        a = torch.zeros((M_tot, K), dtype=torch.bfloat16, device=device)
+    else:
+        a = np.zeros((M_tot, K), dtype=np.uint16)
     r = 0
     for e in range(E):
         c, p = int(counts[e]), int(padded[e])
         if c:
-            a[r:r + c] = _normal_bf16(rng, (c, K))
+            if device is not None:
+                a[r:r + c] = device_normal_bf16((c, K), 1.0, dseed + e, device)
+            else:
+                a[r:r + c] = _normal_bf16(rng, (c, K))
         m_indices[r // TILE:(r + p) // TILE] = e
         r += p
-    b = _normal_bf16(rng, (E, N, K), w_std)
-    return Contiguous("moe_contiguous", a, b, m_indices, counts, {"seed": seed, "tokens": tokens, "topk": topk})
+    if device is not None:
+        b = device_normal_bf16((E, N, K), w_std, dseed + 999, device)
+    else:
+        b = _normal_bf16(rng, (E, N, K), w_std)
+    return Contiguous("moe_contiguous", a, b, m_indices, counts,
+                      {"seed": seed, "shard": shard, "tokens": tokens, "topk": topk,
+                       "draws": "device" if device is not None else "host"})
 
 
 @dataclass
@@ -250,16 +303,27 @@ class Masked:
 
 
 def moe_masked(seed: int = 4, E: int = 32, cap: int = 256, N: int = 4096, K: int = 7168, N2: int = 7168,
-               K2: int = 2048, w_std: float = 0.02, second: bool = True) -> Masked:
-    rng = np.random.default_rng(seed)
+               K2: int = 2048, w_std: float = 0.02, second: bool = True, device=None, shard: int = 0) -> Masked:
+    """With ``device`` given, the activations and weights are bf16 tensors
+    drawn on that device (device_normal_bf16); masked_m is the host draw
+    either way.  ``shard`` r > 0: the r-th rank's experts of an
+    expert-parallel layer, seeded by (seed, r)."""
+    rng = np.random.default_rng([seed, shard] if shard else seed)
     masked_m = rng.integers(0, cap, size=E, endpoint=True).astype(np.int32)
-    a = _normal_bf16(rng, (E, cap, K))
-    b = _normal_bf16(rng, (E, N, K), w_std)
+    if device is not None:
+        def draw(shape, std, k):
+            return device_normal_bf16(shape, std, seed * 1000 + 100000 * shard + k, device)
+    else:
+        def draw(shape, std, k):
+            return _normal_bf16(rng, shape, std)
+    a = draw((E, cap, K), 1.0, 0)
+    b = draw((E, N, K), w_std, 1)
     a2 = b2 = None
     if second:
-        a2 = _normal_bf16(rng, (E, cap, K2))
-        b2 = _normal_bf16(rng, (E, N2, K2), w_std)
-    return Masked("moe_masked", a, b, masked_m, a2, b2, {"seed": seed})
+        a2 = draw((E, cap, K2), 1.0, 2)
+        b2 = draw((E, N2, K2), w_std, 3)
+    return Masked("moe_masked", a, b, masked_m, a2, b2,
+                  {"seed": seed, "shard": shard, "draws": "device" if device is not None else "host"})
 
 
 def parity_rows(rng: np.random.Generator, M: int, per_tile: int = 2, tile: int = TILE) -> np.ndarray:
@@ -275,6 +339,30 @@ def parity_rows(rng: np.random.Generator, M: int, per_tile: int = 2, tile: int =
                                                      replace=False))
         rows.extend(sorted(pick))
     return np.asarray(rows, dtype=np.int64)
+
+
+def row_shard(M: int, world: int, rank: int, tile: int = TILE) -> tuple[int, int]:
+    """Rows [start, stop) of an M-row batch owned by ``rank`` of ``world``:
+    contiguous runs of whole 128-row tiles, as even as the tile count allows
+    (the first M_tiles % world ranks take one tile more); the last rank's run
+    ends at M, ragged tail included.  Every row belongs to exactly one rank."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank %d of world %d" % (rank, world))
+    tiles = -(-M // tile)
+    base, extra = divmod(tiles, world)
+    t0 = rank * base + min(rank, extra)
+    t1 = t0 + base + (1 if rank < extra else 0)
+    return min(M, t0 * tile), min(M, t1 * tile)
+
+
+def expert_shard(E: int, world: int, rank: int) -> tuple[int, int]:
+    """Experts [e0, e1) owned by ``rank`` (expert parallelism): contiguous,
+    as even as E allows; every expert belongs to exactly one rank."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank %d of world %d" % (rank, world))
+    base, extra = divmod(E, world)
+    e0 = rank * base + min(rank, extra)
+    return e0, e0 + base + (1 if rank < extra else 0)
 
 
 def quad_rows(rng: np.random.Generator, M: int, tile: int = TILE, quad: int = 32) -> np.ndarray:
