@@ -229,6 +229,12 @@ def build_sets(name, d, dev, nsets, torch, fq):
     return sets
 
 
+# How a step quantizes a GEMM's two operands: "fused" = one launch of
+# fp8_quant_act_w for both, "separate" = fp8_quant_act_1x128 then
+# fp8_quant_w_128x128.  Set from --quant.
+QUANT_MODE = "fused"
+
+
 def kernel_plan(name, d):
     """(kernel label, algorithmic bytes, algorithmic FLOPs) per launch of one step."""
     def qa_bytes(rows, K):
@@ -240,16 +246,20 @@ def kernel_plan(name, d):
     def gemm_bytes(rows, N, K, G=1):
         return rows * K + rows * (K // TILE) * 4 + G * N * K + G * (N // TILE) * (K // TILE) * 4 + rows * N * 2
 
+    def quant(a_bytes, w_bytes, suffix=""):
+        if QUANT_MODE == "fused":
+            return [("quant_act_w" + suffix, a_bytes + w_bytes, 0.0)]
+        return [("quant_act_1x128" + suffix, a_bytes, 0.0), ("quant_w_128x128" + suffix, w_bytes, 0.0)]
+
     if name in ("tiny_dense", "dense_fprop", "long_k"):
         M, N, K = d.M, d.N, d.K
-        return [("quant_act_1x128", qa_bytes(M, K), 0.0), ("quant_w_128x128", qw_bytes(1, N, K), 0.0),
-                ("gemm_blockscaled", gemm_bytes(M, N, K), 2.0 * M * N * K)]
+        return quant(qa_bytes(M, K), qw_bytes(1, N, K)) + [("gemm_blockscaled", gemm_bytes(M, N, K), 2.0 * M * N * K)]
     if name == "dense_dgrad":
         # dY is d.a [M, Nout], W is d.b [Nout, K]; dX = dY W is [M, K]
         M, Nout, K = d.M, d.N, d.K
-        return [("quant_act_1x128", qa_bytes(M, Nout), 0.0), ("quant_w_128x128", qw_bytes(1, Nout, K), 0.0),
-                ("transpose_w_128x128", 2 * Nout * K + 2 * 4 * (Nout // TILE) * (K // TILE), 0.0),
-                ("gemm_dgrad", gemm_bytes(M, K, Nout), 2.0 * M * Nout * K)]
+        return quant(qa_bytes(M, Nout), qw_bytes(1, Nout, K)) + [
+            ("transpose_w_128x128", 2 * Nout * K + 2 * 4 * (Nout // TILE) * (K // TILE), 0.0),
+            ("gemm_dgrad", gemm_bytes(M, K, Nout), 2.0 * M * Nout * K)]
     if name == "dense_wgrad":
         # both operands quantized along tokens, codes written token-contiguous
         M, N, K = d.M, d.N, d.K
@@ -262,8 +272,8 @@ def kernel_plan(name, d):
         return [("quant_act_128x1_t", qt_bytes(N), 0.0), ("quant_act_128x1_t#2", qt_bytes(K), 0.0),
                 ("gemm_wgrad", gemm, 2.0 * M * N * K)]
     if name == "moe_contiguous":
-        return [("quant_act_1x128", qa_bytes(d.M_tot, d.K), 0.0), ("quant_w_128x128", qw_bytes(d.E, d.N, d.K), 0.0),
-                ("grouped_gemm_contiguous", gemm_bytes(d.M_tot, d.N, d.K, d.E), d.flops)]
+        return quant(qa_bytes(d.M_tot, d.K), qw_bytes(d.E, d.N, d.K)) + [
+            ("grouped_gemm_contiguous", gemm_bytes(d.M_tot, d.N, d.K, d.E), d.flops)]
     E, cap, K = d.a.shape
     N, K2, N2 = d.b.shape[1], d.a2.shape[2], d.b2.shape[1]
     active = int((d.masked_m > 0).sum())
@@ -271,76 +281,89 @@ def kernel_plan(name, d):
     if name == "moe_masked_chain":
         # GEMM1's valid rows in (gate | up, bf16), h's codes and scales out
         swiglu = valid * N * 2 + valid * K2 + valid * (K2 // TILE) * 4
-        return [("quant_act_1x128", qa_bytes(E * cap, K), 0.0), ("quant_w_128x128", qw_bytes(E, N, K), 0.0),
-                ("grouped_gemm_masked", gemm_bytes(valid, N, K, active), d.flops(False)),
-                ("swiglu_quant_1x128", swiglu, 0.0), ("quant_w_128x128#2", qw_bytes(E, N2, K2), 0.0),
-                ("grouped_gemm_masked#2", gemm_bytes(valid, N2, K2, active), d.flops(True))]
-    return [("quant_act_1x128", qa_bytes(E * cap, K), 0.0), ("quant_w_128x128", qw_bytes(E, N, K), 0.0),
+        return quant(qa_bytes(E * cap, K), qw_bytes(E, N, K)) + [
             ("grouped_gemm_masked", gemm_bytes(valid, N, K, active), d.flops(False)),
-            ("quant_act_1x128#2", qa_bytes(E * cap, K2), 0.0), ("quant_w_128x128#2", qw_bytes(E, N2, K2), 0.0),
+            ("swiglu_quant_1x128", swiglu, 0.0), ("quant_w_128x128#2", qw_bytes(E, N2, K2), 0.0),
             ("grouped_gemm_masked#2", gemm_bytes(valid, N2, K2, active), d.flops(True))]
+    return (quant(qa_bytes(E * cap, K), qw_bytes(E, N, K)) +
+            [("grouped_gemm_masked", gemm_bytes(valid, N, K, active), d.flops(False))] +
+            quant(qa_bytes(E * cap, K2), qw_bytes(E, N2, K2), "#2") +
+            [("grouped_gemm_masked#2", gemm_bytes(valid, N2, K2, active), d.flops(True))])
 
 
 def launch_step(name, d, s, fq, events=None):
     """Launch the kernels of one step on the current stream.  `events`, if
-    given, is a list of (start, end) CUDA-event pairs, one per kernel."""
-    def rec(i, which):
+    given, is a list of (start, end) CUDA-event pairs, one per kernel, in
+    kernel_plan's order."""
+    k = [0]
+
+    def rec(which):
         if events is not None:
-            events[i][which].record()
+            events[k[0]][which].record()
+        if which:
+            k[0] += 1
+
+    def quant(a, b, qa, sa, qb, sb):
+        """Both operands of a GEMM; returns (qa, sa, qb, sb)."""
+        if QUANT_MODE == "fused":
+            rec(0)
+            (q1, s1), (q2, s2) = fq.fp8_quant_act_w(s[a], s[b], s.get(qa), s.get(sa), s.get(qb), s.get(sb))
+            rec(1)
+        else:
+            rec(0); q1, s1 = fq.fp8_quant_act_1x128(s[a], s.get(qa), s.get(sa)); rec(1)
+            rec(0); q2, s2 = fq.fp8_quant_w_128x128(s[b], s.get(qb), s.get(sb)); rec(1)
+        s.update({qa: q1, sa: s1, qb: q2, sb: s2})
+        return q1, s1, q2, s2
 
     if name == "moe_masked_chain":
         E, cap, K = d.a.shape
-        rec(0, 0); qa, sa = fq.fp8_quant_act_1x128(s["a"], s.get("qa"), s.get("sa")); rec(0, 1)
-        rec(1, 0); qb, sb = fq.fp8_quant_w_128x128(s["b"], s.get("qb"), s.get("sb")); rec(1, 1)
-        rec(2, 0)
+        qa, sa, qb, sb = quant("a", "b", "qa", "sa", "qb", "sb")
+        rec(0)
         c = fq.fp8_grouped_gemm_masked(qa.view(E, cap, K), sa.view(E, cap, K // TILE), qb, sb, s["mm"],
                                        expected_m=int(d.masked_m.mean()), out=s.get("c"))
-        rec(2, 1)
-        rec(3, 0); qh, sh = fq.fp8_swiglu_quant_1x128(c, s["mm"], s.get("qh"), s.get("sh")); rec(3, 1)
-        rec(4, 0); qb2, sb2 = fq.fp8_quant_w_128x128(s["b2"], s.get("qb2"), s.get("sb2")); rec(4, 1)
-        rec(5, 0)
+        rec(1)
+        rec(0); qh, sh = fq.fp8_swiglu_quant_1x128(c, s["mm"], s.get("qh"), s.get("sh")); rec(1)
+        rec(0); qb2, sb2 = fq.fp8_quant_w_128x128(s["b2"], s.get("qb2"), s.get("sb2")); rec(1)
+        rec(0)
         c2 = fq.fp8_grouped_gemm_masked(qh, sh, qb2, sb2, s["mm"], expected_m=int(d.masked_m.mean()),
                                         out=s.get("c2"))
-        rec(5, 1)
-        s.update(qa=qa, sa=sa, qb=qb, sb=sb, c=c, qh=qh, sh=sh, qb2=qb2, sb2=sb2, c2=c2)
+        rec(1)
+        s.update(c=c, qh=qh, sh=sh, qb2=qb2, sb2=sb2, c2=c2)
         return c2
     if name == "moe_masked":
         E, cap, K = d.a.shape
-        rec(0, 0); qa, sa = fq.fp8_quant_act_1x128(s["a"], s.get("qa"), s.get("sa")); rec(0, 1)
-        rec(1, 0); qb, sb = fq.fp8_quant_w_128x128(s["b"], s.get("qb"), s.get("sb")); rec(1, 1)
-        rec(2, 0)
+        qa, sa, qb, sb = quant("a", "b", "qa", "sa", "qb", "sb")
+        rec(0)
         c = fq.fp8_grouped_gemm_masked(qa.view(E, cap, K), sa.view(E, cap, K // TILE), qb, sb, s["mm"],
                                        expected_m=int(d.masked_m.mean()), out=s.get("c"))
-        rec(2, 1)
+        rec(1)
         K2 = d.a2.shape[2]
-        rec(3, 0); qa2, sa2 = fq.fp8_quant_act_1x128(s["a2"], s.get("qa2"), s.get("sa2")); rec(3, 1)
-        rec(4, 0); qb2, sb2 = fq.fp8_quant_w_128x128(s["b2"], s.get("qb2"), s.get("sb2")); rec(4, 1)
-        rec(5, 0)
+        qa2, sa2, qb2, sb2 = quant("a2", "b2", "qa2", "sa2", "qb2", "sb2")
+        rec(0)
         c2 = fq.fp8_grouped_gemm_masked(qa2.view(E, cap, K2), sa2.view(E, cap, K2 // TILE), qb2, sb2, s["mm"],
                                         expected_m=int(d.masked_m.mean()), out=s.get("c2"))
-        rec(5, 1)
-        s.update(qa=qa, sa=sa, qb=qb, sb=sb, c=c, qa2=qa2, sa2=sa2, qb2=qb2, sb2=sb2, c2=c2)
+        rec(1)
+        s.update(c=c, c2=c2)
         return c2
     if name == "dense_wgrad":
-        rec(0, 0); q_dy, s_dy = fq.fp8_quant_act_128x1_t(s["dy"], s.get("q_dy"), s.get("s_dy")); rec(0, 1)
-        rec(1, 0); q_x, s_x = fq.fp8_quant_act_128x1_t(s["x"], s.get("q_x"), s.get("s_x")); rec(1, 1)
-        rec(2, 0); c = fq.fp8_gemm_wgrad(q_dy, s_dy, q_x, s_x, out=s.get("c")); rec(2, 1)
+        rec(0); q_dy, s_dy = fq.fp8_quant_act_128x1_t(s["dy"], s.get("q_dy"), s.get("s_dy")); rec(1)
+        rec(0); q_x, s_x = fq.fp8_quant_act_128x1_t(s["x"], s.get("q_x"), s.get("s_x")); rec(1)
+        rec(0); c = fq.fp8_gemm_wgrad(q_dy, s_dy, q_x, s_x, out=s.get("c")); rec(1)
         s.update(q_dy=q_dy, s_dy=s_dy, q_x=q_x, s_x=s_x, c=c)
         return c
-    rec(0, 0); qa, sa = fq.fp8_quant_act_1x128(s["a"], s.get("qa"), s.get("sa")); rec(0, 1)
-    rec(1, 0); qb, sb = fq.fp8_quant_w_128x128(s["b"], s.get("qb"), s.get("sb")); rec(1, 1)
+    qa, sa, qb, sb = quant("a", "b", "qa", "sa", "qb", "sb")
     if name == "dense_dgrad":
-        rec(2, 0); qt, st = fq.fp8_transpose_w_128x128(qb, sb, s.get("qt"), s.get("st")); rec(2, 1)
-        rec(3, 0); c = fq.fp8_gemm_blockscaled(qa, sa, qt, st, out=s.get("c")); rec(3, 1)
-        s.update(qa=qa, sa=sa, qb=qb, sb=sb, qt=qt, st=st, c=c)
+        rec(0); qt, st = fq.fp8_transpose_w_128x128(qb, sb, s.get("qt"), s.get("st")); rec(1)
+        rec(0); c = fq.fp8_gemm_blockscaled(qa, sa, qt, st, out=s.get("c")); rec(1)
+        s.update(qt=qt, st=st, c=c)
         return c
-    rec(2, 0)
+    rec(0)
     if name == "moe_contiguous":
         c = fq.fp8_grouped_gemm_contiguous(qa, sa, qb, sb, s["mi"], out=s.get("c"))
     else:
         c = fq.fp8_gemm_blockscaled(qa, sa, qb, sb, out=s.get("c"))
-    rec(2, 1)
-    s.update(qa=qa, sa=sa, qb=qb, sb=sb, c=c)
+    rec(1)
+    s.update(c=c)
     return c
 
 
@@ -562,6 +585,11 @@ def peaks_for(elapsed_ms):
     return peaks, bf16_peak * FP8_OVER_BF16, bf16_peak, sustained
 
 
+def _set_quant_mode(mode):
+    global QUANT_MODE
+    QUANT_MODE = mode
+
+
 # Secondary workloads the default run times after the headline (their own
 # per-kernel tables, rooflines and clocks under one key of the same line).
 SECONDARY = ("long_k", "moe_contiguous", "moe_masked")
@@ -611,6 +639,16 @@ def run_ours(args, name):
     m = measure(name, d, dev, args.steps, args.warmup, world, torch, fq)
     flops = step_flops(name, d)
 
+    # the same step with the operands quantized by the two separate kernels
+    # (their own launch times, for comparison with the one-launch quantizer)
+    other = None
+    if QUANT_MODE == "fused" and name in ("dense_fprop", "long_k", "moe_contiguous", "moe_masked", "dense_dgrad"):
+        try:
+            _set_quant_mode("separate")
+            other = measure(name, d, dev, args.steps, args.warmup, world, torch, fq)
+        finally:
+            _set_quant_mode("fused")
+
     # ------------------------------------------------------------ e2e (host buffers)
     e2e = run_e2e(args, name, d, dev, torch, fq, world)
     extra = None
@@ -643,6 +681,13 @@ def run_ours(args, name):
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": m["launches"], "clocks": m["clocks"],
     }
+    if other is not None:
+        op, ofp8, obf16, osus = peaks_for(other["elapsed_ms"])
+        line["separate_quantizers"] = {
+            "note": "the same step with fp8_quant_act_1x128 and fp8_quant_w_128x128 launched separately",
+            "value": world * flops * args.steps / (other["elapsed_ms"] / 1e3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": other["elapsed_ms"] / args.steps, "kernels": kernel_table(other, op, ofp8),
+            "clocks": other["clocks"]}
     if extra is not None:
         line["secondary_workloads"] = extra
     print(json.dumps(line))
@@ -735,6 +780,8 @@ def main(argv=None):
                     choices=["tiny_dense", "dense_fprop", "long_k", "moe_contiguous", "moe_masked", "dense_dgrad",
                              "moe_masked_chain", "dense_wgrad"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quant", choices=["fused", "separate"], default="fused",
+                    help="quantize a GEMM's two operands in one launch (fp8_quant_act_w) or in two")
     ap.add_argument("--no-secondary", action="store_true",
                     help="time the named workload only (the default dense_fprop run also times long_k, "
                          "moe_contiguous and moe_masked)")
@@ -744,6 +791,8 @@ def main(argv=None):
         args.warmup = 3
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         return relaunch_under_torchrun(raw, args.gpus)
+    global QUANT_MODE
+    QUANT_MODE = args.quant
     if args.impl == "reference":
         return run_reference(args, args.workload)
     return run_ours(args, args.workload)

@@ -10,6 +10,7 @@ Names and semantics match the C entry points:
 
 * :func:`fp8_quant_act_1x128`  -- bf16 [M,K] -> E4M3 [M,K] + f32 scales [M,K/128]
 * :func:`fp8_quant_w_128x128`  -- bf16 [N,K] or [G,N,K] -> E4M3 + f32 scales [..,N/128,K/128]
+* :func:`fp8_quant_act_w`      -- both of the above in one launch (the two operands of one GEMM)
 * :func:`fp8_quant_act_128x1`  -- bf16 [M,K] -> E4M3 [M,K] + f32 scales [ceil(M/128),K] (token-axis tiles)
 * :func:`fp8_quant_act_128x1_t` -- the same groups, codes token-contiguous: E4M3 [K,Mp] (tokens padded to Mp)
 * :func:`fp8_quant_act_1x128_ue8m0`, :func:`fp8_quant_w_128x128_ue8m0` -- the same groups, power-of-two scales
@@ -28,7 +29,7 @@ from pathlib import Path
 import torch
 
 __all__ = [
-    "fp8_quant_act_1x128", "fp8_quant_w_128x128", "fp8_quant_act_128x1", "fp8_quant_act_128x1_t",
+    "fp8_quant_act_1x128", "fp8_quant_w_128x128", "fp8_quant_act_w", "fp8_quant_act_128x1", "fp8_quant_act_128x1_t",
     "fp8_transpose_w_128x128", "fp8_gemm_wgrad", "fp8_swiglu_quant_1x128",
     "fp8_quant_act_1x128_ue8m0", "fp8_quant_w_128x128_ue8m0",
     "fp8_gemm_blockscaled", "fp8_grouped_gemm_contiguous",
@@ -47,6 +48,7 @@ _I64 = ctypes.c_int64
 EXPORTS = {
     "fp8_quant_act_1x128": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
     "fp8_quant_w_128x128": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
+    "fp8_quant_act_w": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P]),
     "fp8_quant_act_128x1": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
     "fp8_quant_act_128x1_t": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "fp8_quant_act_1x128_ue8m0": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
@@ -198,6 +200,38 @@ def fp8_quant_w_128x128(w: torch.Tensor, q: torch.Tensor | None = None, s: torch
     with torch.cuda.device(dev):
         _check(getattr(lib(), _entry)(_p(w), G, N, K, _p(q), _p(s), _stream(stream, dev)), _entry)
     return q, s
+
+
+def fp8_quant_act_w(x: torch.Tensor, w: torch.Tensor, qa: torch.Tensor | None = None, sa: torch.Tensor | None = None,
+                    qw: torch.Tensor | None = None, sw: torch.Tensor | None = None, stream=None):
+    """Both GEMM operands in one launch: returns ((qa, sa), (qw, sw)), exactly what
+    :func:`fp8_quant_act_1x128` (x) and :func:`fp8_quant_w_128x128` (w) return."""
+    _tensor(x, "x", _BF16, (2,))
+    _tensor(w, "w", _BF16, (2, 3))
+    M, K = x.shape
+    _multiple(K, "K")
+    G, N, Kw = (1,) + tuple(w.shape) if w.dim() == 2 else tuple(w.shape)
+    _multiple(N, "N")
+    _multiple(Kw, "K of w")
+    for t, name, dt in ((qa, "qa", _FP8), (sa, "sa", _F32), (qw, "qw", _FP8), (sw, "sw", _F32)):
+        _tensor(t, name, dt)
+    _numel(qa, M * K, "qa")
+    _numel(sa, M * (K // TILE), "sa")
+    _numel(qw, G * N * Kw, "qw")
+    _numel(sw, G * (N // TILE) * (Kw // TILE), "sw")
+    dev = _device_of(x=x, w=w, qa=qa, sa=sa, qw=qw, sw=sw)
+    if qa is None:
+        qa = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev)
+    if sa is None:
+        sa = torch.empty((M, K // TILE), dtype=torch.float32, device=dev)
+    if qw is None:
+        qw = torch.empty(tuple(w.shape), dtype=torch.float8_e4m3fn, device=dev)
+    if sw is None:
+        sw = torch.empty(tuple(w.shape[:-2]) + (N // TILE, Kw // TILE), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().fp8_quant_act_w(_p(x), M, K, _p(qa), _p(sa), _p(w), G, N, Kw, _p(qw), _p(sw),
+                                     _stream(stream, dev)), "fp8_quant_act_w")
+    return (qa, sa), (qw, sw)
 
 
 def fp8_quant_act_1x128_ue8m0(x, q=None, s=None, stream=None):

@@ -21,6 +21,8 @@
 namespace fp8q {
 
 __device__ uint32_t g_device_status;
+// Where fp8q_get_device_error's exchange kernel leaves the word it took.
+__device__ uint32_t g_device_status_taken;
 
 namespace {
 
@@ -157,6 +159,22 @@ int make_row_scale_map(CUtensorMap* map, const float* base, uint64_t rows, uint6
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
+// bf16 output [rows, N] as the epilogue's store target: a box of 32 columns x
+// 32 rows in the 64-byte swizzle.  Rows and columns past the end are not
+// written.
+int make_output_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t N) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FP8Q_ERR_CUDA;
+  const cuuint64_t dims[2] = {N, rows};
+  const cuuint64_t strides[1] = {N * 2};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- GEMM launch
 struct GemmCall {
   const uint8_t* qa;
@@ -176,9 +194,11 @@ struct GemmCall {
 
 template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D = false>
 int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
-  CUtensorMap ma, mb, msa, msb;
+  CUtensorMap ma, mb, msa, msb, mc;
   std::memset(&msa, 0, sizeof msa);
   std::memset(&msb, 0, sizeof msb);
+  int rc0 = make_output_map(&mc, g.c, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.N));
+  if (rc0) return rc0;
   int rc = make_operand_map(&ma, g.qa, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K), kBlockM);
   if (rc) return rc;
   rc = make_operand_map(&mb, g.qb, static_cast<uint64_t>(g.E * g.N), static_cast<uint64_t>(g.K), BN);
@@ -221,7 +241,7 @@ int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
   cfg.stream = stream;
   cudaError_t e =
       cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<BN, STAGES, S, kPromote, kTmaScales, k1D1D>, ma, mb, msa, msb,
-                         a);
+                         mc, a);
   if (e != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FP8Q_OK;
@@ -254,6 +274,10 @@ int check_operands(const uint8_t* qa, const float* sa, const uint8_t* qb, const 
 constexpr int64_t kMaxRows = int64_t(1) << 31;
 
 }  // namespace
+
+// Reads and clears the status word in one atomic step, after the work queued
+// before it on the caller's stream.
+__global__ void status_take_kernel(uint32_t* status, uint32_t* taken) { *taken = atomicExch(status, 0u); }
 
 // Bounded-wait self-test kernel: waits on a barrier nobody completes.
 __global__ void wait_selftest_kernel(uint32_t* status, uint64_t timeout_ns) {
@@ -333,6 +357,33 @@ static int quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, 
 }
 
 extern "C" {
+
+int fp8_quant_act_w(const void* x_bf16, int64_t M, int64_t K, uint8_t* qa, float* sa, const void* w_bf16, int64_t G,
+                    int64_t N, int64_t Kw, uint8_t* qw, float* sw, cudaStream_t stream) {
+  FP8Q_API_RANGE();
+  if (M < 0 || K < 0 || K % 128 || M >= kMaxRows || K >= kMaxRows) return FP8Q_ERR_SHAPE;
+  if (G < 0 || N < 0 || Kw < 0 || N % 128 || Kw % 128 || G >= kMaxRows || N >= kMaxRows || G * N >= kMaxRows ||
+      Kw >= kMaxRows)
+    return FP8Q_ERR_SHAPE;
+  const bool act = M > 0 && K > 0, wt = G > 0 && N > 0 && Kw > 0;
+  if (act && (!x_bf16 || !qa || !sa)) return FP8Q_ERR_NULL;
+  if (wt && (!w_bf16 || !qw || !sw)) return FP8Q_ERR_NULL;
+  if (act && (!aligned(x_bf16, 32) || !aligned(qa, 16) || !aligned(sa, 4))) return FP8Q_ERR_ALIGN;
+  if (wt && (!aligned(w_bf16, 32) || !aligned(qw, 16) || !aligned(sw, 4))) return FP8Q_ERR_ALIGN;
+  const int64_t tiles = act ? M * (K / 128) : 0;
+  const int64_t act_ctas = (tiles + kActTilesPerCta - 1) / kActTilesPerCta;
+  const int64_t blocks = wt ? G * (N / 128) * (Kw / 128) : 0;
+  if (act_ctas + blocks >= kMaxRows) return FP8Q_ERR_SHAPE;  // one CTA per 32 KB unit: the grid's x limit
+  if (act_ctas + blocks == 0) return FP8Q_OK;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  quant_act_w_kernel<<<static_cast<unsigned>(act_ctas + blocks), 256, 0, stream>>>(
+      static_cast<const uint8_t*>(x_bf16), qa, sa, tiles, act_ctas, static_cast<const uint8_t*>(w_bf16), qw, sw, Kw);
+  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
 
 int fp8_quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, float* s, cudaStream_t stream) {
   FP8Q_API_RANGE();
@@ -533,12 +584,16 @@ int fp8q_get_device_error(cudaStream_t stream) {
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);
   if (rc) return rc;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return FP8Q_ERR_CUDA;
+  uint32_t* taken = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&taken), g_device_status_taken) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
+  status_take_kernel<<<1, 1, 0, stream>>>(dev->status, taken);
+  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   uint32_t v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof v) != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (cudaMemcpyAsync(&v, taken, sizeof v, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
   if (v == 0) return FP8Q_OK;
-  const uint32_t zero = 0;
-  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero) != cudaSuccess) return FP8Q_ERR_CUDA;
   return (v & kDevErrTimeout) ? FP8Q_ERR_TIMEOUT : FP8Q_ERR_CUDA;
 }
 

@@ -86,8 +86,11 @@ struct GemmSmem {
   // full[S], empty[S], tfull[B], tempty[B], drain[2]
   static constexpr uint32_t kOffBars = STAGES * kStageBytes;
   static constexpr uint32_t kNumBars = 2 * STAGES + 2 * kAccBufs + 2;
-  static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;     // tmem slot, abort flag, total tiles
-  static constexpr uint32_t kOffPrefix = (kOffMisc + 16 + 15) / 16 * 16;
+  // misc: tmem slot, abort flag, total tiles, epilogue warps finished, and
+  // each epilogue warp's count of TMEM-buffer releases (8 words)
+  static constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;
+  static constexpr uint32_t kMiscBytes = 16 + 4 * 8;
+  static constexpr uint32_t kOffPrefix = (kOffMisc + kMiscBytes + 15) / 16 * 16;
   // Scale ring (TMA-staged scales): per group of kScaleGroup slabs, the 128
   // tile rows' activation scales as a [128][kScaleGroup] f32 box and the
   // weight block's kScaleGroup scales.  With per-row scales on both operands
@@ -98,9 +101,17 @@ struct GemmSmem {
   static constexpr uint32_t kSaSlotBytes = kBlockM * kScaleGroup * 4;  // 2 KB
   static constexpr uint32_t kSbSlotBytes = k1D1D ? BN * kScaleGroup * 4 : kScaleGroup * 4;
   static constexpr uint32_t kSbSlotStride = k1D1D ? kSbSlotBytes : 128;  // TMA destinations 128-byte aligned
-  static constexpr uint32_t kOffSa = (kOffPrefix + 4 * (kMaxMaskedExperts + 1) + 127) / 128 * 128;
+  // the masked layout's tile prefix (the weight-gradient instance is dense-only and has none)
+  static constexpr uint32_t kPrefixBytes = k1D1D ? 0u : 4u * (kMaxMaskedExperts + 1);
+  static constexpr uint32_t kOffSa = (kOffPrefix + kPrefixBytes + 127) / 128 * 128;
   static constexpr uint32_t kOffSb = kOffSa + kScaleSlots * kSaSlotBytes;
-  static constexpr uint32_t kBytes = kOffSb + kScaleSlots * kSbSlotStride;
+  // Output staging for the bf16 TMA store: per epilogue warp a 32-row x
+  // 32-column bf16 box (2 KB, 64-byte rows in the 64-byte swizzle), 1024-byte
+  // aligned so the swizzle's address bits are the box's own.
+  static constexpr uint32_t kOutBoxCols = 32;
+  static constexpr uint32_t kOutWarpBytes = 32 * kOutBoxCols * 2;
+  static constexpr uint32_t kOffOut = (kOffSb + kScaleSlots * kSbSlotStride + 1023) / 1024 * 1024;
+  static constexpr uint32_t kBytes = kOffOut + 8 * kOutWarpBytes;
   static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack for 1024-byte alignment
   static_assert(kDynamicBytes <= 227u * 1024u, "shared memory per CTA");
 };
@@ -217,13 +228,72 @@ struct Bars {
   __device__ uint32_t drain(int i) const { return base + 8u * (2 * STAGES + 2 * ACC + i); }
 };
 
+// What the epilogue warps leave for the producers' abort path: how many
+// TMEM-buffer releases each warp has posted (the kAccBufs initial ones
+// included), published once the warp has stopped, and how many warps have
+// published.
+struct EpiRecord {
+  volatile int* done;        // shared: warps that have published
+  volatile uint32_t* rel;    // shared: [8] releases posted per epilogue warp
+};
+
+// The producers' abort path (see produce): out of line, so the main loop's
+// code is the same as without it.
+template <int STAGES, int ACC>
+__device__ __noinline__ void producer_abort_drain(Bars<STAGES, ACC> bars, WaitCtl wc, uint32_t armed,
+                                                  uint32_t armed_parity, uint32_t last_armed, bool promote,
+                                                  EpiRecord epi) {
+  bool published = true;
+  if (promote) {
+    const uint64_t t0 = globaltimer_ns();
+    while (*epi.done < 8) {
+      if (globaltimer_ns() - t0 > kDrainNs) {
+        atomicOr(wc.status, kDevErrTimeout | kDevErrDrain);
+        published = false;
+        break;
+      }
+    }
+    __threadfence_block();
+  }
+  for (int st = 0; st < STAGES; ++st) {
+    if (!(armed & (1u << st))) continue;
+    const uint32_t par = (armed_parity >> st) & 1u;
+    if (promote && published && !mbar_test_wait(bars.full(st), par)) {
+      // slab of this stage's last arming: the latest j <= last_armed with j % STAGES == st
+      const uint32_t js = last_armed - (last_armed + STAGES - st) % STAGES;
+      uint32_t missing = 0;
+      for (int w = 0; w < 8; ++w)
+        if (epi.rel[w] <= js) missing += 32;
+      if (missing) mbar_arrive_cnt(bars.full(st), missing);
+    }
+    if (!published) {
+      // without the counts the phase may never complete: a short look only
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bars.full(st), par) && globaltimer_ns() - t0 < 1000000ull) {
+      }
+    } else {
+      mbar_drain(bars.full(st), par, wc.status);
+    }
+  }
+}
+
 // TMA producer `who` of two: loads the slabs j with j % 2 == who.
+//
+// Abort path: before the CTA exits, every copy this thread issued must have
+// landed in shared memory.  A stage's phase completes when its bytes have
+// landed and its TMEM-buffer releases have arrived, and after an abort some
+// releases never come, so the producer first adds, from the counts the
+// epilogue warps publish, exactly the releases that are missing (lanes of
+// warps whose count does not reach the slab), then waits for each armed phase
+// (fixed bound kDrainNs).  Release r serves slab r (the first kAccBufs are
+// posted up front, the release of slab i is the (i + kAccBufs)-th), and stage
+// s is only ever armed by producer s % 2 (STAGES is even).
 template <int BN, int STAGES, Sched S, bool kTmaScales, bool k1D1D>
 __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensorMap* tma_b,
                                         const CUtensorMap* tma_sa, const CUtensorMap* tma_sb, const GemmArgs& args,
                                         const int32_t* prefix, uint32_t s_base,
                                         Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
-                                        int32_t total, uint32_t who) {
+                                        int32_t total, uint32_t who, bool promote, EpiRecord epi) {
   using L = GemmSmem<BN, STAGES, k1D1D>;
   const int nnb = args.N / 128;
   int stage = 0;
@@ -266,14 +336,13 @@ __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensor
       }
     }
   }
-  if (*wc.abort) {
-    // let copies still in flight land before the CTA exits (bounded, 1 ms each)
-    for (int st = 0; st < STAGES; ++st)
-      if (armed & (1u << st)) {
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(bars.full(st), (armed_parity >> st) & 1u) && globaltimer_ns() - t0 < 1000000ull) {
-        }
-      }
+  if (*wc.abort && armed) {
+    // The last slab this producer armed: it arms every slab of its parity in
+    // order, and stops either at the wait of slab j (not armed: j - 2) or
+    // after the loop (the last of its slabs below j).
+    uint32_t last = ok ? j - 1u : j - 2u;
+    if ((last & 1u) != who) last -= 1u;
+    producer_abort_drain<STAGES>(bars, wc, armed, armed_parity, last, promote, epi);
   }
 }
 
@@ -324,11 +393,14 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
       }
     }
   }
-  // every MMA this thread issued completes before TMEM is released
+  // Every MMA this thread issued completes before TMEM is released.  The
+  // bound is fixed (kDrainNs), not the caller's wait limit: MMAs already
+  // issued finish in microseconds.  If it still runs out the status word
+  // records a drain timeout; TMEM is freed all the same, since a CTA that
+  // exits holding it would leave the next kernel's allocation on this SM
+  // waiting forever.
   mma_commit(bars.drain(who));
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bars.drain(who), 0) && globaltimer_ns() - t0 < args.timeout_ns) {
-  }
+  mbar_drain(bars.drain(who), 0, wc.status);
 }
 
 // Epilogue warp: promotion of every slab partial into FP32 registers, then the
@@ -339,8 +411,11 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
 // back as soon as the values are in registers, then applies
 // acc += (sa * sb) * partial.  The completion probe of the next slab is issued
 // before this slab's work and read after it.
+// Returns the number of TMEM-buffer releases the warp posted on the stage
+// barriers (with promotion; one per slab read).
 template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D>
-__device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, const int32_t* prefix,
+__device__ __forceinline__ uint32_t epilogue(const CUtensorMap* tma_c, uint32_t s_base, const GemmArgs& args,
+                                             const int32_t* prefix,
                                          Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
                                          int32_t total, uint32_t tmem_base, int warp, int lane) {
   using L = GemmSmem<BN, STAGES, k1D1D>;
@@ -369,6 +444,12 @@ __device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, 
   int buf = 0, stage = 0;
   uint32_t tphase = 0, phase = 0;
   bool ready = false;  // the current slab (or tile, without promotion) is known complete
+  // releases posted so far on the stage barriers: nkb per finished tile, plus
+  // the slabs of the tile in progress (counted where the warp stops)
+  uint32_t released = 0;
+  const uint32_t out_buf = s_base + L::kOffOut + static_cast<uint32_t>(warp - 4) * L::kOutWarpBytes;
+  bool out_pending = false;  // the staging buffer holds a box a TMA store may still be reading
+  static_assert(kCols % L::kOutBoxCols == 0, "the warp's columns are whole output boxes");
   uint32_t group = 0;  // scale groups so far (kTmaScales)
   for (int32_t t = blockIdx.x; t < total && !*wc.abort; t += gridDim.x) {
     Tile tile;
@@ -393,7 +474,11 @@ __device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, 
       // Warp-uniform outcome: the tcgen05.ld below must be executed by all 32 lanes.
       if (!ready) {
         const bool got = promote ? mbar_wait(bars.empty(stage), phase, wc, 4) : mbar_wait(bars.tfull(buf), tphase, wc, 4);
-        if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
+        if (!__all_sync(0xFFFFFFFFu, got)) {
+          ok = false;
+          if (promote) released += static_cast<uint32_t>(it);  // slabs < it were read and released
+          break;
+        }
       }
       float sa_smem = 0.0f, sb_smem = 0.0f;
       uint32_t sb_cols = 0;  // k1D1D: shared address of this half's column scales for the slab
@@ -478,7 +563,40 @@ __device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, 
       }
     }
     if (!ok) break;
-    if (row_ok && col_ok) {
+    if (promote) released += static_cast<uint32_t>(nkb);
+    // The bf16 result.  A quad whose 32 rows are all valid goes out by TMA:
+    // each 32-column half of the warp's columns is staged in the warp's
+    // buffer (lane = row, 64-byte rows, 16-byte chunk c of row l at chunk
+    // c ^ ((l >> 1) & 3): the 64-byte swizzle, so the eight lanes of each
+    // store phase hit eight distinct bank groups) and stored as one box.
+    // Rows of a partly valid quad (the last tile of a ragged M, a masked
+    // expert's last tile) are stored by their lanes, so rows past the valid
+    // ones are never written.
+    const int quad_rows = tile.rows - quad * 32;
+    if (col_ok && quad_rows >= 32) {
+#pragma unroll
+      for (int h = 0; h < kCols / static_cast<int>(L::kOutBoxCols); ++h) {
+        if (out_pending) {
+          if (lane == 0) bulk_wait_group_read0();  // the buffer's last box has been read
+          __syncwarp();
+        }
+        const uint32_t row_addr = out_buf + static_cast<uint32_t>(lane) * (L::kOutBoxCols * 2);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int p0 = h * 16 + 4 * c;
+          const uint4 o = make_uint4(bf16x2_from_pair(acc[p0]), bf16x2_from_pair(acc[p0 + 1]),
+                                     bf16x2_from_pair(acc[p0 + 2]), bf16x2_from_pair(acc[p0 + 3]));
+          sts_v4(row_addr + ((static_cast<uint32_t>(c) ^ ((lane >> 1) & 3u)) << 4), o);
+        }
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(tma_c, out_buf, col0 + h * static_cast<int>(L::kOutBoxCols), tile.a_row + quad * 32);
+          bulk_commit_group();
+        }
+        out_pending = true;
+      }
+    } else if (row_ok && col_ok) {
       __nv_bfloat16* crow = args.c + static_cast<int64_t>(tile.a_row + r) * args.N + col0;
 #pragma unroll
       for (int c = 0; c < kCols; c += 8) {
@@ -491,14 +609,19 @@ __device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, 
       }
     }
   }
+  // every box this warp stored is complete before the CTA can exit
+  if (lane == 0) bulk_wait_group0();
+  __syncwarp();
+  return released;
 }
+
 
 // ----------------------------------------------------------------- kernel
 template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                             const __grid_constant__ CUtensorMap tma_sa, const __grid_constant__ CUtensorMap tma_sb,
-                            const GemmArgs args) {
+                            const __grid_constant__ CUtensorMap tma_c, const GemmArgs args) {
   using L = GemmSmem<BN, STAGES, k1D1D>;
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "UMMA N for M=128 must be a multiple of 16 in [16,256]");
 
@@ -509,6 +632,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
   int32_t* total_slot = reinterpret_cast<int32_t*>(smem + L::kOffMisc + 8);
+  const EpiRecord epi{reinterpret_cast<volatile int*>(smem + L::kOffMisc + 12),
+                      reinterpret_cast<volatile uint32_t*>(smem + L::kOffMisc + 16)};
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + L::kOffPrefix);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -527,9 +652,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     mbar_init(bars.drain(0), 1);
     mbar_init(bars.drain(1), 1);
     *abort_flag = 0;
+    *epi.done = 0;
     fence_barrier_init();
     tma_prefetch_map(&tma_a);
     tma_prefetch_map(&tma_b);
+    tma_prefetch_map(&tma_c);
     if constexpr (kTmaScales) {
       tma_prefetch_map(&tma_sa);
       tma_prefetch_map(&tma_sb);
@@ -560,8 +687,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t n_mma = promote ? 2u : 1u;
     if (lane == 0) {
       if (warp == 0 || warp == 3)
-        produce<BN, STAGES, S, kTmaScales, k1D1D>(&tma_a, &tma_b, &tma_sa, &tma_sb, args, prefix, s_base, bars, wc, total,
-                                           warp == 0 ? 0u : 1u);
+        produce<BN, STAGES, S, kTmaScales, k1D1D>(&tma_a, &tma_b, &tma_sa, &tma_sb, args, prefix, s_base, bars, wc,
+                                                  total, warp == 0 ? 0u : 1u, promote, epi);
       else if (static_cast<uint32_t>(warp - 1) < n_mma)
         issue_mma<BN, STAGES, S, kPromote>(args, prefix, s_base, bars, wc, total, tmem_base, warp - 1, n_mma);
     }
@@ -569,7 +696,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // all TMEM slab buffers start free: every lane releases them for the first slabs
     if (promote)
       for (int b = 0; b < L::kAccBufs; ++b) mbar_arrive(bars.full(b));
-    epilogue<BN, STAGES, S, kPromote, kTmaScales, k1D1D>(s_base, args, prefix, bars, wc, total, tmem_base, warp, lane);
+    const uint32_t released =
+        epilogue<BN, STAGES, S, kPromote, kTmaScales, k1D1D>(&tma_c, s_base, args, prefix, bars, wc, total, tmem_base,
+                                                             warp, lane);
+    // publish this warp's release count for the producers' abort path
+    __syncwarp();
+    if (lane == 0) {
+      epi.rel[warp - 4] = (promote ? static_cast<uint32_t>(L::kAccBufs) : 0u) + released;
+      __threadfence_block();
+      atomicAdd(const_cast<int*>(epi.done), 1);
+    }
   }
 
   __syncwarp();

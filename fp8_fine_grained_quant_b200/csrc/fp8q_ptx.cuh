@@ -12,6 +12,12 @@ namespace fp8q {
 
 // Device status word written by bounded waits that run out.
 constexpr uint32_t kDevErrTimeout = 0x80000000u;
+// Also set when a kernel's final drain (its own copies or MMAs still in
+// flight after an abort) ran out of its fixed bound.
+constexpr uint32_t kDevErrDrain = 0x40000000u;
+// Fixed bound of those drains, independent of the caller's wait limit: the
+// copies and MMAs being drained complete in microseconds on a healthy GPU.
+constexpr uint64_t kDrainNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -39,6 +45,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// `count` arrivals at once (count >= 1).
+__device__ __forceinline__ void mbar_arrive_cnt(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
 // Suspend-time hint of the blocking probe: short, so a waiting thread notices
@@ -95,6 +106,20 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, WaitC
   }
 }
 
+// Drain wait: polls the phase for at most kDrainNs, whatever the caller's
+// limit; if it runs out, records a drain timeout.  Returns whether the phase
+// completed.
+__device__ __noinline__ bool mbar_drain(uint32_t bar, uint32_t parity, uint32_t* status) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kDrainNs) {
+      atomicOr(status, kDevErrTimeout | kDevErrDrain);
+      return false;
+    }
+  }
+  return true;
+}
+
 // Waits until the phase with the given parity has completed.  Returns false
 // (after recording a timeout) if it does not within the limit.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& w, uint32_t site) {
@@ -127,6 +152,30 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
           dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+
+// 2-D tiled bulk copy shared -> global (no multicast): the box at (x, y) of
+// the map's tensor, rows and columns past the tensor's extent not written.
+// Completes as part of this thread's current bulk async-group.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until this thread's committed bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Waits until this thread's committed bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy (TMA) reads of them.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05
@@ -291,6 +340,13 @@ __device__ __forceinline__ void ld_nc_v8(const void* p, uint32_t (&w)[8]) {
 __device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+  return r;
+}
+
+// Per-half maximum of two packed bf16 pairs.
+__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
 

@@ -44,22 +44,39 @@ __device__ __forceinline__ float group_scale(float amax) {
 
 // Division-free codes with an exactness filter.
 //
-// Each code must be E4M3_RNE(fl32(x / s)).  With r = RN(1/s) (s a normal
-// float), r_lo = RN(r (1 - 2^-20)) and r_hi = RN(r (1 + 2^-20)) satisfy
-// r_lo < 1/s < r_hi, so for x > 0, x r_lo < x/s < x r_hi (reversed for
-// x < 0), and by the monotonicity of rounding RN(x r_lo) <= fl32(x/s) <=
-// RN(x r_hi).  Rounding to E4M3 is monotone too, so when the two products get
-// the same code, fl32(x/s) gets that code.  When they differ (a quotient
-// within ~2^-20 of an E4M3 rounding midpoint, a few in 10^5) the IEEE
-// quotient is used.  Products below the binary32 normal range are far below
-// the first E4M3 midpoint (2^-10) and give +-0 on every path (each product
-// keeps the sign of x).
+// Each code must be E4M3_RNE(fl32(x / s)).  Given r_lo < 1/s < r_hi, for
+// x > 0, x r_lo < x/s < x r_hi (reversed for x < 0), and by the monotonicity
+// of rounding RN(x r_lo) <= fl32(x/s) <= RN(x r_hi).  Rounding to E4M3 is
+// monotone too, so when the two products get the same code, fl32(x/s) gets
+// that code.  When they differ (a quotient within ~2^-20 of an E4M3 rounding
+// midpoint, a few in 10^5) the IEEE quotient is used.  Products below the
+// binary32 normal range are far below the first E4M3 midpoint (2^-10) and
+// give +-0 on every path (each product keeps the sign of x).
+//
+// The bracket comes from the hardware's approximate reciprocal r ~ 1/s
+// (s a normal float), widened to r_lo = RN(r (1 - 2^-20)) and r_hi =
+// RN(r (1 + 2^-20)).  Whether it really brackets 1/s is then checked exactly:
+// fma(-s, r_lo, 1) is 1 - s r_lo rounded once, which keeps the sign of the
+// exact residual, so it is > 0 exactly when r_lo < 1/s (and < 0 for r_hi
+// exactly when r_hi > 1/s).  A bracket that fails the check sends its group
+// to the division path, so the codes never depend on how accurate the
+// approximate reciprocal is.
+__device__ __forceinline__ bool recip_bracket(float s, float& lo, float& hi) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+  lo = __fmul_rn(r, 1.0f - 0x1p-20f);
+  hi = __fmul_rn(r, 1.0f + 0x1p-20f);
+  return __fmaf_rn(-s, lo, 1.0f) > 0.0f && __fmaf_rn(-s, hi, 1.0f) < 0.0f;
+}
+
 struct RecipPair {
   uint64_t lo2, hi2;  // {r_lo, r_lo} and {r_hi, r_hi}
+  bool ok;            // the bracket holds (else: the division path)
 };
 __device__ __forceinline__ RecipPair recip_pair(float s) {
-  const float r = __frcp_rn(s);
-  return {pack_f32x2(__fmul_rn(r, 1.0f - 0x1p-20f)), pack_f32x2(__fmul_rn(r, 1.0f + 0x1p-20f))};
+  float lo, hi;
+  const bool ok = recip_bracket(s, lo, hi);
+  return {pack_f32x2(lo), pack_f32x2(hi), ok};
 }
 
 // Scales below this are not safely normal for the reciprocal path.
@@ -94,17 +111,19 @@ __device__ __forceinline__ uint4 quantize16(const uint32_t (&w)[8], float s, con
     hi[i] = e4m3x4_from_f32x2(mul_f32x2(x0, rp.hi2), mul_f32x2(x1, rp.hi2));
   }
   const uint32_t diff = (lo[0] ^ hi[0]) | (lo[1] ^ hi[1]) | (lo[2] ^ hi[2]) | (lo[3] ^ hi[3]);
-  if (exact_only || diff != 0u) return quantize16_exact(w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7], s);
+  if (exact_only || !rp.ok || diff != 0u) return quantize16_exact(w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7], s);
   return make_uint4(lo[0], lo[1], lo[2], lo[3]);
 }
 
-// Largest magnitude of the 16 bf16 in w, as a float.
+// Largest magnitude of the 16 bf16 in w, as a float: packed bf16 maxima of
+// the magnitudes (sign bits cleared; exact, no rounding), then the larger
+// half widened to binary32.
 __device__ __forceinline__ float abs_max16(const uint32_t (&w)[8]) {
-  float m = 0.0f;
+  uint32_t m[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xFFFF0000u))));
-  return m;
+  for (int i = 0; i < 4; ++i) m[i] = max_bf16x2(w[2 * i] & 0x7FFF7FFFu, w[2 * i + 1] & 0x7FFF7FFFu);
+  const uint32_t a = max_bf16x2(max_bf16x2(m[0], m[1]), max_bf16x2(m[2], m[3]));
+  return fmaxf(__uint_as_float(a & 0xFFFF0000u), __uint_as_float(a << 16));
 }
 
 __device__ __forceinline__ void zero8(uint32_t (&w)[8]) {
@@ -192,54 +211,109 @@ __global__ void __launch_bounds__(256, 5) quant_act_1x128_kernel(const uint8_t* 
 // 128x128 weight blocks.  One 256-thread CTA per block: eight lanes cover one
 // 256-byte row segment, 32 rows per pass, 4 passes; the block (32 KB) stays in
 // registers between the amax reduction and the quantization, so it is read
-// from HBM once (four CTAs per SM; the compiler keeps a few words of it in
-// local memory).  Block b = (g * N/128 + nb) * K/128 + kb, also the index of
-// its scale in s[G, N/128, K/128].  Grid-stride over blocks.
+// from HBM once (four CTAs per SM, 59 registers).  Block b = (g * N/128 + nb)
+// * K/128 + kb, also the index of its scale in s[G, N/128, K/128].
+// `warp_max` is 8 floats of shared memory; consecutive blocks of one CTA
+// alternate between two such halves, so one CTA barrier per block suffices.
 // ---------------------------------------------------------------------------
 template <bool kPow2>
-__global__ void __launch_bounds__(256, 4) quant_w_128x128_kernel(const uint8_t* __restrict__ w,
-                                                                 uint8_t* __restrict__ q, float* __restrict__ s,
-                                                                 int64_t K, int64_t num_blocks) {
-  __shared__ float warp_max[2][8];  // alternate halves: one CTA barrier per block
+__device__ __forceinline__ void quant_w_block(const uint8_t* __restrict__ w, uint8_t* __restrict__ q,
+                                              float* __restrict__ s, int64_t K, int64_t b, float* warp_max) {
   const int tid = threadIdx.x;
   const int sub = tid & 7;    // 32-byte chunk within the 256-byte row segment
   const int rsub = tid >> 3;  // row within a pass of 32 rows
   const int64_t nkb = K >> 7;
+  const int64_t kb = b % nkb;
+  const int64_t row0 = (b / nkb) * 128;  // first row in the [G*N, K] view
+  const uint8_t* src = w + (row0 * K + kb * 128) * 2 + sub * 32;
+  uint32_t v[4][8];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) ld_nc_v8(src + (p * 32 + rsub) * K * 2, v[p]);
+  float amax = 0.0f;
+#pragma unroll
+  for (int p = 0; p < 4; ++p) amax = fmaxf(amax, abs_max16(v[p]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+  if ((tid & 31) == 0) warp_max[tid >> 5] = amax;
+  __syncthreads();
+  amax = warp_max[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, warp_max[i]);
+  uint8_t* dst = q + row0 * K + kb * 128 + sub * 16;
+  float sc;
+  if constexpr (kPow2) {
+    float inv;
+    sc = pow2_scale(amax, &inv);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) *reinterpret_cast<uint4*>(dst + (p * 32 + rsub) * K) = quantize16_pow2(v[p], inv);
+  } else {
+    sc = group_scale(amax);
+    const RecipPair rp = recip_pair(sc);
+    const bool exact_only = sc < kMinFastScale;
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+      *reinterpret_cast<uint4*>(dst + (p * 32 + rsub) * K) = quantize16(v[p], sc, rp, exact_only);
+  }
+  if (tid == 0) s[b] = sc;
+}
+
+// Grid-stride over weight blocks.
+template <bool kPow2>
+__global__ void __launch_bounds__(256, 4) quant_w_128x128_kernel(const uint8_t* __restrict__ w,
+                                                                 uint8_t* __restrict__ q, float* __restrict__ s,
+                                                                 int64_t K, int64_t num_blocks) {
+  __shared__ float warp_max[2][8];
   int half = 0;
-  for (int64_t b = blockIdx.x; b < num_blocks; b += gridDim.x, half ^= 1) {
-    const int64_t kb = b % nkb;
-    const int64_t row0 = (b / nkb) * 128;  // first row in the [G*N, K] view
-    const uint8_t* src = w + (row0 * K + kb * 128) * 2 + sub * 32;
-    uint32_t v[4][8];
+  for (int64_t b = blockIdx.x; b < num_blocks; b += gridDim.x, half ^= 1)
+    quant_w_block<kPow2>(w, q, s, K, b, warp_max[half]);
+}
+
+// ---------------------------------------------------------------------------
+// Both operands of a GEMM in one launch: the 1x128 activation quantization
+// and the 128x128 weight quantization, the same codes and scales as the two
+// kernels above, bit for bit.  Every CTA quantizes one 32 KB unit: CTAs
+// below `act_ctas` take 128 consecutive activation tiles (four per lane
+// group, all loaded before any is reduced), the others one weight block.
+// One launch instead of two: the ramp-up and the last partial wave are paid
+// once, and the two streams share the device.
+// ---------------------------------------------------------------------------
+constexpr int kActTilesPerCta = 128;
+
+__global__ void __launch_bounds__(256, 4) quant_act_w_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ qa,
+                                                             float* __restrict__ sa, int64_t num_tiles,
+                                                             int64_t act_ctas, const uint8_t* __restrict__ w,
+                                                             uint8_t* __restrict__ qw, float* __restrict__ sw,
+                                                             int64_t Kw) {
+  __shared__ float warp_max[8];
+  if (static_cast<int64_t>(blockIdx.x) >= act_ctas) {
+    quant_w_block<false>(w, qw, sw, Kw, static_cast<int64_t>(blockIdx.x) - act_ctas, warp_max);
+    return;
+  }
+  const int sub = threadIdx.x & 7;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kActTilesPerCta + (threadIdx.x >> 3);
+  constexpr int kPer = kActTilesPerCta / 32;  // tiles per lane group
+  uint32_t v[kPer][8];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) ld_nc_v8(src + (p * 32 + rsub) * K * 2, v[p]);
-    float amax = 0.0f;
+  for (int u = 0; u < kPer; ++u) {
+    const int64_t t = t0 + u * 32;
+    if (t < num_tiles)
+      ld_nc_v8(x + t * 256 + sub * 32, v[u]);
+    else
+      zero8(v[u]);
+  }
+  // every lane runs every step (the shuffles need all 32); tiles past the end store nothing
 #pragma unroll
-    for (int p = 0; p < 4; ++p) amax = fmaxf(amax, abs_max16(v[p]));
+  for (int u = 0; u < kPer; ++u) {
+    const int64_t t = t0 + u * 32;
+    float amax = abs_max16(v[u]);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-    if ((tid & 31) == 0) warp_max[half][tid >> 5] = amax;
-    __syncthreads();
-    amax = warp_max[half][0];
-#pragma unroll
-    for (int i = 1; i < 8; ++i) amax = fmaxf(amax, warp_max[half][i]);
-    uint8_t* dst = q + row0 * K + kb * 128 + sub * 16;
-    float sc;
-    if constexpr (kPow2) {
-      float inv;
-      sc = pow2_scale(amax, &inv);
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-        *reinterpret_cast<uint4*>(dst + (p * 32 + rsub) * K) = quantize16_pow2(v[p], inv);
-    } else {
-      sc = group_scale(amax);
-      const RecipPair rp = recip_pair(sc);
-      const bool exact_only = sc < kMinFastScale;
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-        *reinterpret_cast<uint4*>(dst + (p * 32 + rsub) * K) = quantize16(v[p], sc, rp, exact_only);
+    for (int off = 4; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+    const float sc = group_scale(amax);
+    const RecipPair rp = recip_pair(sc);
+    if (t < num_tiles) {
+      *reinterpret_cast<uint4*>(qa + t * 128 + sub * 16) = quantize16(v[u], sc, rp, sc < kMinFastScale);
+      if (sub == 0) sa[t] = sc;
     }
-    if (tid == 0) s[b] = sc;
   }
 }
 
@@ -332,10 +406,11 @@ __global__ void __launch_bounds__(256, kMinBlocks) quant_act_128x1_kernel(const 
     bool exact_only = false;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float r0 = __frcp_rn(sc[2 * i]), r1 = __frcp_rn(sc[2 * i + 1]);
-      asm("mov.b64 %0, {%1, %2};" : "=l"(lo2[i]) : "f"(__fmul_rn(r0, 1.0f - 0x1p-20f)), "f"(__fmul_rn(r1, 1.0f - 0x1p-20f)));
-      asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[i]) : "f"(__fmul_rn(r0, 1.0f + 0x1p-20f)), "f"(__fmul_rn(r1, 1.0f + 0x1p-20f)));
-      exact_only |= sc[2 * i] < kMinFastScale || sc[2 * i + 1] < kMinFastScale;
+      float l0, h0, l1, h1;
+      const bool ok0 = recip_bracket(sc[2 * i], l0, h0), ok1 = recip_bracket(sc[2 * i + 1], l1, h1);
+      asm("mov.b64 %0, {%1, %2};" : "=l"(lo2[i]) : "f"(l0), "f"(l1));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[i]) : "f"(h0), "f"(h1));
+      exact_only |= sc[2 * i] < kMinFastScale || sc[2 * i + 1] < kMinFastScale || !ok0 || !ok1;
     }
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
@@ -457,10 +532,11 @@ __global__ void __launch_bounds__(256, kMinBlocks) quant_act_128x1_t_kernel(cons
     bool exact_only = false;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float r0 = __frcp_rn(sc[2 * i]), r1 = __frcp_rn(sc[2 * i + 1]);
-      asm("mov.b64 %0, {%1, %2};" : "=l"(lo2[i]) : "f"(__fmul_rn(r0, 1.0f - 0x1p-20f)), "f"(__fmul_rn(r1, 1.0f - 0x1p-20f)));
-      asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[i]) : "f"(__fmul_rn(r0, 1.0f + 0x1p-20f)), "f"(__fmul_rn(r1, 1.0f + 0x1p-20f)));
-      exact_only |= sc[2 * i] < kMinFastScale || sc[2 * i + 1] < kMinFastScale;
+      float l0, h0, l1, h1;
+      const bool ok0 = recip_bracket(sc[2 * i], l0, h0), ok1 = recip_bracket(sc[2 * i + 1], l1, h1);
+      asm("mov.b64 %0, {%1, %2};" : "=l"(lo2[i]) : "f"(l0), "f"(l1));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[i]) : "f"(h0), "f"(h1));
+      exact_only |= sc[2 * i] < kMinFastScale || sc[2 * i + 1] < kMinFastScale || !ok0 || !ok1;
     }
     // codes of the 8 tokens (zero rows past M give code 0)
     uint32_t clo[8], chi[8];

@@ -37,9 +37,10 @@
  *    FP8Q_ERR_SHAPE.
  *  - Non-finite inputs are outside the contract (results unspecified, no fault).
  *  - Every on-device wait is bounded (default 4 s, see fp8q_set_wait_timeout_ns);
- *    a wait that runs out records FP8Q_ERR_TIMEOUT in a device status word,
- *    the kernel releases its resources and returns, and the host reads the
- *    word with fp8q_get_device_error.
+ *    a wait that runs out records FP8Q_ERR_TIMEOUT in a device status word
+ *    (one per device), the kernel lets its copies and MMAs in flight finish
+ *    (a fixed bound, independent of the wait limit), releases its resources
+ *    and returns, and the host reads the word with fp8q_get_device_error.
  */
 #ifndef FP8Q_H_
 #define FP8Q_H_
@@ -90,6 +91,20 @@ FP8Q_API int fp8_quant_act_1x128(const void* x_bf16, int64_t M, int64_t K, uint8
  */
 FP8Q_API int fp8_quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, uint8_t* q, float* s,
                         cudaStream_t stream);
+
+/*
+ * Both operands of one GEMM in a single launch: exactly the codes and scales
+ * of fp8_quant_act_1x128(x) and fp8_quant_w_128x128(w), bit for bit (the
+ * same per-group rule: "The Insider Secrets Of Deepseek Discovered", FP8
+ * passage, Figure 7 (a)).  One launch instead of two, so the ramp-up and the
+ * last partial wave of a launch are paid once per GEMM step.
+ *   x_bf16, M, K, qa, sa     : as fp8_quant_act_1x128 (M = 0 or K = 0: no activations)
+ *   w_bf16, G, N, Kw, qw, sw : as fp8_quant_w_128x128 (G, N or Kw = 0: no weights)
+ * Same requirements and errors as the two calls; the argument checks of both
+ * run before anything is launched.
+ */
+FP8Q_API int fp8_quant_act_w(const void* x_bf16, int64_t M, int64_t K, uint8_t* qa, float* sa, const void* w_bf16,
+                             int64_t G, int64_t N, int64_t Kw, uint8_t* qw, float* sw, cudaStream_t stream);
 
 /*
  * The same two quantizers with power-of-two (UE8M0) group scales: the
@@ -253,9 +268,15 @@ FP8Q_API int fp8_gemm_unpromoted_diag(const uint8_t* qa, const float* sa, const 
 FP8Q_API const char* fp8q_status_string(int status);
 
 /*
- * Synchronizes `stream`, then reads and clears the device status word that
- * bounded waits write.  Returns FP8Q_OK, FP8Q_ERR_TIMEOUT, or FP8Q_ERR_CUDA if
- * the synchronization itself failed.
+ * Reads and clears, in one atomic exchange queued on `stream` after the work
+ * already on it, the device status word that bounded waits write, then
+ * synchronizes `stream`.  Returns FP8Q_OK, FP8Q_ERR_TIMEOUT, or FP8Q_ERR_CUDA
+ * if the launch or the synchronization failed.
+ * The word is one per device, shared by every stream and every call of the
+ * library on that device: a timeout is not attributed to a call or a stream,
+ * and a call still running on another stream may record one after the
+ * exchange (it is then reported by the next query).  A timeout also covers a
+ * kernel's final drain running out of its fixed bound (2 s) after an abort.
  */
 FP8Q_API int fp8q_get_device_error(cudaStream_t stream);
 

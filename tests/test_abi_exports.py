@@ -57,6 +57,7 @@ A16 = 0x10000  # a 256-byte aligned fake address; never dereferenced
 A16_ONLY = 0x10010  # 16-byte but not 32-byte aligned
 A4 = 0x10004   # 4-byte aligned only
 A1 = 0x10001
+BIG_ = 1 << 31
 
 
 def _call(name, *args):
@@ -89,6 +90,27 @@ def test_quant_act_validation(args, expect):
 ])
 def test_quant_w_validation(args, expect):
     assert _call("fp8_quant_w_128x128", *args) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((A16, 4, 100, A16, A16, A16, 1, 128, 128, A16, A16, None), fq.ERR_SHAPE),   # activation K
+    ((A16, 4, 128, A16, A16, A16, 1, 100, 128, A16, A16, None), fq.ERR_SHAPE),   # weight N
+    ((A16, 4, 128, A16, A16, A16, 1, 128, 100, A16, A16, None), fq.ERR_SHAPE),   # weight K
+    ((A16, BIG_, 128, A16, A16, A16, 1, 128, 128, A16, A16, None), fq.ERR_SHAPE),
+    ((A16, 4, 128, A16, A16, A16, 1 << 24, 1 << 8, 128, A16, A16, None), fq.ERR_SHAPE),  # G*N = 2^32
+    ((None, 4, 128, A16, A16, A16, 1, 128, 128, A16, A16, None), fq.ERR_NULL),
+    ((A16, 4, 128, A16, A16, None, 1, 128, 128, A16, A16, None), fq.ERR_NULL),
+    ((A16, 4, 128, A16, A16, A16, 1, 128, 128, A16, None, None), fq.ERR_NULL),
+    ((A16_ONLY, 4, 128, A16, A16, A16, 1, 128, 128, A16, A16, None), fq.ERR_ALIGN),
+    ((A16, 4, 128, A16, A16, A16_ONLY, 1, 128, 128, A16, A16, None), fq.ERR_ALIGN),
+    ((A16, 4, 128, A16, A1, A16, 1, 128, 128, A16, A16, None), fq.ERR_ALIGN),
+    ((A16, 0, 128, A16, A16, A16, 0, 128, 128, A16, A16, None), fq.OK),           # both empty
+    ((None, 0, 128, None, None, None, 0, 128, 128, None, None, None), fq.OK),     # empty parts need no pointers
+])
+def test_quant_act_w_validation(args, expect):
+    """The fused two-operand quantizer checks both operands' shapes, pointers
+    and alignment before anything is launched."""
+    assert _call("fp8_quant_act_w", *args) == expect
 
 
 @pytest.mark.parametrize("name", ["fp8_gemm_blockscaled", "fp8_gemm_unpromoted_diag"])

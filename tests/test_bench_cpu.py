@@ -33,10 +33,17 @@ def test_reference_arm_prints_contract_line():
 
 def test_kernel_plan_accounting():
     d = wl.tiny_dense()
-    plan = dict((k, (b, f)) for k, b, f in bench.kernel_plan("tiny_dense", d))
     M, N, K = 128, 256, 512
-    assert plan["quant_act_1x128"][0] == M * K * 3 + M * (K // 128) * 4
-    assert plan["quant_w_128x128"][0] == N * K * 3 + (N // 128) * (K // 128) * 4
+    act = M * K * 3 + M * (K // 128) * 4
+    wt = N * K * 3 + (N // 128) * (K // 128) * 4
+    try:
+        bench._set_quant_mode("separate")
+        plan = dict((k, (b, f)) for k, b, f in bench.kernel_plan("tiny_dense", d))
+        assert plan["quant_act_1x128"][0] == act and plan["quant_w_128x128"][0] == wt
+    finally:
+        bench._set_quant_mode("fused")
+    plan = dict((k, (b, f)) for k, b, f in bench.kernel_plan("tiny_dense", d))
+    assert plan["quant_act_w"][0] == act + wt  # one launch for both operands
     assert plan["gemm_blockscaled"][1] == 2.0 * M * N * K
     assert plan["gemm_blockscaled"][0] == M * K + M * (K // 128) * 4 + N * K + (N // 128) * (K // 128) * 4 + M * N * 2
 
@@ -106,6 +113,6 @@ def test_dgrad_plan_counts_the_transposed_gemm():
     d = SimpleNamespace(M=4096, N=7168, K=7168)
     plan = bench.kernel_plan("dense_dgrad", d)
     labels = [l for l, _, _ in plan]
-    assert labels == ["quant_act_1x128", "quant_w_128x128", "transpose_w_128x128", "gemm_dgrad"]
+    assert labels == ["quant_act_w", "transpose_w_128x128", "gemm_dgrad"]
     assert plan[-1][2] == 2.0 * 4096 * 7168 * 7168
-    assert plan[2][1] == 2 * 7168 * 7168 + 8 * 56 * 56
+    assert plan[1][1] == 2 * 7168 * 7168 + 8 * 56 * 56

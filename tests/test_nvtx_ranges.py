@@ -32,6 +32,7 @@ calls = [
     ("fp8_quant_act_1x128", (A16, 4, 100, A16, A16, None)),
     ("fp8_quant_act_1x128_ue8m0", (A16, 0, 128, A16, A16, None)),
     ("fp8_quant_w_128x128", (None, 1, 128, 128, A16, A16, None)),
+    ("fp8_quant_act_w", (A16, 4, 100, A16, A16, A16, 1, 128, 128, A16, A16, None)),
     ("fp8_quant_w_128x128_ue8m0", (A16, 1, 100, 128, A16, A16, None)),
     ("fp8_quant_act_128x1", (A16, 4, 128, A16, A1, None)),
     ("fp8_transpose_w_128x128", (A16, A16, 1, 128, 0, A16, A16, None)),
@@ -71,7 +72,7 @@ def test_every_entry_point_pushes_and_pops_one_named_range(recorder):
     res = subprocess.run([sys.executable, "-c", CHILD, str(ROOT), str(recorder)], env=env,
                          capture_output=True, text=True, timeout=300, check=True)
     rows = json.loads(res.stdout.strip().splitlines()[-1])
-    assert len(rows) == 13
+    assert len(rows) == 14
     for r in rows:
         assert r["rc"] in (fq.OK, fq.ERR_SHAPE, fq.ERR_NULL, fq.ERR_ALIGN), r
         assert r["log"] == "push %s\npop\n" % r["name"], r

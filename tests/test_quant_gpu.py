@@ -258,3 +258,62 @@ def test_ue8m0_w_matches_oracle(dev, G, N, K):
     oq, os_ = oracle.quant_w_128x128_ue8m0(w)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
     assert np.array_equal(bytes_of(q).reshape(oq.shape), oq)
+
+
+# ------------------------------------------------------------------ both operands in one launch
+def _fused_exact(a_bits, w_bits, dev):
+    x = to_torch_bf16(a_bits, dev)
+    w = to_torch_bf16(w_bits, dev)
+    (qa, sa), (qw, sw) = fq.fp8_quant_act_w(x, w)
+    torch.cuda.synchronize(dev)
+    assert fq.get_device_error(device=dev) == fq.OK
+    if a_bits.size:
+        oq, os_ = oracle.quant_act_1x128(a_bits)
+        assert np.array_equal(sa.cpu().numpy().reshape(os_.shape).view(np.uint32), os_.view(np.uint32))
+        assert np.array_equal(bytes_of(qa).reshape(oq.shape), oq)
+    if w_bits.size:
+        oq, os_ = oracle.quant_w_128x128(w_bits)
+        assert np.array_equal(sw.cpu().numpy().reshape(os_.shape).view(np.uint32), os_.view(np.uint32))
+        assert np.array_equal(bytes_of(qw).reshape(oq.shape), oq)
+    return (qa, sa), (qw, sw)
+
+
+@pytest.mark.parametrize("M,K,Gw,N,Kw", [
+    (300, 384, 1, 256, 640),     # 900 tiles: a partial last activation unit
+    (1, 128, 3, 128, 128),       # one tile, batched weights
+    (4097, 1024, 2, 384, 256),   # ragged rows, more units than SMs
+])
+def test_fused_operands_exact(dev, M, K, Gw, N, Kw):
+    rng = np.random.default_rng(M + K + N)
+    a = wl.bf16_bits((rng.standard_normal((M, K)) * np.exp(rng.standard_normal(K))).astype(np.float32))
+    w = wl.bf16_bits((0.02 * rng.standard_normal((Gw, N, Kw))).astype(np.float32))
+    _fused_exact(a, w if Gw > 1 else w[0], dev)
+
+
+def test_fused_operands_equal_the_separate_kernels_dense_fprop(dev):
+    """dense_fprop in full: the fused launch gives the bytes of the two
+    separate quantizers, which are bit-exact against the oracle."""
+    d = wl.dense_fprop()
+    (qa, sa), (qw, sw) = _fused_exact(d.a, d.b, dev)
+    qa2, sa2 = fq.fp8_quant_act_1x128(to_torch_bf16(d.a, dev))
+    qw2, sw2 = fq.fp8_quant_w_128x128(to_torch_bf16(d.b, dev))
+    torch.cuda.synchronize(dev)
+    assert torch.equal(qa.view(torch.uint8), qa2.view(torch.uint8)) and torch.equal(sa, sa2)
+    assert torch.equal(qw.view(torch.uint8), qw2.view(torch.uint8)) and torch.equal(sw, sw2)
+
+
+def test_fused_operands_one_side_empty(dev):
+    rng = np.random.default_rng(9)
+    a = wl.bf16_bits(rng.standard_normal((64, 256)).astype(np.float32))
+    w = wl.bf16_bits(rng.standard_normal((128, 256)).astype(np.float32))
+    x = to_torch_bf16(a, dev)
+    ww = to_torch_bf16(w, dev)
+    (qa, sa), _ = fq.fp8_quant_act_w(x, torch.empty((0, 128, 256), dtype=torch.bfloat16, device=dev))
+    torch.cuda.synchronize(dev)
+    oq, os_ = oracle.quant_act_1x128(a)
+    assert np.array_equal(bytes_of(qa).reshape(oq.shape), oq)
+    _, (qw, sw) = fq.fp8_quant_act_w(torch.empty((0, 128), dtype=torch.bfloat16, device=dev), ww)
+    torch.cuda.synchronize(dev)
+    oq, os_ = oracle.quant_w_128x128(w)
+    assert np.array_equal(bytes_of(qw).reshape(oq.shape), oq)
+    assert fq.get_device_error(device=dev) == fq.OK
