@@ -149,15 +149,31 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- workloads
+# Reduced sizes of the same workloads for ncu captures that take many passes
+# (a few GB on the device at most); never a bench line of their own.
+PROFILE_SIZES = {
+    "dense_fprop": dict(M=2048), "long_k": dict(M=1024), "moe_contiguous": dict(tokens=1024, E=8),
+    "moe_masked": dict(E=8),
+}
+PROFILE_SIZE = False
+
+
 def make_workload(name: str, shard: int = 0, device=None):
     """The named workload; ``shard`` r > 0 is rank r's part of the batch
     (row blocks for the dense shapes, experts for the MoE ones; see
     workloads.row_shard / expert_shard).  ``device`` draws the large MoE
     tensors on that device instead of the host."""
     import workloads as wl
-    if name in ("dense_fprop", "dense_dgrad"):
+    if PROFILE_SIZE and name in PROFILE_SIZES:
+        kw = PROFILE_SIZES[name]
+        if name.startswith("moe"):
+            return wl.CONFIGS[name](device=device, **kw)
+        return wl.CONFIGS[name](**kw)
+    if name in ("dense_fprop", "dense_dgrad", "dense_fprop_mx"):
         # dense_dgrad: the activation-gradient GEMM of the dense_fprop layer;
-        # dY takes the shape and distribution of the forward activations
+        # dY takes the shape and distribution of the forward activations.
+        # dense_fprop_mx: the same GEMM with power-of-two scales applied by
+        # the tensor cores
         return wl.dense_fprop(shard=shard)
     if name == "long_k":
         return wl.long_k(shard=shard)
@@ -167,13 +183,13 @@ def make_workload(name: str, shard: int = 0, device=None):
         # moe_masked_chain: GEMM2's activation is the SwiGLU of GEMM1's output,
         # requantized (its own A2 draw is not used)
         return wl.moe_masked(shard=shard, device=device)
-    if name == "moe_contiguous":
+    if name in ("moe_contiguous", "moe_contiguous_mx"):
         return wl.moe_contiguous(shard=shard, device=device)
     return wl.CONFIGS[name]()
 
 
 def describe(name: str, d) -> dict:
-    if name in ("tiny_dense", "dense_fprop", "long_k"):
+    if name in ("tiny_dense", "dense_fprop", "long_k", "dense_fprop_mx"):
         return {"workload": "%s M=%d N=%d K=%d" % (name, d.M, d.N, d.K), "M": d.M, "N": d.N, "K": d.K,
                 "seed": d.meta["seed"]}
     if name == "dense_dgrad":
@@ -182,9 +198,9 @@ def describe(name: str, d) -> dict:
     if name == "dense_wgrad":
         return {"workload": "dense_wgrad dW[N,K] = dY[M,N]^T X[M,K] M=%d N=%d K=%d" % (d.M, d.N, d.K), "M": d.M,
                 "N": d.N, "K": d.K, "seed": d.meta["seed"]}
-    if name == "moe_contiguous":
-        return {"workload": "moe_contiguous E=%d M_tot=%d (valid %d) N=%d K=%d" % (d.E, d.M_tot, int(d.counts.sum()),
-                                                                                 d.N, d.K),
+    if name in ("moe_contiguous", "moe_contiguous_mx"):
+        return {"workload": "%s E=%d M_tot=%d (valid %d) N=%d K=%d" % (name, d.E, d.M_tot, int(d.counts.sum()),
+                                                                     d.N, d.K),
                 "E": d.E, "M_tot": d.M_tot, "valid_rows": int(d.counts.sum()), "N": d.N, "K": d.K,
                 "seed": d.meta["seed"]}
     return {"workload": "%s E=%d cap=%d valid=%d (N,K)=(%d,%d)+(%d,%d)" % (
@@ -223,7 +239,7 @@ def build_sets(name, d, dev, nsets, torch, fq):
         else:
             s["a"] = _to_dev_bf16(torch, d.a, dev)
             s["b"] = _to_dev_bf16(torch, d.b, dev)
-            if name == "moe_contiguous":
+            if name in ("moe_contiguous", "moe_contiguous_mx"):
                 s["mi"] = _to_dev_i32(torch, d.m_indices, dev)
         sets.append(s)
     return sets
@@ -254,6 +270,20 @@ def kernel_plan(name, d):
     if name in ("tiny_dense", "dense_fprop", "long_k"):
         M, N, K = d.M, d.N, d.K
         return quant(qa_bytes(M, K), qw_bytes(1, N, K)) + [("gemm_blockscaled", gemm_bytes(M, N, K), 2.0 * M * N * K)]
+    if name in ("dense_fprop_mx", "moe_contiguous_mx"):
+        # power-of-two scales: the _ue8m0 quantizers, the scales' E8M0 atoms,
+        # then the GEMM with the scales applied in the tensor cores
+        contiguous = name == "moe_contiguous_mx"
+        rows, G = (d.M_tot, d.E) if contiguous else (d.M, 1)
+        N, K = d.N, d.K
+        nkb = K // TILE
+        atoms_a, atoms_b = -(-rows // TILE) * nkb * 512, G * (N // TILE) * nkb * 512
+        gemm = rows * K + G * N * K + atoms_a + atoms_b + rows * N * 2
+        return [("quant_act_1x128_ue8m0", qa_bytes(rows, K), 0.0), ("quant_w_128x128_ue8m0", qw_bytes(G, N, K), 0.0),
+                ("mx_scales_act", rows * nkb * 4 + atoms_a, 0.0),
+                ("mx_scales_w", G * (N // TILE) * nkb * 4 + atoms_b, 0.0),
+                ("grouped_gemm_mx_contiguous" if contiguous else "gemm_mx", gemm,
+                 d.flops if contiguous else 2.0 * rows * N * K)]
     if name == "dense_dgrad":
         # dY is d.a [M, Nout], W is d.b [Nout, K]; dX = dY W is [M, K]
         M, Nout, K = d.M, d.N, d.K
@@ -345,6 +375,19 @@ def launch_step(name, d, s, fq, events=None):
         rec(1)
         s.update(c=c, c2=c2)
         return c2
+    if name in ("dense_fprop_mx", "moe_contiguous_mx"):
+        rec(0); qa, sa = fq.fp8_quant_act_1x128_ue8m0(s["a"], s.get("qa"), s.get("sa")); rec(1)
+        rec(0); qb, sb = fq.fp8_quant_w_128x128_ue8m0(s["b"], s.get("qb"), s.get("sb")); rec(1)
+        rec(0); sfa = fq.fp8_mx_scales_act(sa, s.get("sfa")); rec(1)
+        rec(0); sfb = fq.fp8_mx_scales_w(sb, s.get("sfb")); rec(1)
+        rec(0)
+        if name == "moe_contiguous_mx":
+            c = fq.fp8_grouped_gemm_mx_contiguous(qa, sfa, qb, sfb, s["mi"], out=s.get("c"))
+        else:
+            c = fq.fp8_gemm_mx(qa, sfa, qb, sfb, out=s.get("c"))
+        rec(1)
+        s.update(qa=qa, sa=sa, qb=qb, sb=sb, sfa=sfa, sfb=sfb, c=c)
+        return c
     if name == "dense_wgrad":
         rec(0); q_dy, s_dy = fq.fp8_quant_act_128x1_t(s["dy"], s.get("q_dy"), s.get("s_dy")); rec(1)
         rec(0); q_x, s_x = fq.fp8_quant_act_128x1_t(s["x"], s.get("q_x"), s.get("s_x")); rec(1)
@@ -392,7 +435,7 @@ def oracle_sample_step(name, d, rows: int, nblocks: int):
         return dt, 2.0 * rows * TILE * nblocks * d.M
     if name in ("moe_masked", "moe_masked_chain"):
         a, b = d.a[0], d.b[0]
-    elif name == "moe_contiguous":
+    elif name in ("moe_contiguous", "moe_contiguous_mx"):
         a, b = d.a, d.b[int(d.m_indices[0])]
     else:
         a, b = d.a, d.b
@@ -690,6 +733,8 @@ def run_ours(args, name):
             "clocks": other["clocks"]}
     if extra is not None:
         line["secondary_workloads"] = extra
+    if PROFILE_SIZE:
+        line["profile_size"] = "reduced shapes for a profiler capture: not a bench line"
     print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist
@@ -778,10 +823,12 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dense_fprop",
                     choices=["tiny_dense", "dense_fprop", "long_k", "moe_contiguous", "moe_masked", "dense_dgrad",
-                             "moe_masked_chain", "dense_wgrad"])
+                             "moe_masked_chain", "dense_wgrad", "dense_fprop_mx", "moe_contiguous_mx"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quant", choices=["fused", "separate"], default="fused",
                     help="quantize a GEMM's two operands in one launch (fp8_quant_act_w) or in two")
+    ap.add_argument("--profile-size", action="store_true",
+                    help="reduced shapes of the same workload, for ncu captures (the line says so)")
     ap.add_argument("--no-secondary", action="store_true",
                     help="time the named workload only (the default dense_fprop run also times long_k, "
                          "moe_contiguous and moe_masked)")
@@ -791,8 +838,9 @@ def main(argv=None):
         args.warmup = 3
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         return relaunch_under_torchrun(raw, args.gpus)
-    global QUANT_MODE
+    global QUANT_MODE, PROFILE_SIZE
     QUANT_MODE = args.quant
+    PROFILE_SIZE = args.profile_size
     if args.impl == "reference":
         return run_reference(args, args.workload)
     return run_ours(args, args.workload)

@@ -16,6 +16,8 @@ Names and semantics match the C entry points:
 * :func:`fp8_quant_act_1x128_ue8m0`, :func:`fp8_quant_w_128x128_ue8m0` -- the same groups, power-of-two scales
 * :func:`fp8_transpose_w_128x128` -- block-quantized W [..,N,K] -> W^T [..,K,N] (codes and block scales)
 * :func:`fp8_swiglu_quant_1x128` -- GEMM1 output [.., 2I] bf16 -> SwiGLU -> 1x128 E4M3 [.., I] + scales
+* :func:`fp8_mx_scales_act`, :func:`fp8_mx_scales_w`, :func:`fp8_gemm_mx` -- power-of-two scales applied by
+  the tensor cores (E8M0 scale atoms, no CUDA-core promotion)
 * :func:`fp8_gemm_blockscaled` -- C = A * B^T (bf16) with per-128-slab promotion
 * :func:`fp8_grouped_gemm_contiguous` -- MoE grouped GEMM, contiguous layout
 * :func:`fp8_grouped_gemm_masked`     -- MoE grouped GEMM, masked layout
@@ -33,7 +35,8 @@ __all__ = [
     "fp8_transpose_w_128x128", "fp8_gemm_wgrad", "fp8_swiglu_quant_1x128",
     "fp8_quant_act_1x128_ue8m0", "fp8_quant_w_128x128_ue8m0",
     "fp8_gemm_blockscaled", "fp8_grouped_gemm_contiguous",
-    "fp8_grouped_gemm_masked", "fp8_gemm_unpromoted_diag", "get_device_error", "set_wait_timeout_ns",
+    "fp8_grouped_gemm_masked", "fp8_gemm_unpromoted_diag", "fp8_mx_scales_act", "fp8_mx_scales_w", "fp8_gemm_mx",
+    "fp8_grouped_gemm_mx_contiguous", "fp8_grouped_gemm_mx_masked", "get_device_error", "set_wait_timeout_ns",
     "selftest_wait_timeout", "launch_count", "status_string", "Fp8qError", "lib", "LIB_PATH", "EXPORTS",
 ]
 
@@ -59,6 +62,11 @@ EXPORTS = {
     "fp8_grouped_gemm_contiguous": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "fp8_grouped_gemm_masked": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P]),
     "fp8_gemm_unpromoted_diag": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "fp8_mx_scales_act": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
+    "fp8_mx_scales_w": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P]),
+    "fp8_gemm_mx": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "fp8_grouped_gemm_mx_contiguous": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
+    "fp8_grouped_gemm_mx_masked": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "fp8_gemm_wgrad": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "fp8q_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fp8q_get_device_error": (ctypes.c_int, [_P]),
@@ -423,6 +431,124 @@ def fp8_gemm_wgrad(q_dy_t, s_dy, q_x_t, s_x, out: torch.Tensor | None = None, st
     with torch.cuda.device(dev):
         _check(lib().fp8_gemm_wgrad(_p(q_dy_t), _p(s_dy), _p(q_x_t), _p(s_x), _p(out), N, K, Mp,
                                     _stream(stream, dev)), "fp8_gemm_wgrad")
+    return out
+
+
+MX_ATOM = 512  # bytes of E8M0 scales per 128-row tile and 128-deep slab
+
+
+def fp8_mx_scales_act(sa: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Power-of-two 1x128 scales sa [M, K/128] f32 -> E8M0 atoms [ceil(M/128), K/128, 512] uint8."""
+    _tensor(sa, "sa", _F32, (2,))
+    M, nkb = sa.shape
+    mt = (M + TILE - 1) // TILE
+    _tensor(out, "out", (torch.uint8,))
+    _numel(out, mt * nkb * MX_ATOM, "out")
+    dev = _device_of(sa=sa, out=out)
+    if out is None:
+        out = torch.empty((mt, nkb, MX_ATOM), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().fp8_mx_scales_act(_p(sa), M, nkb * TILE, _p(out), _stream(stream, dev)), "fp8_mx_scales_act")
+    return out
+
+
+def fp8_mx_scales_w(sb: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Power-of-two 128x128 block scales sb [(G,) N/128, K/128] f32 -> E8M0 atoms [G*N/128, K/128, 512]."""
+    _tensor(sb, "sb", _F32, (2, 3))
+    G, nnb, nkb = (1,) + tuple(sb.shape) if sb.dim() == 2 else tuple(sb.shape)
+    _tensor(out, "out", (torch.uint8,))
+    _numel(out, G * nnb * nkb * MX_ATOM, "out")
+    dev = _device_of(sb=sb, out=out)
+    if out is None:
+        out = torch.empty((G * nnb, nkb, MX_ATOM), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().fp8_mx_scales_w(_p(sb), G, nnb * TILE, nkb * TILE, _p(out), _stream(stream, dev)),
+               "fp8_mx_scales_w")
+    return out
+
+
+def fp8_gemm_mx(qa, sfa_mx, qb, sfb_mx, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """C[M,N] (bf16) = A * B^T with power-of-two scales applied by the tensor cores: qa [M,K], qb [N,K]
+    E4M3 from the _ue8m0 quantizers, their scales converted by fp8_mx_scales_act / fp8_mx_scales_w."""
+    _tensor(qa, "qa", _FP8, (2,))
+    _tensor(qb, "qb", _FP8, (2,))
+    _tensor(sfa_mx, "sfa_mx", (torch.uint8,))
+    _tensor(sfb_mx, "sfb_mx", (torch.uint8,))
+    _tensor(out, "out", _BF16)
+    M, K = qa.shape
+    N = qb.shape[0]
+    if qb.shape[1] != K:
+        raise ValueError("qa and qb differ in K (%d, %d)" % (K, qb.shape[1]))
+    _multiple(N, "N")
+    _multiple(K, "K")
+    _numel(sfa_mx, ((M + TILE - 1) // TILE) * (K // TILE) * MX_ATOM, "sfa_mx")
+    _numel(sfb_mx, (N // TILE) * (K // TILE) * MX_ATOM, "sfb_mx")
+    _numel(out, M * N, "out")
+    dev = _device_of(qa=qa, sfa_mx=sfa_mx, qb=qb, sfb_mx=sfb_mx, out=out)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().fp8_gemm_mx(_p(qa), _p(sfa_mx), _p(qb), _p(sfb_mx), _p(out), M, N, K, _stream(stream, dev)),
+               "fp8_gemm_mx")
+    return out
+
+
+def fp8_grouped_gemm_mx_contiguous(qa, sfa_mx, qb, sfb_mx, m_indices, out: torch.Tensor | None = None, stream=None):
+    """Contiguous-layout grouped GEMM with power-of-two scales applied by the tensor cores:
+    qa [M_tot,K], qb [E,N,K] E4M3, their scale atoms, m_indices int32 [M_tot/128]."""
+    _tensor(qa, "qa", _FP8, (2,))
+    _tensor(qb, "qb", _FP8, (3,))
+    _tensor(sfa_mx, "sfa_mx", (torch.uint8,))
+    _tensor(sfb_mx, "sfb_mx", (torch.uint8,))
+    _tensor(m_indices, "m_indices", _I32)
+    _tensor(out, "out", _BF16)
+    M_tot, K = qa.shape
+    E, N, K2 = qb.shape
+    if K2 != K:
+        raise ValueError("qa and qb differ in K (%d, %d)" % (K, K2))
+    _multiple(M_tot, "M_tot")
+    _multiple(N, "N")
+    _multiple(K, "K")
+    _numel(sfa_mx, (M_tot // TILE) * (K // TILE) * MX_ATOM, "sfa_mx")
+    _numel(sfb_mx, E * (N // TILE) * (K // TILE) * MX_ATOM, "sfb_mx")
+    _numel(m_indices, M_tot // TILE, "m_indices")
+    _numel(out, M_tot * N, "out")
+    dev = _device_of(qa=qa, sfa_mx=sfa_mx, qb=qb, sfb_mx=sfb_mx, m_indices=m_indices, out=out)
+    if out is None:
+        out = torch.empty((M_tot, N), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().fp8_grouped_gemm_mx_contiguous(_p(qa), _p(sfa_mx), _p(qb), _p(sfb_mx), _p(m_indices), _p(out),
+                                                    M_tot, N, K, E, _stream(stream, dev)),
+               "fp8_grouped_gemm_mx_contiguous")
+    return out
+
+
+def fp8_grouped_gemm_mx_masked(qa, sfa_mx, qb, sfb_mx, masked_m, out: torch.Tensor | None = None, stream=None):
+    """Masked-layout grouped GEMM with power-of-two scales applied by the tensor cores:
+    qa [E,cap,K], qb [E,N,K] E4M3, their scale atoms, masked_m int32 [E]; rows >= masked_m[e] unwritten."""
+    _tensor(qa, "qa", _FP8, (3,))
+    _tensor(qb, "qb", _FP8, (3,))
+    _tensor(sfa_mx, "sfa_mx", (torch.uint8,))
+    _tensor(sfb_mx, "sfb_mx", (torch.uint8,))
+    _tensor(masked_m, "masked_m", _I32)
+    _tensor(out, "out", _BF16)
+    E, cap, K = qa.shape
+    E2, N, K2 = qb.shape
+    if E2 != E or K2 != K:
+        raise ValueError("qa [E=%d, K=%d] and qb [E=%d, K=%d] do not agree" % (E, K, E2, K2))
+    _multiple(cap, "cap")
+    _multiple(N, "N")
+    _multiple(K, "K")
+    _numel(sfa_mx, E * (cap // TILE) * (K // TILE) * MX_ATOM, "sfa_mx")
+    _numel(sfb_mx, E * (N // TILE) * (K // TILE) * MX_ATOM, "sfb_mx")
+    _numel(masked_m, E, "masked_m")
+    _numel(out, E * cap * N, "out")
+    dev = _device_of(qa=qa, sfa_mx=sfa_mx, qb=qb, sfb_mx=sfb_mx, masked_m=masked_m, out=out)
+    if out is None:
+        out = torch.empty((E, cap, N), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().fp8_grouped_gemm_mx_masked(_p(qa), _p(sfa_mx), _p(qb), _p(sfb_mx), _p(masked_m), _p(out), E,
+                                                cap, N, K, _stream(stream, dev)), "fp8_grouped_gemm_mx_masked")
     return out
 
 

@@ -15,6 +15,7 @@
 
 #include "fp8q.h"
 #include "fp8q_gemm.cuh"
+#include "fp8q_gemm_mx.cuh"
 #include "fp8q_ptx.cuh"
 #include "fp8q_quant.cuh"
 
@@ -82,6 +83,15 @@ int device_info(DeviceInfo** out) {
         if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kMasked, true, true>();
         if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kMasked, true, false>();
         if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kDense, true, true, true>();
+        if (e == cudaSuccess)
+          e = cudaFuncSetAttribute(gemm_mx_kernel<Sched::kDense>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   MxSmem::kDynamicBytes);
+        if (e == cudaSuccess)
+          e = cudaFuncSetAttribute(gemm_mx_kernel<Sched::kContiguous>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   MxSmem::kDynamicBytes);
+        if (e == cudaSuccess)
+          e = cudaFuncSetAttribute(gemm_mx_kernel<Sched::kMasked>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   MxSmem::kDynamicBytes);
         if (e != cudaSuccess) return FP8Q_ERR_CUDA;
       }
       d.ready.store(true, std::memory_order_release);
@@ -159,22 +169,6 @@ int make_row_scale_map(CUtensorMap* map, const float* base, uint64_t rows, uint6
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
-// bf16 output [rows, N] as the epilogue's store target: a box of 32 columns x
-// 32 rows in the 64-byte swizzle.  Rows and columns past the end are not
-// written.
-int make_output_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t N) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return FP8Q_ERR_CUDA;
-  const cuuint64_t dims[2] = {N, rows};
-  const cuuint64_t strides[1] = {N * 2};
-  const cuuint32_t box[2] = {32, 32};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
-}
-
 // ---------------------------------------------------------------- GEMM launch
 struct GemmCall {
   const uint8_t* qa;
@@ -192,13 +186,29 @@ struct GemmCall {
   int promote;
 };
 
+// One launch of one kernel instance.
+template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D>
+int launch_instance(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa, const CUtensorMap& msb,
+                    const GemmArgs& a, int64_t grid, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = GemmSmem<BN, STAGES, k1D1D>::kDynamicBytes;
+  cfg.stream = stream;
+  cudaError_t e =
+      cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<BN, STAGES, S, kPromote, kTmaScales, k1D1D>, ma, mb, msa, msb,
+                         a);
+  if (e != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
 template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D = false>
 int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
-  CUtensorMap ma, mb, msa, msb, mc;
+  CUtensorMap ma, mb, msa, msb;
   std::memset(&msa, 0, sizeof msa);
   std::memset(&msb, 0, sizeof msb);
-  int rc0 = make_output_map(&mc, g.c, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.N));
-  if (rc0) return rc0;
   int rc = make_operand_map(&ma, g.qa, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K), kBlockM);
   if (rc) return rc;
   rc = make_operand_map(&mb, g.qb, static_cast<uint64_t>(g.E * g.N), static_cast<uint64_t>(g.K), BN);
@@ -217,6 +227,7 @@ int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
     if (rc) return rc;
   }
   GemmArgs a;
+  std::memset(&a, 0, sizeof a);
   a.sa = g.sa;
   a.sb = g.sb;
   a.c = static_cast<__nv_bfloat16*>(g.c);
@@ -230,21 +241,10 @@ int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
   a.E = static_cast<int32_t>(g.E);
   a.m_tiles = static_cast<int32_t>(g.m_tiles);
   a.n_tiles = static_cast<int32_t>((g.N + BN - 1) / BN);
-  int64_t max_tiles = g.m_tiles * a.n_tiles * (S == Sched::kMasked ? g.E : 1);
-  const int grid = static_cast<int>(max_tiles < dev.num_sms ? max_tiles : dev.num_sms);
+  const int64_t max_tiles = g.m_tiles * a.n_tiles * (S == Sched::kMasked ? g.E : 1);
+  const int64_t grid = max_tiles < dev.num_sms ? max_tiles : dev.num_sms;
   if (grid <= 0) return FP8Q_OK;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof cfg);
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = GemmSmem<BN, STAGES, k1D1D>::kDynamicBytes;
-  cfg.stream = stream;
-  cudaError_t e =
-      cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<BN, STAGES, S, kPromote, kTmaScales, k1D1D>, ma, mb, msa, msb,
-                         mc, a);
-  if (e != cudaSuccess) return FP8Q_ERR_CUDA;
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return FP8Q_OK;
+  return launch_instance<BN, STAGES, S, kPromote, kTmaScales, k1D1D>(ma, mb, msa, msb, a, grid, stream);
 }
 
 template <Sched S>
@@ -353,6 +353,55 @@ static int quant_w_128x128(const void* w_bf16, int64_t G, int64_t N, int64_t K, 
                                                                            K, blocks);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
+// Launch of the block-scaled GEMM for one layout; g carries the GemmCall
+// shapes (a_rows, M, N, K, E, m_tiles) and layout arrays.
+template <Sched S>
+static int launch_mx(const GemmCall& g, const uint8_t* sfa_mx, const uint8_t* sfb_mx, cudaStream_t stream) {
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  CUtensorMap ma, mb;
+  rc = make_operand_map(&ma, g.qa, static_cast<uint64_t>(g.a_rows), static_cast<uint64_t>(g.K), kBlockM);
+  if (rc) return rc;
+  rc = make_operand_map(&mb, g.qb, static_cast<uint64_t>(g.E * g.N), static_cast<uint64_t>(g.K), 128);
+  if (rc) return rc;
+  MxArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.g.c = static_cast<__nv_bfloat16*>(g.c);
+  a.g.m_indices = g.m_indices;
+  a.g.masked_m = g.masked_m;
+  a.g.status = dev->status;
+  a.g.timeout_ns = g_timeout_ns.load();
+  a.g.M = static_cast<int32_t>(g.M);
+  a.g.N = static_cast<int32_t>(g.N);
+  a.g.nkb = static_cast<int32_t>(g.K / kSlabK);
+  a.g.E = static_cast<int32_t>(g.E);
+  a.g.m_tiles = static_cast<int32_t>(g.m_tiles);
+  a.g.n_tiles = static_cast<int32_t>(g.N / 128);
+  a.sfa = sfa_mx;
+  a.sfb = sfb_mx;
+  const int64_t max_tiles = g.m_tiles * (g.N / 128) * (S == Sched::kMasked ? g.E : 1);
+  const int grid = static_cast<int>(max_tiles < dev->num_sms ? max_tiles : dev->num_sms);
+  if (grid <= 0) return FP8Q_OK;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = MxSmem::kDynamicBytes;
+  cfg.stream = stream;
+  if (cudaLaunchKernelEx(&cfg, gemm_mx_kernel<S>, ma, mb, a) != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
+static int check_mx_operands(const uint8_t* qa, const uint8_t* sfa_mx, const uint8_t* qb, const uint8_t* sfb_mx,
+                             const void* c) {
+  if (!qa || !sfa_mx || !qb || !sfb_mx || !c) return FP8Q_ERR_NULL;
+  if (!aligned(qa, 16) || !aligned(qb, 16) || !aligned(c, 16) || !aligned(sfa_mx, 16) || !aligned(sfb_mx, 16))
+    return FP8Q_ERR_ALIGN;
   return FP8Q_OK;
 }
 
@@ -467,6 +516,88 @@ int fp8_quant_act_128x1_t(const void* x_bf16, int64_t M, int64_t K, int64_t Mp, 
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FP8Q_OK;
+}
+
+int fp8_mx_scales_act(const float* sa, int64_t M, int64_t K, uint8_t* sfa_mx, cudaStream_t stream) {
+  FP8Q_API_RANGE();
+  if (M < 0 || K < 0 || K % 128 || M >= kMaxRows || K >= kMaxRows) return FP8Q_ERR_SHAPE;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (!sa || !sfa_mx) return FP8Q_ERR_NULL;
+  if (!aligned(sa, 4) || !aligned(sfa_mx, 16)) return FP8Q_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  const int64_t nkb = K / 128, total = ((M + 127) / 128) * nkb * 32;
+  int64_t grid = (total + 255) / 256;
+  if (grid > dev->num_sms * 8) grid = dev->num_sms * 8;
+  mx_scales_act_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(sa, sfa_mx, M, nkb, total);
+  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
+int fp8_mx_scales_w(const float* sb, int64_t G, int64_t N, int64_t K, uint8_t* sfb_mx, cudaStream_t stream) {
+  FP8Q_API_RANGE();
+  if (G < 0 || N < 0 || K < 0 || N % 128 || K % 128 || G >= kMaxRows || N >= kMaxRows || G * N >= kMaxRows ||
+      K >= kMaxRows)
+    return FP8Q_ERR_SHAPE;
+  if (G == 0 || N == 0 || K == 0) return FP8Q_OK;
+  if (!sb || !sfb_mx) return FP8Q_ERR_NULL;
+  if (!aligned(sb, 4) || !aligned(sfb_mx, 16)) return FP8Q_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  const int64_t total = G * (N / 128) * (K / 128) * 32;
+  int64_t grid = (total + 255) / 256;
+  if (grid > dev->num_sms * 8) grid = dev->num_sms * 8;
+  mx_scales_w_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(sb, sfb_mx, total);
+  if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
+int fp8_gemm_mx(const uint8_t* qa, const uint8_t* sfa_mx, const uint8_t* qb, const uint8_t* sfb_mx, void* c_bf16,
+                int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+  FP8Q_API_RANGE();
+  if (M < 0 || N < 0 || K < 128 || K % 128 || N % 128 || M >= kMaxRows || N >= kMaxRows || K >= kMaxRows)
+    return FP8Q_ERR_SHAPE;
+  if (M == 0 || N == 0) return FP8Q_OK;
+  int rc = check_mx_operands(qa, sfa_mx, qb, sfb_mx, c_bf16);
+  if (rc) return rc;
+  GemmCall g{qa, nullptr, qb, nullptr, c_bf16, nullptr, nullptr, M, M, N, K, 1, (M + kBlockM - 1) / kBlockM, 0, 1};
+  return launch_mx<Sched::kDense>(g, sfa_mx, sfb_mx, stream);
+}
+
+int fp8_grouped_gemm_mx_contiguous(const uint8_t* qa, const uint8_t* sfa_mx, const uint8_t* qb,
+                                   const uint8_t* sfb_mx, const int32_t* m_indices, void* c_bf16, int64_t M_tot,
+                                   int64_t N, int64_t K, int64_t E, cudaStream_t stream) {
+  FP8Q_API_RANGE();
+  if (M_tot < 0 || N < 0 || E < 0 || K < 128 || K % 128 || N % 128 || M_tot % 128 || M_tot >= kMaxRows ||
+      K >= kMaxRows || E * N >= kMaxRows)
+    return FP8Q_ERR_SHAPE;
+  if (M_tot == 0 || N == 0 || E == 0) return FP8Q_OK;
+  int rc = check_mx_operands(qa, sfa_mx, qb, sfb_mx, c_bf16);
+  if (rc) return rc;
+  if (!m_indices) return FP8Q_ERR_NULL;
+  if (!aligned(m_indices, 4)) return FP8Q_ERR_ALIGN;
+  GemmCall g{qa, nullptr, qb, nullptr, c_bf16, m_indices, nullptr, M_tot, M_tot, N, K, E, M_tot / kBlockM, 0, 1};
+  return launch_mx<Sched::kContiguous>(g, sfa_mx, sfb_mx, stream);
+}
+
+int fp8_grouped_gemm_mx_masked(const uint8_t* qa, const uint8_t* sfa_mx, const uint8_t* qb, const uint8_t* sfb_mx,
+                               const int32_t* masked_m, void* c_bf16, int64_t E, int64_t cap, int64_t N, int64_t K,
+                               cudaStream_t stream) {
+  FP8Q_API_RANGE();
+  if (E < 0 || cap < 0 || N < 0 || K < 128 || K % 128 || N % 128 || cap % 128 || E > kMaxMaskedExperts ||
+      E * cap >= kMaxRows || E * N >= kMaxRows || K >= kMaxRows)
+    return FP8Q_ERR_SHAPE;
+  if (E == 0 || cap == 0 || N == 0) return FP8Q_OK;
+  int rc = check_mx_operands(qa, sfa_mx, qb, sfb_mx, c_bf16);
+  if (rc) return rc;
+  if (!masked_m) return FP8Q_ERR_NULL;
+  if (!aligned(masked_m, 4)) return FP8Q_ERR_ALIGN;
+  GemmCall g{qa, nullptr, qb, nullptr, c_bf16, nullptr, masked_m, E * cap, cap, N, K, E, cap / kBlockM, 0, 1};
+  return launch_mx<Sched::kMasked>(g, sfa_mx, sfb_mx, stream);
 }
 
 int fp8_transpose_w_128x128(const uint8_t* q, const float* s, int64_t G, int64_t N, int64_t K, uint8_t* qt,

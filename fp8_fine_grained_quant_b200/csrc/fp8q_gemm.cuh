@@ -105,13 +105,7 @@ struct GemmSmem {
   static constexpr uint32_t kPrefixBytes = k1D1D ? 0u : 4u * (kMaxMaskedExperts + 1);
   static constexpr uint32_t kOffSa = (kOffPrefix + kPrefixBytes + 127) / 128 * 128;
   static constexpr uint32_t kOffSb = kOffSa + kScaleSlots * kSaSlotBytes;
-  // Output staging for the bf16 TMA store: per epilogue warp a 32-row x
-  // 32-column bf16 box (2 KB, 64-byte rows in the 64-byte swizzle), 1024-byte
-  // aligned so the swizzle's address bits are the box's own.
-  static constexpr uint32_t kOutBoxCols = 32;
-  static constexpr uint32_t kOutWarpBytes = 32 * kOutBoxCols * 2;
-  static constexpr uint32_t kOffOut = (kOffSb + kScaleSlots * kSbSlotStride + 1023) / 1024 * 1024;
-  static constexpr uint32_t kBytes = kOffOut + 8 * kOutWarpBytes;
+  static constexpr uint32_t kBytes = kOffSb + kScaleSlots * kSbSlotStride;
   static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack for 1024-byte alignment
   static_assert(kDynamicBytes <= 227u * 1024u, "shared memory per CTA");
 };
@@ -228,21 +222,18 @@ struct Bars {
   __device__ uint32_t drain(int i) const { return base + 8u * (2 * STAGES + 2 * ACC + i); }
 };
 
-// What the epilogue warps leave for the producers' abort path: how many
-// TMEM-buffer releases each warp has posted (the kAccBufs initial ones
-// included), published once the warp has stopped, and how many warps have
-// published.
+// What the epilogue warps leave for the producers' abort path: where each
+// warp stopped, as (stage + STAGES * phase) of the next slab it had not yet
+// read (its slab index modulo 2 * STAGES), and how many warps have published.
 struct EpiRecord {
   volatile int* done;        // shared: warps that have published
-  volatile uint32_t* rel;    // shared: [8] releases posted per epilogue warp
+  volatile uint32_t* pos;    // shared: [8] stopping position per epilogue warp
 };
 
-// The producers' abort path (see produce): out of line, so the main loop's
-// code is the same as without it.
+// The producers' abort path (see produce).
 template <int STAGES, int ACC>
 __device__ __noinline__ void producer_abort_drain(Bars<STAGES, ACC> bars, WaitCtl wc, uint32_t armed,
-                                                  uint32_t armed_parity, uint32_t last_armed, bool promote,
-                                                  EpiRecord epi) {
+                                                  uint32_t armed_parity, bool promote, EpiRecord epi) {
   bool published = true;
   if (promote) {
     const uint64_t t0 = globaltimer_ns();
@@ -259,15 +250,24 @@ __device__ __noinline__ void producer_abort_drain(Bars<STAGES, ACC> bars, WaitCt
     if (!(armed & (1u << st))) continue;
     const uint32_t par = (armed_parity >> st) & 1u;
     if (promote && published && !mbar_test_wait(bars.full(st), par)) {
-      // slab of this stage's last arming: the latest j <= last_armed with j % STAGES == st
-      const uint32_t js = last_armed - (last_armed + STAGES - st) % STAGES;
+      // The stage's pending slab js (js mod 2 STAGES = st + STAGES par) needs
+      // the release of slab js - ACC from every warp.  A warp that stopped
+      // before slab je (je mod 2 STAGES published) has released the slabs
+      // below je.  0 <= js - je: js's MMAs have not run, so no warp read it.
+      // js - je < STAGES + ACC <= 2 STAGES: js was armed after the MMAs of
+      // js - STAGES completed, which needed every warp's release of slab
+      // js - STAGES - ACC.  So js - je is their difference modulo 2 STAGES,
+      // and the warp's release is missing when js - je >= ACC.
+      const uint32_t js = static_cast<uint32_t>(st) + STAGES * par;
       uint32_t missing = 0;
-      for (int w = 0; w < 8; ++w)
-        if (epi.rel[w] <= js) missing += 32;
+      for (int w = 0; w < 8; ++w) {
+        const uint32_t d = (js + 2 * STAGES - epi.pos[w]) % (2 * STAGES);
+        if (d >= static_cast<uint32_t>(ACC)) missing += 32;
+      }
       if (missing) mbar_arrive_cnt(bars.full(st), missing);
     }
     if (!published) {
-      // without the counts the phase may never complete: a short look only
+      // without the positions the phase may never complete: a short look only
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(bars.full(st), par) && globaltimer_ns() - t0 < 1000000ull) {
       }
@@ -282,12 +282,12 @@ __device__ __noinline__ void producer_abort_drain(Bars<STAGES, ACC> bars, WaitCt
 // Abort path: before the CTA exits, every copy this thread issued must have
 // landed in shared memory.  A stage's phase completes when its bytes have
 // landed and its TMEM-buffer releases have arrived, and after an abort some
-// releases never come, so the producer first adds, from the counts the
-// epilogue warps publish, exactly the releases that are missing (lanes of
-// warps whose count does not reach the slab), then waits for each armed phase
-// (fixed bound kDrainNs).  Release r serves slab r (the first kAccBufs are
-// posted up front, the release of slab i is the (i + kAccBufs)-th), and stage
-// s is only ever armed by producer s % 2 (STAGES is even).
+// releases never come, so the producer first adds, from the stopping
+// positions the epilogue warps publish, exactly the releases that are missing,
+// then waits for each armed phase (fixed bound kDrainNs).  The stage barrier
+// of slab j takes the release of slab j - kAccBufs (the first kAccBufs slabs'
+// are posted up front), and stage s is only ever armed by producer s % 2
+// (STAGES is even).
 template <int BN, int STAGES, Sched S, bool kTmaScales, bool k1D1D>
 __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensorMap* tma_b,
                                         const CUtensorMap* tma_sa, const CUtensorMap* tma_sb, const GemmArgs& args,
@@ -336,14 +336,7 @@ __device__ __forceinline__ void produce(const CUtensorMap* tma_a, const CUtensor
       }
     }
   }
-  if (*wc.abort && armed) {
-    // The last slab this producer armed: it arms every slab of its parity in
-    // order, and stops either at the wait of slab j (not armed: j - 2) or
-    // after the loop (the last of its slabs below j).
-    uint32_t last = ok ? j - 1u : j - 2u;
-    if ((last & 1u) != who) last -= 1u;
-    producer_abort_drain<STAGES>(bars, wc, armed, armed_parity, last, promote, epi);
-  }
+  if (*wc.abort && armed) producer_abort_drain<STAGES>(bars, wc, armed, armed_parity, promote, epi);
 }
 
 // MMA issuer `who` of `n`: four K = 32 MMAs per slab.  With promotion every
@@ -411,11 +404,9 @@ __device__ __forceinline__ void issue_mma(const GemmArgs& args, const int32_t* p
 // back as soon as the values are in registers, then applies
 // acc += (sa * sb) * partial.  The completion probe of the next slab is issued
 // before this slab's work and read after it.
-// Returns the number of TMEM-buffer releases the warp posted on the stage
-// barriers (with promotion; one per slab read).
+// At its end the warp publishes where it stopped (EpiRecord).
 template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D>
-__device__ __forceinline__ uint32_t epilogue(const CUtensorMap* tma_c, uint32_t s_base, const GemmArgs& args,
-                                             const int32_t* prefix,
+__device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, EpiRecord epi, const int32_t* prefix,
                                          Bars<STAGES, GemmSmem<BN, STAGES>::kAccBufs> bars, WaitCtl wc,
                                          int32_t total, uint32_t tmem_base, int warp, int lane) {
   using L = GemmSmem<BN, STAGES, k1D1D>;
@@ -444,12 +435,6 @@ __device__ __forceinline__ uint32_t epilogue(const CUtensorMap* tma_c, uint32_t 
   int buf = 0, stage = 0;
   uint32_t tphase = 0, phase = 0;
   bool ready = false;  // the current slab (or tile, without promotion) is known complete
-  // releases posted so far on the stage barriers: nkb per finished tile, plus
-  // the slabs of the tile in progress (counted where the warp stops)
-  uint32_t released = 0;
-  const uint32_t out_buf = s_base + L::kOffOut + static_cast<uint32_t>(warp - 4) * L::kOutWarpBytes;
-  bool out_pending = false;  // the staging buffer holds a box a TMA store may still be reading
-  static_assert(kCols % L::kOutBoxCols == 0, "the warp's columns are whole output boxes");
   uint32_t group = 0;  // scale groups so far (kTmaScales)
   for (int32_t t = blockIdx.x; t < total && !*wc.abort; t += gridDim.x) {
     Tile tile;
@@ -474,11 +459,7 @@ __device__ __forceinline__ uint32_t epilogue(const CUtensorMap* tma_c, uint32_t 
       // Warp-uniform outcome: the tcgen05.ld below must be executed by all 32 lanes.
       if (!ready) {
         const bool got = promote ? mbar_wait(bars.empty(stage), phase, wc, 4) : mbar_wait(bars.tfull(buf), tphase, wc, 4);
-        if (!__all_sync(0xFFFFFFFFu, got)) {
-          ok = false;
-          if (promote) released += static_cast<uint32_t>(it);  // slabs < it were read and released
-          break;
-        }
+        if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
       }
       float sa_smem = 0.0f, sb_smem = 0.0f;
       uint32_t sb_cols = 0;  // k1D1D: shared address of this half's column scales for the slab
@@ -563,40 +544,9 @@ __device__ __forceinline__ uint32_t epilogue(const CUtensorMap* tma_c, uint32_t 
       }
     }
     if (!ok) break;
-    if (promote) released += static_cast<uint32_t>(nkb);
-    // The bf16 result.  A quad whose 32 rows are all valid goes out by TMA:
-    // each 32-column half of the warp's columns is staged in the warp's
-    // buffer (lane = row, 64-byte rows, 16-byte chunk c of row l at chunk
-    // c ^ ((l >> 1) & 3): the 64-byte swizzle, so the eight lanes of each
-    // store phase hit eight distinct bank groups) and stored as one box.
-    // Rows of a partly valid quad (the last tile of a ragged M, a masked
-    // expert's last tile) are stored by their lanes, so rows past the valid
-    // ones are never written.
-    const int quad_rows = tile.rows - quad * 32;
-    if (col_ok && quad_rows >= 32) {
-#pragma unroll
-      for (int h = 0; h < kCols / static_cast<int>(L::kOutBoxCols); ++h) {
-        if (out_pending) {
-          if (lane == 0) bulk_wait_group_read0();  // the buffer's last box has been read
-          __syncwarp();
-        }
-        const uint32_t row_addr = out_buf + static_cast<uint32_t>(lane) * (L::kOutBoxCols * 2);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int p0 = h * 16 + 4 * c;
-          const uint4 o = make_uint4(bf16x2_from_pair(acc[p0]), bf16x2_from_pair(acc[p0 + 1]),
-                                     bf16x2_from_pair(acc[p0 + 2]), bf16x2_from_pair(acc[p0 + 3]));
-          sts_v4(row_addr + ((static_cast<uint32_t>(c) ^ ((lane >> 1) & 3u)) << 4), o);
-        }
-        fence_proxy_async_shared();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(tma_c, out_buf, col0 + h * static_cast<int>(L::kOutBoxCols), tile.a_row + quad * 32);
-          bulk_commit_group();
-        }
-        out_pending = true;
-      }
-    } else if (row_ok && col_ok) {
+    // The bf16 result: each lane stores its row's columns (rows past the
+    // valid ones are never written).
+    if (row_ok && col_ok) {
       __nv_bfloat16* crow = args.c + static_cast<int64_t>(tile.a_row + r) * args.N + col0;
 #pragma unroll
       for (int c = 0; c < kCols; c += 8) {
@@ -609,10 +559,13 @@ __device__ __forceinline__ uint32_t epilogue(const CUtensorMap* tma_c, uint32_t 
       }
     }
   }
-  // every box this warp stored is complete before the CTA can exit
-  if (lane == 0) bulk_wait_group0();
+  // where this warp stopped, for the producers' abort path
+  if (lane == 0) {
+    epi.pos[warp - 4] = static_cast<uint32_t>(stage) + STAGES * phase;
+    __threadfence_block();
+    atomicAdd(const_cast<int*>(epi.done), 1);
+  }
   __syncwarp();
-  return released;
 }
 
 
@@ -621,7 +574,7 @@ template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                             const __grid_constant__ CUtensorMap tma_sa, const __grid_constant__ CUtensorMap tma_sb,
-                            const __grid_constant__ CUtensorMap tma_c, const GemmArgs args) {
+                            const GemmArgs args) {
   using L = GemmSmem<BN, STAGES, k1D1D>;
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "UMMA N for M=128 must be a multiple of 16 in [16,256]");
 
@@ -633,7 +586,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
   int32_t* total_slot = reinterpret_cast<int32_t*>(smem + L::kOffMisc + 8);
   const EpiRecord epi{reinterpret_cast<volatile int*>(smem + L::kOffMisc + 12),
-                      reinterpret_cast<volatile uint32_t*>(smem + L::kOffMisc + 16)};
+                      reinterpret_cast<volatile uint32_t*>(smem + L::kOffMisc + 16)};  // 8 positions
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + L::kOffPrefix);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -656,7 +609,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_barrier_init();
     tma_prefetch_map(&tma_a);
     tma_prefetch_map(&tma_b);
-    tma_prefetch_map(&tma_c);
     if constexpr (kTmaScales) {
       tma_prefetch_map(&tma_sa);
       tma_prefetch_map(&tma_sb);
@@ -696,16 +648,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // all TMEM slab buffers start free: every lane releases them for the first slabs
     if (promote)
       for (int b = 0; b < L::kAccBufs; ++b) mbar_arrive(bars.full(b));
-    const uint32_t released =
-        epilogue<BN, STAGES, S, kPromote, kTmaScales, k1D1D>(&tma_c, s_base, args, prefix, bars, wc, total, tmem_base,
-                                                             warp, lane);
-    // publish this warp's release count for the producers' abort path
-    __syncwarp();
-    if (lane == 0) {
-      epi.rel[warp - 4] = (promote ? static_cast<uint32_t>(L::kAccBufs) : 0u) + released;
-      __threadfence_block();
-      atomicAdd(const_cast<int*>(epi.done), 1);
-    }
+    epilogue<BN, STAGES, S, kPromote, kTmaScales, k1D1D>(s_base, args, epi, prefix, bars, wc, total, tmem_base,
+                                                         warp, lane);
   }
 
   __syncwarp();

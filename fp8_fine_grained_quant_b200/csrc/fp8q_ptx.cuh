@@ -154,27 +154,11 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// 2-D tiled bulk copy shared -> global (no multicast): the box at (x, y) of
-// the map's tensor, rows and columns past the tensor's extent not written.
-// Completes as part of this thread's current bulk async-group.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(src), "r"(x), "r"(y)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Waits until this thread's committed bulk stores have finished reading shared memory.
-__device__ __forceinline__ void bulk_wait_group_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// Waits until this thread's committed bulk stores are complete.
-__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// Orders this thread's generic-proxy shared-memory writes before later
-// async-proxy (TMA) reads of them.
-__device__ __forceinline__ void fence_proxy_async_shared() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+// Untiled bulk copy global -> shared of `bytes` (a multiple of 16; both
+// addresses 16-byte aligned), completing on `bar` (tx bytes).  No multicast.
+__device__ __forceinline__ void bulk_load_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
                : "memory");
 }
 
@@ -225,6 +209,50 @@ __device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// Shared-memory matrix descriptor, K-major without swizzle: 8-row core
+// matrices of 16-byte rows stored contiguously (128 bytes), consecutive core
+// matrices along M/N `sbo` bytes apart.  Fields as smem_desc_k_sw128, layout
+// type 0 (no swizzle); the leading byte offset is unused for one 16-byte
+// column.
+__device__ __forceinline__ uint64_t smem_desc_k_none(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(sbo >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Instruction descriptor of tcgen05.mma.kind::mxf8f6f4.block_scale, E4M3 x
+// E4M3 -> F32, both operands K-major, UE8M0 scale factors: B scale-factor id
+// (bits 4-5), A/B formats (7-9, 10-12) = 0 (E4M3), N >> 3 (17-22), scale
+// format (23) = 1 (E8M0), M >> 4 (24-28), A scale-factor id (29-30).  The ids
+// pick the byte of each 32-bit scale-factor column that this K = 32 step uses.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int m, int n, uint32_t sfa_id, uint32_t sfb_id) {
+  return (sfb_id << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(m >> 4) << 24) | (sfa_id << 29);
+}
+
+// D[tmem] (+)= (A * SFA)[smem] * (B * SFB)[smem]^T for one K = 32 step: each
+// row's 32-element block of A and of B scaled by 2^(sf - 127) in the tensor
+// core.  sfa/sfb: TMEM addresses of the scale-factor columns (the byte this
+// step uses also in bits 30-31, as the instruction descriptor's ids).
+__device__ __forceinline__ void mma_mx_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+      : "memory");
+}
+
+// Shared -> TMEM copy of 32 rows x 128 bits (rows 16 bytes apart, described
+// by `sdesc`) into 32 lanes x 4 columns at `taddr`, replicated into all four
+// 32-lane quarters.  Executes in order with this thread's tcgen05.mma.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Arrives once on `bar` when every previously issued tcgen05.mma of this

@@ -266,3 +266,31 @@ def test_quant_act_128x1_t_validation(args, expect):
 ])
 def test_wgrad_validation(nkm, ptrs, expect):
     assert _call("fp8_gemm_wgrad", *ptrs, *nkm, None) == expect
+
+
+@pytest.mark.parametrize("name,args,expect", [
+    ("fp8_mx_scales_act", (A16, 4, 100, A16, None), fq.ERR_SHAPE),
+    ("fp8_mx_scales_act", (A16, 0, 128, A16, None), fq.OK),
+    ("fp8_mx_scales_act", (None, 4, 128, A16, None), fq.ERR_NULL),
+    ("fp8_mx_scales_act", (A16, 4, 128, A4, None), fq.ERR_ALIGN),
+    ("fp8_mx_scales_w", (A16, 1, 100, 128, A16, None), fq.ERR_SHAPE),
+    ("fp8_mx_scales_w", (A16, 1, 128, 128, A1, None), fq.ERR_ALIGN),
+    ("fp8_gemm_mx", (A16, A16, A16, A16, A16, 128, 256, 100, None), fq.ERR_SHAPE),
+    ("fp8_gemm_mx", (A16, A16, A16, A16, A16, 0, 256, 128, None), fq.OK),
+    ("fp8_gemm_mx", (A16, None, A16, A16, A16, 128, 256, 128, None), fq.ERR_NULL),
+    ("fp8_gemm_mx", (A16, A4, A16, A16, A16, 128, 256, 128, None), fq.ERR_ALIGN),   # bulk-copied atoms
+])
+def test_mx_validation(name, args, expect):
+    assert _call(name, *args) == expect
+
+
+@pytest.mark.parametrize("name,args,expect", [
+    ("fp8_grouped_gemm_mx_contiguous", (A16, A16, A16, A16, A16, A16, 200, 256, 128, 4, None), fq.ERR_SHAPE),
+    ("fp8_grouped_gemm_mx_contiguous", (A16, A16, A16, A16, None, A16, 256, 256, 128, 4, None), fq.ERR_NULL),
+    ("fp8_grouped_gemm_mx_contiguous", (A16, A4, A16, A16, A16, A16, 256, 256, 128, 4, None), fq.ERR_ALIGN),
+    ("fp8_grouped_gemm_mx_masked", (A16, A16, A16, A16, A16, A16, 4, 200, 256, 128, None), fq.ERR_SHAPE),
+    ("fp8_grouped_gemm_mx_masked", (A16, A16, A16, A16, A16, A16, 0, 128, 256, 128, None), fq.OK),
+    ("fp8_grouped_gemm_mx_masked", (A16, A16, A16, A16, A1, A16, 4, 128, 256, 128, None), fq.ERR_ALIGN),
+])
+def test_grouped_mx_validation(name, args, expect):
+    assert _call(name, *args) == expect

@@ -302,7 +302,19 @@ def simulate_abort(tiles, nkb, abort_at, stages=6, acc=4, warps=8, lanes=32, pro
             phase = js // stages
             complete = full[s].done >= phase + 1
             if not complete and fixup:
-                missing = lanes * sum(1 for w in range(warps) if released[w] <= js)
+                # the kernel's rule: each warp publishes je mod 2*stages (je = the
+                # next slab it had not read) and the stage's pending slab is known
+                # mod 2*stages; the release is missing when (js - je) mod 2*stages >= acc
+                js_mod = (s + stages * ((js // stages) % 2)) % (2 * stages)
+                assert js_mod == js % (2 * stages)
+                missing = 0
+                for w in range(warps):
+                    je = released[w] - acc
+                    assert 0 <= js - je < stages + acc, (js, je)   # the window the rule relies on
+                    d = (js_mod - je % (2 * stages)) % (2 * stages)
+                    assert (d >= acc) == (released[w] <= js)
+                    if d >= acc:
+                        missing += lanes
                 if missing:
                     full[s].arrive(missing)
     while inflight_tma:

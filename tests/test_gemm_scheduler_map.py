@@ -4,8 +4,7 @@ The GEMM kernel (fp8q_gemm.cuh) walks tiles t = blockIdx.x, +gridDim.x, ...
 below a total, maps each t to a tile with get_tile (dense, MoE contiguous,
 MoE masked), and its eight epilogue warps each own one TMEM lane quarter
 (32 rows) and one half of the tile's columns, storing only rows below the
-tile's valid count and columns below N: a quad whose 32 rows are all valid
-goes out as two 32 x 32 TMA boxes, a partly valid one row by row.  For the masked form one warp first
+tile's valid count and columns below N.  For the masked form one warp first
 builds the per-expert prefix of tile counts with a chunked warp scan.
 
 These tests restate that arithmetic (and the launcher's grid choice in
@@ -125,21 +124,8 @@ def replay(kind, *, M, N, K, E=1, m_indices=None, masked_m=None, num_sms=148):
                     row_ok = r < rows
                     sa_row = a_row + (r if row_ok else 0)
                     assert 0 <= sa_row < a_rows                 # sa is [a_rows, nkb]
-                if col_ok and rows - quad * 32 >= 32:
-                    # a full quad: two 32 x 32 TMA store boxes, which must lie
-                    # inside the output map ([a_rows, N]) with a 16-byte-aligned
-                    # column start and no negative coordinate
-                    for h in range(2):
-                        x, y = col0 + 32 * h, a_row + quad * 32
-                        assert x >= 0 and y >= 0 and (x * 2) % 16 == 0
-                        assert x + 32 <= N and y + 32 <= a_rows
-                        writes[y:y + 32, x:x + 32] += 1
-                elif col_ok:
-                    # a partly valid quad: each lane stores its own row if valid
-                    for lane in range(32):
-                        r = quad * 32 + lane
-                        if r < rows:
-                            writes[a_row + r, col0:col0 + BN // 2] += 1
+                    if row_ok and col_ok:
+                        writes[a_row + r, col0:col0 + BN // 2] += 1
     return writes
 
 

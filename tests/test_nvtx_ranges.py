@@ -43,6 +43,11 @@ calls = [
     ("fp8_swiglu_quant_1x128", (A16, 4, 100, None, 0, A16, A16, None)),
     ("fp8_quant_act_128x1_t", (A16, 4, 100, 128, A16, A16, None)),
     ("fp8_gemm_wgrad", (A16, A16, A16, A16, A16, 256, 256, 0, None)),
+    ("fp8_mx_scales_act", (A16, 4, 100, A16, None)),
+    ("fp8_mx_scales_w", (None, 1, 128, 128, A16, None)),
+    ("fp8_gemm_mx", (A16, A16, A16, A16, A16, 0, 256, 128, None)),
+    ("fp8_grouped_gemm_mx_contiguous", (A16, A16, A16, A16, A1, A16, 256, 256, 128, 4, None)),
+    ("fp8_grouped_gemm_mx_masked", (A16, A16, A16, A16, A16, A16, 4, 200, 256, 128, None)),
 ]
 out = []
 lib = fq.lib()
@@ -72,7 +77,7 @@ def test_every_entry_point_pushes_and_pops_one_named_range(recorder):
     res = subprocess.run([sys.executable, "-c", CHILD, str(ROOT), str(recorder)], env=env,
                          capture_output=True, text=True, timeout=300, check=True)
     rows = json.loads(res.stdout.strip().splitlines()[-1])
-    assert len(rows) == 14
+    assert len(rows) == 19
     for r in rows:
         assert r["rc"] in (fq.OK, fq.ERR_SHAPE, fq.ERR_NULL, fq.ERR_ALIGN), r
         assert r["log"] == "push %s\npop\n" % r["name"], r
