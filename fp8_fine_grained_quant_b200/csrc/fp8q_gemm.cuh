@@ -206,6 +206,12 @@ __device__ __forceinline__ bool get_tile(const GemmArgs& a, const int32_t* prefi
 // by then every epilogue warp has read the scales of slabs <= 4g + 5.  The
 // epilogue reads a slab's scales after observing that slab's MMAs complete,
 // and those MMAs were issued after full[] of slab 4g (the copies landed).
+// Visibility of those bytes to the epilogue threads follows one causality
+// chain: the copies' complete-tx on full[] releases the async proxy's writes,
+// the MMA thread's wait on full[] acquires them, its tcgen05.commit arrives on
+// empty[] after that wait in program order (an arrive-on with release
+// semantics at CTA scope), and the epilogue's wait on empty[] acquires.  The
+// epilogue never waits on full[] itself.
 //
 // Each waiting role costs its thread ~150 cycles per barrier probe, and an MMA
 // instruction is accepted only as the tensor pipe frees up, so the TMA and MMA

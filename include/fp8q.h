@@ -262,42 +262,10 @@ FP8Q_API int fp8_gemm_wgrad(const uint8_t* q_dy_t, const float* s_dy, const uint
  * cores, no CUDA-core promotion.  The scales go in as E8M0 atoms:
  *   fp8_mx_scales_act: sa [M, K/128] f32 -> sfa_mx [ceil(M/128), K/128, 512] bytes
  *   fp8_mx_scales_w  : sb [G, N/128, K/128] f32 -> sfb_mx [G*N/128, K/128, 512] bytes
- * (atom byte 16*m0 + 4*m1 + j = E8M0 of row 32*m1 + m0 of the 128-row tile,
- * K block j; a scale that is not a power of two is truncated to one).
- *   qa : [M, K] E4M3, qb : [N, K] E4M3, c_bf16 : [M, N] bf16.
- * N, K multiples of 128; any M >= 0.  sfa_mx, sfb_mx and every code/output
- * pointer 16-byte aligned; sa, sb 4-byte aligned.
- */
-FP8Q_API int fp8_mx_scales_act(const float* sa, int64_t M, int64_t K, uint8_t* sfa_mx, cudaStream_t stream);
-FP8Q_API int fp8_mx_scales_w(const float* sb, int64_t G, int64_t N, int64_t K, uint8_t* sfb_mx, cudaStream_t stream);
-FP8Q_API int fp8_gemm_mx(const uint8_t* qa, const uint8_t* sfa_mx, const uint8_t* qb, const uint8_t* sfb_mx,
-                         void* c_bf16, int64_t M, int64_t N, int64_t K, cudaStream_t stream);
-
-/*
- * The two MoE layouts of fp8_gemm_mx, with the arguments and semantics of
- * fp8_grouped_gemm_contiguous / fp8_grouped_gemm_masked: sfa_mx holds the
- * atoms of qa's 128-row blocks (fp8_mx_scales_act of its [M_tot or E*cap,
- * K/128] scales), sfb_mx those of qb [E, N, K] (fp8_mx_scales_w with G = E).
- */
-FP8Q_API int fp8_grouped_gemm_mx_contiguous(const uint8_t* qa, const uint8_t* sfa_mx, const uint8_t* qb,
-                                            const uint8_t* sfb_mx, const int32_t* m_indices, void* c_bf16,
-                                            int64_t M_tot, int64_t N, int64_t K, int64_t E, cudaStream_t stream);
-FP8Q_API int fp8_grouped_gemm_mx_masked(const uint8_t* qa, const uint8_t* sfa_mx, const uint8_t* qb,
-                                        const uint8_t* sfb_mx, const int32_t* masked_m, void* c_bf16, int64_t E,
-                                        int64_t cap, int64_t N, int64_t K, cudaStream_t stream);
-
-/*
- * Block-scaled FP8 GEMM with power-of-two (UE8M0) scales applied by the
- * tensor cores ("The Insider Secrets Of Deepseek Discovered", FP8 passage:
- * the microscaling form Blackwell's tensor cores support):
- *   C[m,n] = bf16_rne( sum_kb sa[m,kb] * sb[n/128,kb] * sum_{k in slab kb} A[m,k] * B[n,k] )
- * with every sa, sb a power of two (fp8_quant_act_1x128_ue8m0,
- * fp8_quant_w_128x128_ue8m0), the whole K accumulated in FP32 in the tensor
- * cores, no CUDA-core promotion.  The scales go in as E8M0 atoms:
- *   fp8_mx_scales_act: sa [M, K/128] f32 -> sfa_mx [ceil(M/128), K/128, 512] bytes
- *   fp8_mx_scales_w  : sb [G, N/128, K/128] f32 -> sfb_mx [G*N/128, K/128, 512] bytes
- * (atom byte 16*m0 + 4*m1 + j = E8M0 of row 32*m1 + m0 of the 128-row tile,
- * K block j; a scale that is not a power of two is truncated to one).
+ * (one 512-byte atom per 128-row tile and 128-deep K slab: byte
+ * 16*m0 + 4*m1 + j = E8M0 of row 32*m1 + m0 of the tile for the slab's
+ * 32-element K block j, the four j equal; a normal scale that is not a
+ * power of two is truncated to the power of two below it).
  *   qa : [M, K] E4M3, qb : [N, K] E4M3, c_bf16 : [M, N] bf16.
  * N, K multiples of 128; any M >= 0.  sfa_mx, sfb_mx and every code/output
  * pointer 16-byte aligned; sa, sb 4-byte aligned.
