@@ -22,8 +22,11 @@
 namespace fp8q {
 
 __device__ uint32_t g_device_status;
-// Where fp8q_get_device_error's exchange kernel leaves the word it took.
-__device__ uint32_t g_device_status_taken;
+// Where fp8q_get_device_error's exchange kernel leaves the word it took: one
+// slot per query, taken round-robin, so queries that overlap on different
+// streams do not read each other's result.
+constexpr int kTakeSlots = 64;
+__device__ uint32_t g_device_status_taken[kTakeSlots];
 
 namespace {
 
@@ -32,6 +35,7 @@ constexpr int kMaxDevices = 64;
 
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<uint64_t> g_launches{0};
+std::atomic<uint32_t> g_take_slot{0};
 
 struct DeviceInfo {
   // set (release) once every other field is final; read (acquire) without the lock
@@ -39,6 +43,7 @@ struct DeviceInfo {
   bool supported = false;
   int num_sms = 0;
   uint32_t* status = nullptr;  // device address of g_device_status
+  bool wide_ok = false;        // the wide-tile instances were built with the register count their split needs
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -52,10 +57,26 @@ cudaError_t opt_in_smem() {
                               GemmSmem<BN, STAGES, k1D1D>::kDynamicBytes);
 }
 
+// Whether an instance that splits registers between its warpgroups was
+// built with the launch count the split assumes (a split larger than the
+// launch's allocation would never be granted).
+template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D = false>
+bool split_regs_ok() {
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, gemm_blockscaled_kernel<BN, STAGES, S, kPromote, kTmaScales, k1D1D>) != cudaSuccess)
+    return false;
+  return static_cast<uint32_t>(fa.numRegs) * kGemmThreads >= 128 * kCtlRegs + 256 * kEpiRegs;
+}
+
 // Output tile 128 x kTileN: 64 FP32 accumulators per epilogue thread, four
 // TMEM slab buffers, six 32 KB pipeline stages.
 constexpr int kTileN = 128;
 constexpr int kStages128 = 6;
+// Wide output tile 128 x 256: 128 FP32 accumulators per epilogue thread
+// (registers split between the warpgroups), two TMEM slab buffers of 256
+// columns, four 48 KB stages.  Each A slab loaded serves twice the columns.
+constexpr int kTileWide = 256;
+constexpr int kStagesWide = 4;
 
 int device_info(DeviceInfo** out) {
   int dev = 0;
@@ -83,6 +104,12 @@ int device_info(DeviceInfo** out) {
         if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kMasked, true, true>();
         if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kMasked, true, false>();
         if (e == cudaSuccess) e = opt_in_smem<kTileN, kStages128, Sched::kDense, true, true, true>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileWide, kStagesWide, Sched::kDense, true, true>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileWide, kStagesWide, Sched::kContiguous, true, true>();
+        if (e == cudaSuccess) e = opt_in_smem<kTileWide, kStagesWide, Sched::kMasked, true, true>();
+        d.wide_ok = split_regs_ok<kTileWide, kStagesWide, Sched::kDense, true, true>() &&
+                    split_regs_ok<kTileWide, kStagesWide, Sched::kContiguous, true, true>() &&
+                    split_regs_ok<kTileWide, kStagesWide, Sched::kMasked, true, true>();
         if (e == cudaSuccess)
           e = cudaFuncSetAttribute(gemm_mx_kernel<Sched::kDense>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    MxSmem::kDynamicBytes);
@@ -223,7 +250,8 @@ int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
     const uint64_t nkb = static_cast<uint64_t>(g.K / kSlabK);
     rc = make_scale_map(&msa, g.sa, static_cast<uint64_t>(g.a_rows), nkb, kBlockM);
     if (rc) return rc;
-    rc = make_scale_map(&msb, g.sb, static_cast<uint64_t>(g.E * (g.N / 128)), nkb, 1);
+    rc = make_scale_map(&msb, g.sb, static_cast<uint64_t>(g.E * (g.N / 128)), nkb,
+                        GemmSmem<BN, STAGES, k1D1D>::kSbBlocks);
     if (rc) return rc;
   }
   GemmArgs a;
@@ -247,6 +275,23 @@ int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
   return launch_instance<BN, STAGES, S, kPromote, kTmaScales, k1D1D>(ma, mb, msa, msb, a, grid, stream);
 }
 
+// Tile width.  Wide tiles need N to be a multiple of 256 (no half-empty tile
+// column).  A wide tile does the work of two 128-column tiles in about 0.95
+// of their time, but there are half as many, so the last partial round of
+// tiles over the SMs can cost more than that gains: for the dense and
+// contiguous layouts (tile count known on the host) wide tiles are taken
+// only when 2 x 0.95 x (rounds of wide tiles) <= rounds of 128-column tiles.
+// The masked layout's tile count is known on the device only; it takes wide
+// tiles whenever N allows.
+template <Sched S>
+bool use_wide_tiles(const GemmCall& g, int64_t sms) {
+  if (g.N % kTileWide != 0) return false;
+  if constexpr (S == Sched::kMasked) return true;
+  const int64_t narrow = g.m_tiles * (g.N / kTileN), wide = g.m_tiles * (g.N / kTileWide);
+  const int64_t r_narrow = (narrow + sms - 1) / sms, r_wide = (wide + sms - 1) / sms;
+  return 19 * r_wide <= 10 * r_narrow;
+}
+
 template <Sched S>
 int run_gemm(const GemmCall& g, cudaStream_t stream) {
   DeviceInfo* dev = nullptr;
@@ -255,8 +300,11 @@ int run_gemm(const GemmCall& g, cudaStream_t stream) {
   if (g.promote) {
     // scales staged by TMA with the operands when their rows are 16-byte
     // multiples (K % 512 == 0) and both scale tensors are 16-byte aligned
-    if ((g.K / kSlabK) % 4 == 0 && aligned(g.sa, 16) && aligned(g.sb, 16))
+    if ((g.K / kSlabK) % 4 == 0 && aligned(g.sa, 16) && aligned(g.sb, 16)) {
+      if (dev->wide_ok && use_wide_tiles<S>(g, dev->num_sms))
+        return launch_gemm<kTileWide, kStagesWide, S, true, true>(g, *dev, stream);
       return launch_gemm<kTileN, kStages128, S, true, true>(g, *dev, stream);
+    }
     return launch_gemm<kTileN, kStages128, S, true, false>(g, *dev, stream);
   }
   // only the dense form has the unpromoted (accumulation diagnostic) build
@@ -718,6 +766,7 @@ int fp8q_get_device_error(cudaStream_t stream) {
   uint32_t* taken = nullptr;
   if (cudaGetSymbolAddress(reinterpret_cast<void**>(&taken), g_device_status_taken) != cudaSuccess)
     return FP8Q_ERR_CUDA;
+  taken += g_take_slot.fetch_add(1) % kTakeSlots;
   status_take_kernel<<<1, 1, 0, stream>>>(dev->status, taken);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   uint32_t v = 0;

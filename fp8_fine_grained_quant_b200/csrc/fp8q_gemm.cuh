@@ -46,6 +46,14 @@ enum class Sched : int { kDense = 0, kContiguous = 1, kMasked = 2 };
 constexpr int kBlockM = 128;
 constexpr int kSlabK = 128;  // promotion interval = scale slab
 constexpr int kGemmThreads = 384;  // warpgroup 0: TMA + MMA (+ scheduler set-up); 1-2: epilogue
+// Register split of the wide-tile (BN = 256) instances: launched at
+// kLaunchRegs per thread (the most __launch_bounds__(384, 1) allows), the
+// control warpgroup drops to kCtlRegs and the epilogue warpgroups rise to
+// kEpiRegs.  The host checks the launch count before the first launch.
+constexpr uint32_t kLaunchRegs = 168;
+constexpr uint32_t kCtlRegs = 56;
+constexpr uint32_t kEpiRegs = 224;
+static_assert(128 * kCtlRegs + 256 * kEpiRegs <= kGemmThreads * kLaunchRegs, "register split exceeds the launch");
 constexpr int kMaxMaskedExperts = 1024;
 
 
@@ -99,7 +107,9 @@ struct GemmSmem {
   static constexpr int kScaleGroup = 4;
   static constexpr int kScaleSlots = 4;
   static constexpr uint32_t kSaSlotBytes = kBlockM * kScaleGroup * 4;  // 2 KB
-  static constexpr uint32_t kSbSlotBytes = k1D1D ? BN * kScaleGroup * 4 : kScaleGroup * 4;
+  // (block scales: one row of kScaleGroup per 128-column weight block the tile spans)
+  static constexpr uint32_t kSbBlocks = BN >= 128 ? BN / 128 : 1;
+  static constexpr uint32_t kSbSlotBytes = k1D1D ? BN * kScaleGroup * 4 : kSbBlocks * kScaleGroup * 4;
   static constexpr uint32_t kSbSlotStride = k1D1D ? kSbSlotBytes : 128;  // TMA destinations 128-byte aligned
   // the masked layout's tile prefix (the weight-gradient instance is dense-only and has none)
   static constexpr uint32_t kPrefixBytes = k1D1D ? 0u : 4u * (kMaxMaskedExperts + 1);
@@ -464,7 +474,8 @@ __device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, 
       uint64_t scale2;
       // Warp-uniform outcome: the tcgen05.ld below must be executed by all 32 lanes.
       if (!ready) {
-        const bool got = promote ? mbar_wait(bars.empty(stage), phase, wc, 4) : mbar_wait(bars.tfull(buf), tphase, wc, 4);
+        const bool got = promote ? mbar_wait_inl(bars.empty(stage), phase, wc, 4)
+                                 : mbar_wait_inl(bars.tfull(buf), tphase, wc, 4);
         if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
       }
       float sa_smem = 0.0f, sb_smem = 0.0f;
@@ -478,7 +489,8 @@ __device__ __forceinline__ void epilogue(uint32_t s_base, const GemmArgs& args, 
           sb_cols = s_base + L::kOffSb + slot * L::kSbSlotStride + k * (BN * 4) + half * (kCols * 4);
         } else {
           sa_smem = lds_f32(s_base + L::kOffSa + slot * L::kSaSlotBytes + r * (L::kScaleGroup * 4) + k * 4);
-          sb_smem = lds_f32(s_base + L::kOffSb + slot * L::kSbSlotStride + k * 4);
+          sb_smem = lds_f32(s_base + L::kOffSb + slot * L::kSbSlotStride +
+                            ((half * kCols) / 128) * (L::kScaleGroup * 4) + k * 4);
         }
         if (k == L::kScaleGroup - 1) ++group;
       }
@@ -639,7 +651,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int32_t total = *total_slot;
 
+  // Wide tiles hold 128 FP32 sums per epilogue thread: the control
+  // warpgroup hands registers to the two epilogue warpgroups
+  // (128 x kCtlRegs + 256 x kEpiRegs = 384 x kLaunchRegs).  Each role then
+  // finishes on its own path, and the epilogue calls no out-of-line function.
+  constexpr bool kSplitRegs = BN > 128;
   if (warp < 4) {
+    if constexpr (kSplitRegs) setmaxnreg_dec<kCtlRegs>();
     // warps 0 and 3: TMA producers; warps 1 and 2: MMA issuers (one issuer
     // when a tile accumulates in a single buffer)
     const uint32_t n_mma = promote ? 2u : 1u;
@@ -650,20 +668,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       else if (static_cast<uint32_t>(warp - 1) < n_mma)
         issue_mma<BN, STAGES, S, kPromote>(args, prefix, s_base, bars, wc, total, tmem_base, warp - 1, n_mma);
     }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem_base, L::kTmemCols);
+    }
   } else {
+    if constexpr (kSplitRegs) setmaxnreg_inc<kEpiRegs>();
     // all TMEM slab buffers start free: every lane releases them for the first slabs
     if (promote)
       for (int b = 0; b < L::kAccBufs; ++b) mbar_arrive(bars.full(b));
     epilogue<BN, STAGES, S, kPromote, kTmaScales, k1D1D>(s_base, args, epi, prefix, bars, wc, total, tmem_base,
                                                          warp, lane);
-  }
-
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, L::kTmemCols);
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
   }
 }
 

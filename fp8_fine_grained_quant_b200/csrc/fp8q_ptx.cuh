@@ -120,6 +120,36 @@ __device__ __noinline__ bool mbar_drain(uint32_t bar, uint32_t parity, uint32_t*
   return true;
 }
 
+// mbar_wait with its slow loop inlined.  For code that runs with more
+// registers than the kernel was launched with (after setmaxnreg.inc): ptxas
+// cannot allocate such a region if it calls an out-of-line function.
+__device__ __forceinline__ bool mbar_wait_inl(uint32_t bar, uint32_t parity, const WaitCtl& w, uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    for (int i = 0; i < 128; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*w.abort) return false;
+    if (globaltimer_ns() - t0 > w.timeout_ns) {
+      atomicCAS(w.status, 0u, kDevErrTimeout | site);
+      *w.abort = 1;
+      return false;
+    }
+  }
+}
+
+// Register split between warpgroups (every warp of a warpgroup executes the
+// same one): dec hands registers back to the CTA's pool, inc waits until the
+// pool has them.  The counts must add up to at most the launch's allocation.
+template <uint32_t R>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+
 // Waits until the phase with the given parity has completed.  Returns false
 // (after recording a timeout) if it does not within the limit.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& w, uint32_t site) {

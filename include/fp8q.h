@@ -311,8 +311,10 @@ FP8Q_API const char* fp8q_status_string(int status);
  * The word is one per device, shared by every stream and every call of the
  * library on that device: a timeout is not attributed to a call or a stream,
  * and a call still running on another stream may record one after the
- * exchange (it is then reported by the next query).  A timeout also covers a
- * kernel's final drain running out of its fixed bound (2 s) after an abort.
+ * exchange (it is then reported by the next query).  Queries that overlap
+ * on different streams each get the value their own exchange took (up to 64
+ * queries in flight at once).  A timeout also covers a kernel's final drain
+ * running out of its fixed bound (2 s) after an abort.
  */
 FP8Q_API int fp8q_get_device_error(cudaStream_t stream);
 

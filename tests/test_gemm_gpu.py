@@ -113,13 +113,14 @@ def test_dense_workloads_sampled(dev, name):
 
 
 @pytest.mark.parametrize("M,N,K", [
-    (1024, 5120, 512),   # 320 tiles: one scale group per tile, the scale ring's slot moves on every tile
-    (2048, 2560, 2048),  # 320 tiles, four scale groups per tile
-    (1000, 4864, 1664),  # 304 tiles, ragged M; K % 512 != 0: scales loaded from global memory
+    (1024, 9472, 512),   # 296 wide (128 x 256) tiles: one scale group per tile, the ring's slot moves every tile
+    (2048, 4608, 2048),  # 288 wide tiles, four scale groups per tile
+    (1024, 4992, 512),   # N/128 odd: 312 128 x 128 tiles on the staged-scale path
+    (1000, 4864, 1664),  # 304 128 x 128 tiles, ragged M; K % 512 != 0: scales loaded from global memory
 ])
 def test_dense_many_tiles_full(dev, M, N, K):
-    """More than two tiles per SM, every element compared: each CTA's second
-    and later tiles, in every epilogue warp."""
+    """About two or more tiles per SM, every element compared: each CTA's
+    second and later tiles, in every epilogue warp, for both tile widths."""
     rng = np.random.default_rng(M + 5 * N + 11 * K)
     a = rng.standard_normal((M, K)).astype(np.float32) * np.exp(rng.standard_normal(K)).astype(np.float32)
     b = (0.02 * rng.standard_normal((N, K))).astype(np.float32)
@@ -171,11 +172,12 @@ def test_contiguous_small(dev):
     _contiguous_case(dev, wl.moe_contiguous(tokens=96, topk=4, E=6, N=384, K=512, seed=21), all_rows=True)
 
 
-@pytest.mark.parametrize("K", [512, 2048])
-def test_contiguous_many_tiles_full(dev, K):
-    """Over 300 tiles of mixed experts, every element compared."""
-    d = wl.moe_contiguous(tokens=512, topk=6, E=8, N=2560, K=K, seed=40 + K)
-    assert (d.M_tot // TILE) * (d.N // TILE) > 2 * 148
+@pytest.mark.parametrize("N,K,tile_n", [(5120, 512, 256), (5120, 2048, 256), (2432, 512, 128)])
+def test_contiguous_many_tiles_full(dev, N, K, tile_n):
+    """Over 2 x 148 tiles of mixed experts, every element compared; 128 x 256
+    tiles when N is a multiple of 256 (staged scales), else 128 x 128."""
+    d = wl.moe_contiguous(tokens=512, topk=6, E=8, N=N, K=K, seed=40 + K + N)
+    assert (d.M_tot // TILE) * (d.N // tile_n) > 2 * 148
     _contiguous_case(dev, d, all_rows=True)
 
 
@@ -254,14 +256,15 @@ def test_masked_out_of_range_counts_clamped(dev):
     _masked_case(dev, a, b, [-4, 500, 77])
 
 
-def test_masked_many_tiles_full(dev):
-    """Over 300 tiles (counts spanning 0..cap), every valid element compared
-    and every other row checked untouched."""
-    rng = np.random.default_rng(34)
-    E, cap, N, K = 12, 256, 2560, 1024
+@pytest.mark.parametrize("N,tile_n", [(5120, 256), (2432, 128)])
+def test_masked_many_tiles_full(dev, N, tile_n):
+    """Over 2 x 148 tiles (counts spanning 0..cap), every valid element
+    compared and every other row checked untouched; both tile widths."""
+    rng = np.random.default_rng(34 + N)
+    E, cap, K = 12, 256, 1024
     masked_m = rng.integers(0, cap, size=E, endpoint=True)
     masked_m[:3] = [cap, 129, 0]
-    tiles = sum((int(m) + TILE - 1) // TILE for m in masked_m) * (N // TILE)
+    tiles = sum((int(m) + TILE - 1) // TILE for m in masked_m) * (N // tile_n)
     assert tiles > 2 * 148
     a = wl.bf16_bits(rng.standard_normal((E, cap, K)).astype(np.float32))
     b = wl.bf16_bits((0.02 * rng.standard_normal((E, N, K))).astype(np.float32))

@@ -62,7 +62,7 @@ def test_gemm_mx_matches_oracle(dev, M, N, K):
 
 def test_gemm_mx_full_size_sampled_rows(dev):
     d = wl.dense_fprop()
-    rows = sorted({r for t in range(d.M // TILE) for r in (t * TILE, t * TILE + 77)})
+    rows = wl.quad_rows(np.random.default_rng(12), d.M).tolist()
     got, ref, _ = _mx_case(dev, d.a, d.b, rows=rows)
     assert_gemm_close(got, ref, "gemm_mx dense_fprop, %d rows" % len(rows))
 

@@ -349,3 +349,22 @@ def test_abort_fixup_counts_are_needed():
             hit = True
             break
     assert hit
+
+
+# ------------------------------------------------------------- wide tiles
+# The 128 x 256 instances run four 48 KB stages and two 256-column TMEM slab
+# buffers; the same protocol with those counts.
+
+@pytest.mark.parametrize("seed", range(8))
+def test_wide_tile_configuration(seed):
+    assert _slots_needed(4, 2) <= 4
+    simulate(tiles=3, nkb=8, stages=4, acc=2, seed=1100 + seed)
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_wide_tile_abort_path(seed):
+    rng = random.Random(seed)
+    nkb = rng.choice([4, 8, 13])
+    tiles = rng.choice([2, 3])
+    simulate_abort(tiles=tiles, nkb=nkb, abort_at=rng.randrange(1, 40 * tiles * nkb), stages=4, acc=2,
+                   seed=1200 + seed)

@@ -19,8 +19,22 @@ fp8q_api.cu) on the CPU for many shapes and grid sizes and check:
 import numpy as np
 import pytest
 
-BM, BN, SLAB_K = 128, 128, 128
+BM, SLAB_K = 128, 128
 EPI_WARPS = range(4, 12)
+
+
+def tile_n(N, K, staged=True, kind="masked", m_tiles=1, num_sms=148):
+    """The launcher's tile width (fp8q_api.cu, use_wide_tiles): 256 columns on
+    the staged-scale path when N is a multiple of 256 and, for the dense and
+    contiguous layouts, 2 x 0.95 x (rounds of wide tiles) <= rounds of
+    128-column tiles; else 128."""
+    if not (staged and (K // SLAB_K) % 4 == 0 and N % 256 == 0):
+        return 128
+    if kind == "masked":
+        return 256
+    r_narrow = -(-(m_tiles * (N // 128)) // num_sms)
+    r_wide = -(-(m_tiles * (N // 256)) // num_sms)
+    return 256 if 19 * r_wide <= 10 * r_narrow else 128
 
 
 def masked_rows(masked_m, e, cap):
@@ -54,7 +68,7 @@ def warp_scan_prefix(masked_m, cap, n_tiles):
     return prefix
 
 
-def get_tile(kind, t, *, M, N, E, n_tiles, m_indices=None, masked_m=None, prefix=None):
+def get_tile(kind, t, *, M, N, E, n_tiles, m_indices=None, masked_m=None, prefix=None, bn=128):
     """Returns (a_row, b_row, n0, e, rows) or None for a skipped tile."""
     if kind == "masked":
         lo, hi = 0, E
@@ -69,10 +83,10 @@ def get_tile(kind, t, *, M, N, E, n_tiles, m_indices=None, masked_m=None, prefix
         mt_count = -(-rows_e // BM)
         local = t - prefix[e]
         nt, mt = divmod(local, mt_count)
-        n0 = nt * BN
+        n0 = nt * bn
         return e * M + mt * BM, e * N + n0, n0, e, min(BM, rows_e - mt * BM)
     mt, nt = divmod(t, n_tiles)
-    a_row, n0 = mt * BM, nt * BN
+    a_row, n0 = mt * BM, nt * bn
     if kind == "contiguous":
         e = int(m_indices[mt])
         if e < 0 or e >= E:
@@ -83,9 +97,10 @@ def get_tile(kind, t, *, M, N, E, n_tiles, m_indices=None, masked_m=None, prefix
     return a_row, e * N + n0, n0, e, rows
 
 
-def replay(kind, *, M, N, K, E=1, m_indices=None, masked_m=None, num_sms=148):
+def replay(kind, *, M, N, K, E=1, m_indices=None, masked_m=None, num_sms=148, staged=True):
     """Runs the scheduler and the epilogue stores of every CTA; returns the
     per-element write counts of C (shape [a_rows, N])."""
+    BN = tile_n(N, K, staged, kind, (M // BM) if kind == "contiguous" else -(-M // BM), num_sms)
     n_tiles = -(-N // BN)
     nnb = N // 128
     assert K >= SLAB_K and K % SLAB_K == 0
@@ -106,7 +121,7 @@ def replay(kind, *, M, N, K, E=1, m_indices=None, masked_m=None, num_sms=148):
     for bx in range(grid):
         for t in range(bx, total, grid):
             tile = get_tile(kind, t, M=M, N=N, E=E, n_tiles=n_tiles, m_indices=m_indices, masked_m=masked_m,
-                            prefix=prefix)
+                            prefix=prefix, bn=BN)
             if tile is None:
                 continue
             a_row, b_row, n0, e, rows = tile
@@ -119,6 +134,14 @@ def replay(kind, *, M, N, K, E=1, m_indices=None, masked_m=None, num_sms=148):
                 col_ok = col0 < N
                 sb_row = e * nnb + (col0 // 128 if col_ok else 0)
                 assert 0 <= sb_row < E * nnb                    # sb is [E*N/128, nkb]
+                if staged and (K // SLAB_K) % 4 == 0:
+                    # the staged box: BN/128 block rows from the tile's first; this half reads row (half*BN/2)//128
+                    box0, box_rows = e * nnb + n0 // 128, max(1, BN // 128)
+                    assert (half * (BN // 2)) // 128 < box_rows
+                    if col_ok:
+                        assert box0 + (half * (BN // 2)) // 128 == sb_row
+                    if BN > 128:
+                        assert box0 + box_rows <= E * nnb       # a wide tile's box stays inside sb
                 for lane in range(32):
                     r = quad * 32 + lane
                     row_ok = r < rows
@@ -131,9 +154,24 @@ def replay(kind, *, M, N, K, E=1, m_indices=None, masked_m=None, num_sms=148):
 
 @pytest.mark.parametrize("M,N,sms", [(1, 128, 148), (128, 256, 148), (300, 384, 5), (4096, 7168, 148),
                                      (129, 128, 1), (1000, 1024, 7)])
-def test_dense_writes_every_element_once(M, N, sms):
-    w = replay("dense", M=M, N=N, K=256, num_sms=sms)
+@pytest.mark.parametrize("K", [256, 512])
+def test_dense_writes_every_element_once(M, N, sms, K):
+    """K = 512 takes the staged-scale path, so N % 256 == 0 shapes use wide tiles."""
+    w = replay("dense", M=M, N=N, K=K, num_sms=sms)
     assert np.all(w == 1)
+
+
+def test_tile_width_choice():
+    # only whole 256-column blocks on the staged-scale path
+    assert tile_n(7168, 7168) == 256 and tile_n(4096, 2048) == 256
+    assert tile_n(384, 512) == 128 and tile_n(7168, 1664) == 128 and tile_n(7168, 512, staged=False) == 128
+    # dense 4096 x 7168: 896 wide tiles take 7 rounds against 13 of 1792 narrow ones (13.3 > 13): narrow
+    assert tile_n(7168, 7168, kind="dense", m_tiles=32) == 128
+    # 8192 x 4096: 7 rounds against 14: wide; 2048 x 2048: 1 against 2: wide
+    assert tile_n(4096, 7168, kind="dense", m_tiles=64) == 256
+    assert tile_n(2048, 16384, kind="dense", m_tiles=16) == 256
+    # the MoE contiguous workload (274 row blocks, N = 4096): 30 rounds against 60: wide
+    assert tile_n(4096, 7168, kind="contiguous", m_tiles=274) == 256
 
 
 def test_contiguous_skips_padding_blocks():
@@ -143,6 +181,11 @@ def test_contiguous_skips_padding_blocks():
     m_indices[[3, 17, 39]] = -1          # padding blocks
     m_indices[20] = E                    # out of range: skipped as well
     for sms in (148, 9, 1):
+        for K in (128, 512):
+            w = replay("contiguous", M=blocks * BM, N=N, K=K, E=E, m_indices=m_indices, num_sms=sms)
+            for b in range(blocks):
+                want = 1 if 0 <= m_indices[b] < E else 0
+                assert np.all(w[b * BM:(b + 1) * BM] == want), (sms, b, K)
         w = replay("contiguous", M=blocks * BM, N=N, K=128, E=E, m_indices=m_indices, num_sms=sms)
         for b in range(blocks):
             want = 1 if 0 <= m_indices[b] < E else 0
