@@ -584,34 +584,50 @@ __global__ void __launch_bounds__(256, kMinBlocks) quant_act_128x1_t_kernel(cons
 // so the forward GEMM on the transposed codes computes dY * W (the
 // activation-gradient GEMM).
 //
-// One 256-thread CTA per block, no shared memory: thread (l = t % 16,
-// j = t / 16) loads the 8x8 bytes at rows 8l.., columns 8j.. (eight 8-byte
-// loads; the two warps reading a 32-byte sector share it through L1),
-// transposes them in registers and stores eight 8-byte pieces, rows 8j..,
-// columns 8l.. of the output: each warp store writes two full 128-byte rows.
+// One 256-thread CTA per block.  The 16 KB block is read with coalesced
+// 16-byte loads (eight lanes per 128-byte row) into a shared tile whose
+// 8-byte slots are XOR-swizzled by row group (slot s of row R sits at
+// s ^ (R / 8)); thread (l = t % 16, j = t / 16) then takes the 8x8 bytes at
+// rows 8l.., columns 8j.. (eight 8-byte shared loads, one wavefront per half
+// warp), transposes them in registers and stores eight 8-byte pieces at rows
+// 8j.., columns 8l.. of the output: each warp store writes two full 128-byte
+// rows.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint2 ldg_u2(const uint8_t* p) {
-  return __ldg(reinterpret_cast<const uint2*>(p));
-}
-
 __global__ void __launch_bounds__(256) transpose_w_128x128_kernel(const uint8_t* __restrict__ qw,
                                                                   const float* __restrict__ sw,
                                                                   uint8_t* __restrict__ qt, float* __restrict__ st,
                                                                   int64_t N, int64_t K, int64_t num_blocks) {
+  __shared__ __align__(16) uint8_t tile[128 * 128];
   const int tid = threadIdx.x;
   const int l = tid & 15, j = tid >> 4;
   const int64_t nkb = K >> 7, nnb = N >> 7;
   for (int64_t b = blockIdx.x; b < num_blocks; b += gridDim.x) {
     const int64_t g = b / (nnb * nkb), rem = b % (nnb * nkb);
     const int64_t nb = rem / nkb, kb = rem % nkb;
-    const uint8_t* src = qw + (g * N + nb * 128 + 8 * l) * K + kb * 128 + 8 * j;
+    const uint8_t* src = qw + (g * N + nb * 128) * K + kb * 128;
+    // rows tid / 8 + 32 i, 16-byte chunk tid % 8 (slots 2c, 2c + 1)
+    uint4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int row = (tid >> 3) + 32 * i, c = tid & 7;
+      v[i] = ld_nc_v4(src + static_cast<int64_t>(row) * K + c * 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int row = (tid >> 3) + 32 * i, c = tid & 7, x = (row >> 3) & 15;
+      *reinterpret_cast<uint2*>(tile + row * 128 + (((2 * c) ^ x) << 3)) = make_uint2(v[i].x, v[i].y);
+      *reinterpret_cast<uint2*>(tile + row * 128 + (((2 * c + 1) ^ x) << 3)) = make_uint2(v[i].z, v[i].w);
+    }
+    __syncthreads();
     uint32_t lo[8], hi[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      const uint2 v = ldg_u2(src + static_cast<int64_t>(r) * K);
-      lo[r] = v.x;
-      hi[r] = v.y;
+      const int row = 8 * l + r;  // row group l
+      const uint2 w = *reinterpret_cast<const uint2*>(tile + row * 128 + ((j ^ l) << 3));
+      lo[r] = w.x;
+      hi[r] = w.y;
     }
+    __syncthreads();  // the tile is reused by the next block
     transpose8x8_bytes(lo, hi);  // lo[c], hi[c]: column 8j + c, rows 8l .. 8l + 7
     uint8_t* dst = qt + (g * K + kb * 128 + 8 * j) * N + nb * 128 + 8 * l;
 #pragma unroll

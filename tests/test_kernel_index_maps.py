@@ -74,10 +74,13 @@ def test_act_128x1_covers_every_element_once(M, K, grid):
 
 
 def transpose_map(G, N, K, grid):
-    """transpose_w_128x128_kernel: block b -> (g, nb, kb); thread (l = t % 16,
-    j = t / 16) reads the 8x8 bytes at rows 8l.., columns 8j.. of the block
-    and writes them transposed at output rows 8j.., columns 8l..  Returns the
-    read and write counts and the output as tags of the source elements."""
+    """transpose_w_128x128_kernel: block b -> (g, nb, kb).  Thread t reads the
+    16-byte chunk t % 8 of block rows t / 8 + 32 i (i < 4) and writes its two
+    8-byte slots 2c, 2c + 1 to the shared tile at slot s ^ (R / 8) of row R;
+    then thread (l = t % 16, j = t / 16) reads slot j ^ l of rows 8l + r
+    (r < 8), i.e. the 8x8 bytes at rows 8l.., columns 8j.., and writes them
+    transposed at output rows 8j.., columns 8l..  Returns the read and write
+    counts and the output as tags of the source elements."""
     nkb, nnb = K // TILE, N // TILE
     blocks = G * nnb * nkb
     out = np.full((G, K, N), -1, dtype=np.int64)
@@ -90,17 +93,40 @@ def transpose_map(G, N, K, grid):
         while b < blocks:
             g, rem = b // (nnb * nkb), b % (nnb * nkb)
             nb, kb = rem // nkb, rem % nkb
+            tile = np.full((128, 16, 8), -1, dtype=np.int64)   # [row][physical 8-byte slot][byte]
+            tile_writes = np.zeros((128, 16), dtype=np.int32)
+            for t in range(256):
+                for i in range(4):
+                    row, c = (t >> 3) + 32 * i, t & 7
+                    r0, c0 = nb * 128 + row, kb * 128 + 16 * c
+                    src[g, r0, c0:c0 + 16] += 1
+                    x = (row >> 3) & 15
+                    for h in range(2):
+                        slot = (2 * c + h) ^ x
+                        tile[row, slot] = tags[g, r0, c0 + 8 * h:c0 + 8 * h + 8]
+                        tile_writes[row, slot] += 1
+            assert np.all(tile_writes == 1)            # the swizzle is a permutation of each row's slots
             for t in range(256):
                 l, j = t & 15, t >> 4
-                r0, c0 = nb * 128 + 8 * l, kb * 128 + 8 * j
-                src[g, r0:r0 + 8, c0:c0 + 8] += 1
-                block = tags[g, r0:r0 + 8, c0:c0 + 8]          # [r][c]
+                block = np.stack([tile[8 * l + r, j ^ l] for r in range(8)])   # [r][c]
                 o0, oc = kb * 128 + 8 * j, nb * 128 + 8 * l
                 out[g, o0:o0 + 8, oc:oc + 8] = block.T       # lo[c], hi[c] after the register transpose
                 writes[g, o0:o0 + 8, oc:oc + 8] += 1
             st[g, kb, nb] += 1
             b += grid
     return src, writes, st, out, tags
+
+
+def test_transpose_tile_reads_are_conflict_free():
+    """Each half-warp's eight-byte shared loads (fixed j, l = 0..15, fixed r)
+    cover all 32 banks once: one wavefront per half warp."""
+    for r in range(8):
+        for j in range(16):
+            banks = set()
+            for l in range(16):
+                addr = (8 * l + r) * 128 + ((j ^ l) << 3)
+                banks.update({(addr // 4) % 32, (addr // 4 + 1) % 32})
+            assert len(banks) == 32
 
 
 @pytest.mark.parametrize("G,N,K,grid", [(1, 128, 128, 1), (1, 256, 384, 2), (3, 128, 256, 5)])
