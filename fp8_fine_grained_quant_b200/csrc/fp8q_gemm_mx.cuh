@@ -15,9 +15,8 @@
 // with the slab's operands, then copied to TMEM by the MMA thread
 // (tcgen05.cp 32x128b.warpx4): TMEM lane l, column c holds rows l + 32 c of
 // the tile, byte j the scale of K block j.  The MMA's scale-factor id j picks
-// the byte.  tcgen05.cp and tcgen05.mma of one thread execute in order; the
-// slabs rotate over four sets of eight TMEM columns, so the copy for the next
-// slab does not overwrite what the current slab's MMAs still read.
+// the byte.  tcgen05.cp and tcgen05.mma of one thread execute in order, so
+// the same eight TMEM columns serve every slab.
 //
 // Global scale layout (written by mx_scales_*_kernel): atoms [tile][slab][512]
 // with byte 16 m0 + 4 m1 + j = the scale of tile row 32 m1 + m0 (all four j
@@ -55,12 +54,8 @@ struct MxSmem {
   static constexpr uint32_t kBytes = kOffPrefix + 4 * (kMaxMaskedExperts + 1);
   static constexpr uint32_t kDynamicBytes = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;    // 2 accumulators x 128 + scale factors
-  // Scale factors of slab j in slot j % kSfSlots (4 columns for A, then 4 for
-  // B): the copy for slab j + 1 never writes the columns the MMAs of slab j
-  // read, so it need not wait for them.
-  static constexpr int kSfSlots = 4;
-  static constexpr uint32_t kTmemSf = 256;      // kSfSlots x 8 columns
-  static_assert(kTmemSf + 8 * kSfSlots <= kTmemCols, "scale-factor slots fit in TMEM");
+  static constexpr uint32_t kTmemSfa = 256;     // 4 columns
+  static constexpr uint32_t kTmemSfb = 260;     // 4 columns
   static_assert(kDynamicBytes <= 227u * 1024u, "shared memory per CTA");
 };
 
@@ -125,13 +120,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int32_t total = *total_slot;
 
-  if ((warp == 0 || warp == 3) && lane == 0) {
-    // ---------------------------------------------------------------- producers
-    // two threads on alternate slabs (an even stage count keeps each on its own stages)
-    static_assert(kMxStages % 2 == 0, "two producers take alternate slabs");
-    const uint32_t who = warp == 0 ? 0u : 1u;
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- producer
     int stage = 0;
-    uint32_t phase = 0, j = 0;
+    uint32_t phase = 0;
     uint32_t armed = 0, armed_parity = 0;
     bool ok = true;
     for (int32_t t = blockIdx.x; ok && t < total && !*wc.abort; t += gridDim.x) {
@@ -140,14 +132,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // scale atoms of this tile's 128 A rows and 128 B rows (both multiples of 128)
       const uint8_t* sfa_t = args.sfa + static_cast<int64_t>(tile.a_row / kBlockM) * nkb * kMxAtomBytes;
       const uint8_t* sfb_t = args.sfb + static_cast<int64_t>(tile.b_row / 128) * nkb * kMxAtomBytes;
-      for (int kb = 0; kb < nkb; ++kb, ++j) {
-        if ((j & 1u) != who) {
-          if (++stage == kMxStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-          continue;
-        }
+      for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait(bars.empty(stage), phase ^ 1u, wc, 0x11)) { ok = false; break; }
         mbar_arrive_expect_tx(bars.full(stage), L::kStageBytes + 2 * kMxAtomBytes);
         tma_load_2d(s_base + L::kOffA + stage * L::kABytes, &tma_a, bars.full(stage), kb * kSlabK, tile.a_row);
@@ -174,7 +159,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int stage = 0, buf = 0;
     uint32_t phase = 0, tphase = 0;
     bool ok = true;
-    uint32_t sf_slot = 0;
+    const uint32_t sfa_t = tmem_base + L::kTmemSfa, sfb_t = tmem_base + L::kTmemSfb;
     for (int32_t t = blockIdx.x; ok && t < total && !*wc.abort; t += gridDim.x) {
       Tile tile;
       if (!get_tile<S, 128>(ga, prefix, t, tile)) continue;
@@ -185,8 +170,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait(bars.full(stage), phase, wc, 0x13)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sf = s_base + L::kOffSf + stage * 2 * kMxAtomBytes;
-        const uint32_t sfa_t = tmem_base + L::kTmemSf + 8u * sf_slot, sfb_t = sfa_t + 4u;
-        sf_slot = sf_slot + 1 == static_cast<uint32_t>(L::kSfSlots) ? 0u : sf_slot + 1;
         tmem_cp_32x128b_warpx4(sfa_t, smem_desc_k_none(sf, 128));
         tmem_cp_32x128b_warpx4(sfb_t, smem_desc_k_none(sf + kMxAtomBytes, 128));
         const uint64_t adesc = smem_desc_k_sw128(s_base + L::kOffA + stage * L::kABytes);

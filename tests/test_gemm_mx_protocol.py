@@ -1,9 +1,8 @@
 """Host model of the block-scaled (UE8M0) GEMM's barrier protocol.
 
 Roles of gemm_mx_kernel (fp8q_gemm_mx.cuh), meeting only through mbarriers:
-  * producers (two threads on alternate slabs): per slab, wait empty[s] (the
-    slab STAGES back released the stage), then the copies (A, B tiles and both
-    scale atoms) land on full[s];
+  * producer: per slab, wait empty[s] (the slab STAGES back released the
+    stage), then the copies (A, B tiles and both scale atoms) land on full[s];
   * MMA thread: per tile, wait tempty[b] (the epilogue has read the tile two
     back out of accumulator b); per slab, wait full[s], copy the atoms to the
     scale-factor columns and issue the MMAs; one commit per slab arrives on
@@ -40,7 +39,7 @@ class Bar:
         return ok
 
 
-def simulate(tiles, nkb, stages=6, warps=8, producers=2, seed=0, max_steps=1_000_000):
+def simulate(tiles, nkb, stages=6, warps=8, seed=0, max_steps=1_000_000):
     rng = random.Random(seed)
     full = [Bar(1) for _ in range(stages)]
     empty = [Bar(1) for _ in range(stages)]
@@ -49,7 +48,7 @@ def simulate(tiles, nkb, stages=6, warps=8, producers=2, seed=0, max_steps=1_000
     J = tiles * nkb
     stage_slab, stage_busy = [None] * stages, [False] * stages
     acc_tile, acc_readers = [None] * 2, [0] * 2
-    prod_j = list(range(producers))  # next slab of each producer
+    prod_j = 0
     mma_t, mma_kb = 0, 0          # next tile / slab of the MMA thread
     epi_t = [0] * warps
     tma, pipe = [], []            # in-flight copies; tensor-pipe queue (in order): ("mma", j, s, b) / ("tile", t, b)
@@ -58,10 +57,10 @@ def simulate(tiles, nkb, stages=6, warps=8, producers=2, seed=0, max_steps=1_000
 
     def acts():
         a = []
-        for p in range(producers):
-            j = prod_j[p]
-            if j < J and (j < stages or empty[j % stages].passes(j // stages - 1)):
-                a.append(("prod", p))
+        if prod_j < J:
+            s = prod_j % stages
+            if prod_j < stages or empty[s].passes(prod_j // stages - 1):
+                a.append("prod")
         if mma_t < tiles:
             b = mma_t % 2
             j = mma_t * nkb + mma_kb
@@ -86,12 +85,11 @@ def simulate(tiles, nkb, stages=6, warps=8, producers=2, seed=0, max_steps=1_000
         act = rng.choice(a)
         steps += 1
         assert steps < max_steps
-        if isinstance(act, tuple) and act[0] == "prod":
-            p = act[1]
-            s = prod_j[p] % stages
+        if act == "prod":
+            s = prod_j % stages
             assert not stage_busy[s], "stage refilled before its MMAs read it"
-            tma.append((prod_j[p], s))
-            prod_j[p] += producers
+            tma.append((prod_j, s))
+            prod_j += 1
         elif act == "land":
             j, s = tma.pop(rng.randrange(len(tma)))
             stage_slab[s], stage_busy[s] = j, True
