@@ -559,7 +559,7 @@ int fp8_quant_act_128x1_t(const void* x_bf16, int64_t M, int64_t K, int64_t Mp, 
   const int64_t blocks = (Mp / 128) * (K / 128);
   const int64_t cap = static_cast<int64_t>(dev->num_sms) * 16;
   const int64_t grid = blocks < cap ? blocks : cap;
-  quant_act_128x1_t_kernel<2><<<static_cast<unsigned>(grid), 256, 0, stream>>>(static_cast<const uint8_t*>(x_bf16), qt,
+  quant_act_128x1_t_kernel<3><<<static_cast<unsigned>(grid), 256, 0, stream>>>(static_cast<const uint8_t*>(x_bf16), qt,
                                                                              s, M, K, Mp, blocks);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);

@@ -475,7 +475,7 @@ __device__ __forceinline__ void transpose8x8_bytes(uint32_t (&lo)[8], uint32_t (
   }
 }
 
-// kMinBlocks: CTAs per SM the register budget is fitted to (2: 128 registers).
+// kMinBlocks: CTAs per SM the register budget is fitted to (3: 80 registers, launched so).
 template <int kMinBlocks = 2>
 __global__ void __launch_bounds__(256, kMinBlocks) quant_act_128x1_t_kernel(const uint8_t* __restrict__ x,
                                                                 uint8_t* __restrict__ qt, float* __restrict__ s,
