@@ -685,7 +685,7 @@ __device__ __forceinline__ void swiglu16(const uint32_t (&gw)[8], const uint32_t
 // scales.  Tile t = row * (inter/128) + kb, as in quant_act_1x128_kernel.  With
 // masked_m, row = e * cap + r is valid when r < clamp(masked_m[e], 0, cap);
 // other rows are neither read nor written.
-__global__ void __launch_bounds__(256, 4) swiglu_quant_1x128_kernel(const uint8_t* __restrict__ c1,
+__global__ void __launch_bounds__(256, 5) swiglu_quant_1x128_kernel(const uint8_t* __restrict__ c1,
                                                                     uint8_t* __restrict__ qh, float* __restrict__ sh,
                                                                     int64_t inter, int64_t num_tiles,
                                                                     const int32_t* __restrict__ masked_m,

@@ -47,17 +47,19 @@ def test_set_timeout_roundtrip(dev):
 
 
 @pytest.mark.parametrize("limit_ns", [1_000, 20_000])
-def test_gemm_with_a_short_wait_limit_returns_and_recovers(dev, limit_ns):
+@pytest.mark.parametrize("M", [1024, 2048])
+def test_gemm_with_a_short_wait_limit_returns_and_recovers(dev, limit_ns, M):
     """A GEMM launched with a wait limit of a few microseconds: waits may run
     out (the call then records FP8Q_ERR_TIMEOUT and the kernel drains its
     copies and MMAs before it frees TMEM and exits) or not (FP8Q_OK); either
     way the call returns, and a GEMM run afterwards with the default limit is
-    exact against the oracle."""
+    exact against the oracle.  M = 1024 runs 128 x 128 tiles, M = 2048 the
+    128 x 256 tiles (one round of 128 against two)."""
     import oracle
     import workloads as wl
     from parity import assert_gemm_close, bf16_bits_of, to_torch_bf16
-    rng = np.random.default_rng(limit_ns)
-    a = wl.bf16_bits(rng.standard_normal((1024, 4096)).astype(np.float32))
+    rng = np.random.default_rng(limit_ns + M)
+    a = wl.bf16_bits(rng.standard_normal((M, 4096)).astype(np.float32))
     b = wl.bf16_bits((0.02 * rng.standard_normal((2048, 4096))).astype(np.float32))
     qa, sa = fq.fp8_quant_act_1x128(to_torch_bf16(a, dev))
     qb, sb = fq.fp8_quant_w_128x128(to_torch_bf16(b, dev))
@@ -73,7 +75,7 @@ def test_gemm_with_a_short_wait_limit_returns_and_recovers(dev, limit_ns):
     c = fq.fp8_gemm_blockscaled(qa, sa, qb, sb)
     torch.cuda.synchronize(dev)
     assert fq.get_device_error(device=dev) == fq.OK
-    rows = wl.quad_rows(np.random.default_rng(1), 1024)
+    rows = wl.quad_rows(np.random.default_rng(1), M)
     oqa, osa = oracle.quant_act_1x128(a)
     oqb, osb = oracle.quant_w_128x128(b)
     assert_gemm_close(bf16_bits_of(c)[rows], oracle.gemm_blockscaled(oqa, osa, oqb, osb, rows=rows),
