@@ -213,6 +213,10 @@ struct GemmCall {
   int promote;
 };
 
+// Output tiles of one GEMM launch: the kernels number them (and walk them,
+// t += gridDim.x) in 32-bit integers.
+constexpr int64_t kMaxTiles = (int64_t(1) << 31) - (int64_t(1) << 16);
+
 // One launch of one kernel instance.
 template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D>
 int launch_instance(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa, const CUtensorMap& msb,
@@ -270,6 +274,7 @@ int launch_gemm(const GemmCall& g, const DeviceInfo& dev, cudaStream_t stream) {
   a.m_tiles = static_cast<int32_t>(g.m_tiles);
   a.n_tiles = static_cast<int32_t>((g.N + BN - 1) / BN);
   const int64_t max_tiles = g.m_tiles * a.n_tiles * (S == Sched::kMasked ? g.E : 1);
+  if (max_tiles >= kMaxTiles) return FP8Q_ERR_SHAPE;  // the kernel numbers tiles in 32 bits
   const int64_t grid = max_tiles < dev.num_sms ? max_tiles : dev.num_sms;
   if (grid <= 0) return FP8Q_OK;
   return launch_instance<BN, STAGES, S, kPromote, kTmaScales, k1D1D>(ma, mb, msa, msb, a, grid, stream);
@@ -432,6 +437,7 @@ static int launch_mx(const GemmCall& g, const uint8_t* sfa_mx, const uint8_t* sf
   a.sfa = sfa_mx;
   a.sfb = sfb_mx;
   const int64_t max_tiles = g.m_tiles * (g.N / 128) * (S == Sched::kMasked ? g.E : 1);
+  if (max_tiles >= kMaxTiles) return FP8Q_ERR_SHAPE;  // the kernel numbers tiles in 32 bits
   const int grid = static_cast<int>(max_tiles < dev->num_sms ? max_tiles : dev->num_sms);
   if (grid <= 0) return FP8Q_OK;
   cudaLaunchConfig_t cfg;

@@ -100,3 +100,17 @@ def test_masked_gemm_with_a_short_wait_limit_returns(dev):
     torch.cuda.synchronize(dev)
     assert fq.get_device_error(device=dev) == fq.OK
     assert torch.isfinite(c[0].float()).all()
+
+
+def test_gemm_rejects_tile_counts_beyond_32_bits(dev):
+    """Shapes whose output-tile count does not fit the kernels' 32-bit tile
+    numbers are refused before any launch (the pointers are never used: the
+    call stops at the tile count, after encoding the tensor maps)."""
+    lib = fq.lib()
+    fake = 0x10000  # 256-byte aligned, never dereferenced
+    big = 1 << 30
+    with torch.cuda.device(dev):
+        for M, N in ((big, big), (1 << 28, 1 << 24)):
+            st = lib.fp8_gemm_blockscaled(fake, fake, fake, fake, fake, M, N, 512, None)
+            assert st == fq.ERR_SHAPE, (M, N, st)
+    assert fq.get_device_error(device=dev) == fq.OK
