@@ -33,8 +33,9 @@
  *  - Pointer alignment: the quantizers' bf16 inputs 32 bytes; every other
  *    bf16 / FP8 / output pointer 16 bytes; scale and index pointers 4 bytes.
  *  - Size limits: every row count, column count and K below 2^31, and so are
- *    the stacked row counts E*N, G*N and E*cap; larger shapes return
- *    FP8Q_ERR_SHAPE.
+ *    the stacked row counts E*N, G*N and E*cap; a GEMM's count of 128-row
+ *    output tiles times its column tiles (times E for the masked layout) stays
+ *    below 2^31 - 2^16; larger shapes return FP8Q_ERR_SHAPE.
  *  - Non-finite inputs are outside the contract (results unspecified, no fault).
  *  - Every on-device wait is bounded (default 4 s, see fp8q_set_wait_timeout_ns);
  *    a wait that runs out records FP8Q_ERR_TIMEOUT in a device status word
