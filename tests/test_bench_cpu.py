@@ -116,3 +116,18 @@ def test_dgrad_plan_counts_the_transposed_gemm():
     assert labels == ["quant_act_w", "transpose_w_128x128", "gemm_dgrad"]
     assert plan[-1][2] == 2.0 * 4096 * 7168 * 7168
     assert plan[1][1] == 2 * 7168 * 7168 + 8 * 56 * 56
+
+
+def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(tmp_path, monkeypatch):
+    """profiles/traffic.json entries carry the kernel sources' hash: an entry
+    counts only while the sources hash to it (else the line's traffic is null)."""
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    entry = {"dram_bytes_per_launch": 123, "source_hash": bench.source_hash()}
+    (prof / "traffic.json").write_text(json.dumps({"gemm_blockscaled:dense_fprop": entry,
+                                                  "quant_act_w:dense_fprop": dict(entry, source_hash="0" * 16)}))
+    monkeypatch.setattr(bench, "ROOT", tmp_path)
+    monkeypatch.setattr(bench, "source_hash", lambda: entry["source_hash"])
+    assert bench.traffic_for("gemm_blockscaled", "dense_fprop") == 123
+    assert bench.traffic_for("quant_act_w", "dense_fprop") is None      # taken on other sources
+    assert bench.traffic_for("gemm_blockscaled", "long_k") is None       # never taken
