@@ -154,7 +154,7 @@ def _near_midpoint_tiles(seed=17, n_scales=400):
     xs_all = wl.bf16_to_f32(pos)
     tiles = []
     for _ in range(n_scales):
-        amax = np.float32(wl.bf16_to_f32(wl.bf16_bits(np.float32(np.exp(rng.uniform(-30, 30))))))
+        amax = wl.bf16_to_f32(wl.bf16_bits(np.float32(np.exp(rng.uniform(-30, 30))))).reshape(-1)[0]
         s = np.float32(amax / np.float32(448.0))
         if s == 0 or s < np.float32(2.0 ** -125):
             continue
