@@ -42,7 +42,9 @@ def bytes_of(t: torch.Tensor) -> np.ndarray:
 
 
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
-    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    # a signalling-NaN pattern raises the invalid flag in the widening; it stays a NaN
+    with np.errstate(invalid="ignore"):
+        return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def bf16_rne_f64(x: np.ndarray) -> np.ndarray:
