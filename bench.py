@@ -153,7 +153,7 @@ class ClockSampler:
 # (a few GB on the device at most); never a bench line of their own.
 PROFILE_SIZES = {
     "dense_fprop": dict(M=2048), "long_k": dict(M=1024), "moe_contiguous": dict(tokens=1024, E=8),
-    "moe_masked": dict(E=8),
+    "moe_masked": dict(E=8), "moe_masked_chain": dict(E=8),
 }
 PROFILE_SIZE = False
 
@@ -166,6 +166,8 @@ def make_workload(name: str, shard: int = 0, device=None):
     import workloads as wl
     if PROFILE_SIZE and name in PROFILE_SIZES:
         kw = PROFILE_SIZES[name]
+        if name == "moe_masked_chain":
+            return wl.moe_masked(device=device, **kw)
         if name.startswith("moe"):
             return wl.CONFIGS[name](device=device, **kw)
         return wl.CONFIGS[name](**kw)
