@@ -49,12 +49,25 @@ DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
 // Per-device set-up, done once: SM count, arch check, status-word address,
-// and the dynamic shared-memory opt-in of every GEMM instantiation.
+// and the dynamic shared-memory opt-in of every GEMM instantiation (and of
+// the token-axis quantizer).
 template <int BN, int STAGES, Sched S, bool kPromote, bool kTmaScales, bool k1D1D = false>
 cudaError_t opt_in_smem() {
   return cudaFuncSetAttribute(gemm_blockscaled_kernel<BN, STAGES, S, kPromote, kTmaScales, k1D1D>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               GemmSmem<BN, STAGES, k1D1D>::kDynamicBytes);
+}
+
+// The token-axis quantizer's two 32 KB stages (dynamic shared memory), with
+// the carveout that lets kTokCtasPerSm of its CTAs share an SM.
+template <bool kTokenContiguous>
+cudaError_t opt_in_token_axis_smem() {
+  cudaError_t e = cudaFuncSetAttribute(quant_act_128x1_kernel<kTokenContiguous>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kTokSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(quant_act_128x1_kernel<kTokenContiguous>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  return e;
 }
 
 // Whether an instance that splits registers between its warpgroups was
@@ -119,6 +132,8 @@ int device_info(DeviceInfo** out) {
         if (e == cudaSuccess)
           e = cudaFuncSetAttribute(gemm_mx_kernel<Sched::kMasked>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    MxSmem::kDynamicBytes);
+        if (e == cudaSuccess) e = opt_in_token_axis_smem<false>();
+        if (e == cudaSuccess) e = opt_in_token_axis_smem<true>();
         if (e != cudaSuccess) return FP8Q_ERR_CUDA;
       }
       d.ready.store(true, std::memory_order_release);
@@ -326,6 +341,17 @@ int check_operands(const uint8_t* qa, const float* sa, const uint8_t* qb, const 
 
 constexpr int64_t kMaxRows = int64_t(1) << 31;
 
+// Persistent: at most kTokCtasPerSm CTAs per SM, each walking its blocks.
+template <bool kTokenContiguous>
+void launch_quant_act_128x1(const uint8_t* x, uint8_t* q, float* s, int64_t M, int64_t K, int64_t Mp, int num_sms,
+                            cudaStream_t stream) {
+  const int64_t blocks = (Mp / 128) * (K / 128);
+  const int64_t cap = static_cast<int64_t>(num_sms) * kTokCtasPerSm;
+  const int64_t grid = blocks < cap ? blocks : cap;
+  quant_act_128x1_kernel<kTokenContiguous>
+      <<<static_cast<unsigned>(grid), 256, kTokSmemBytes, stream>>>(x, q, s, M, K, Mp, blocks);
+}
+
 }  // namespace
 
 // Reads and clears the status word in one atomic step, after the work queued
@@ -519,11 +545,8 @@ int fp8_quant_act_128x1(const void* x_bf16, int64_t M, int64_t K, uint8_t* q, fl
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);
   if (rc) return rc;
-  const int64_t blocks = ((M + 127) / 128) * (K / 128);
-  const int64_t cap = static_cast<int64_t>(dev->num_sms) * 16;
-  const int64_t grid = blocks < cap ? blocks : cap;
-  quant_act_128x1_kernel<2><<<static_cast<unsigned>(grid), 256, 0, stream>>>(static_cast<const uint8_t*>(x_bf16), q, s,
-                                                                           M, K, blocks);
+  const int64_t Mp = (M + 127) / 128 * 128;
+  launch_quant_act_128x1<false>(static_cast<const uint8_t*>(x_bf16), q, s, M, K, Mp, dev->num_sms, stream);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FP8Q_OK;
@@ -562,11 +585,7 @@ int fp8_quant_act_128x1_t(const void* x_bf16, int64_t M, int64_t K, int64_t Mp, 
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);
   if (rc) return rc;
-  const int64_t blocks = (Mp / 128) * (K / 128);
-  const int64_t cap = static_cast<int64_t>(dev->num_sms) * 16;
-  const int64_t grid = blocks < cap ? blocks : cap;
-  quant_act_128x1_t_kernel<3><<<static_cast<unsigned>(grid), 256, 0, stream>>>(static_cast<const uint8_t*>(x_bf16), qt,
-                                                                             s, M, K, Mp, blocks);
+  launch_quant_act_128x1<true>(static_cast<const uint8_t*>(x_bf16), qt, s, M, K, Mp, dev->num_sms, stream);
   if (cudaGetLastError() != cudaSuccess) return FP8Q_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FP8Q_OK;

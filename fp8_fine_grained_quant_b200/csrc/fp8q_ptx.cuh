@@ -377,6 +377,19 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
 }
 
 
+// 16 bytes global -> shared through the L2 only (cp.async.cg); both addresses
+// 16-byte aligned.  With src_bytes = 0 nothing is read and the 16 bytes are
+// zero-filled.  Completion is tracked per thread by commit groups.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Waits until at most N of this thread's committed groups are still pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // 16 bytes in one 128-bit load (read-only, not kept in L1); p 16-byte aligned.
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   uint4 v;

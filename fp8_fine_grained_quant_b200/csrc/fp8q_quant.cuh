@@ -49,9 +49,15 @@ __device__ __forceinline__ float group_scale(float amax) {
 // of rounding RN(x r_lo) <= fl32(x/s) <= RN(x r_hi).  Rounding to E4M3 is
 // monotone too, so when the two products get the same code, fl32(x/s) gets
 // that code.  When they differ (a quotient within ~2^-20 of an E4M3 rounding
-// midpoint, a few in 10^5) the IEEE quotient is used.  Products below the
-// binary32 normal range are far below the first E4M3 midpoint (2^-10) and
+// midpoint) that element's code comes from the IEEE quotient.  Products below
+// the binary32 normal range are far below the first E4M3 midpoint (2^-10) and
 // give +-0 on every path (each product keeps the sign of x).
+//
+// With bf16 data such quotients are not rare: x and amax both carry 8-bit
+// significands, and 448 x / amax lands exactly on an E4M3 midpoint for about
+// 0.5% of the elements of normally distributed data.  So most warps meet one
+// in every step, but a lane seldom meets more than one: the fallback
+// recomputes single elements, not the lane's whole run.
 //
 // The bracket comes from the hardware's approximate reciprocal r ~ 1/s
 // (s a normal float), widened to r_lo = RN(r (1 - 2^-20)) and r_hi =
@@ -99,9 +105,30 @@ __device__ __noinline__ uint4 quantize16_exact(uint32_t w0, uint32_t w1, uint32_
   return make_uint4(c[0], c[1], c[2], c[3]);
 }
 
+// Bit 8j + 7 of the result is set when byte j of d is nonzero (the low seven
+// bits of a byte plus 0x7F carry into its top bit, never into the next byte).
+__device__ __forceinline__ uint32_t nonzero_bytes(uint32_t d) {
+  return (((d & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | d) & 0x80808080u;
+}
+
+// The bf16 element j (0..3) of a code word's two source words: byte j of a
+// word of four codes comes from word j / 2, half j % 2 (low half first).
+__device__ __forceinline__ float bf16_of_pair(uint32_t w_even, uint32_t w_odd, int j) {
+  const uint32_t word = (j & 2) ? w_odd : w_even;
+  return __uint_as_float((j & 1) ? (word & 0xFFFF0000u) : (word << 16));
+}
+
+// Replaces byte j of c by the E4M3 code of fl32(x / s).
+__device__ __forceinline__ uint32_t with_exact_code(uint32_t c, int j, float x, float s) {
+  const uint32_t code = cvt_e4m3x2(__fdiv_rn(x, s), 0.0f) & 0xFFu;
+  const int sh = 8 * j;
+  return (c & ~(0xFFu << sh)) | (code << sh);
+}
+
 // 16 bf16 (eight words) -> 16 E4M3 codes of fl32(x / s), low byte first.
 // `exact_only` forces the division (scales that are not safely normal).
 __device__ __forceinline__ uint4 quantize16(const uint32_t (&w)[8], float s, const RecipPair& rp, bool exact_only) {
+  if (exact_only || !rp.ok) return quantize16_exact(w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7], s);
   uint32_t lo[4], hi[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -110,8 +137,14 @@ __device__ __forceinline__ uint4 quantize16(const uint32_t (&w)[8], float s, con
     lo[i] = e4m3x4_from_f32x2(mul_f32x2(x0, rp.lo2), mul_f32x2(x1, rp.lo2));
     hi[i] = e4m3x4_from_f32x2(mul_f32x2(x0, rp.hi2), mul_f32x2(x1, rp.hi2));
   }
-  const uint32_t diff = (lo[0] ^ hi[0]) | (lo[1] ^ hi[1]) | (lo[2] ^ hi[2]) | (lo[3] ^ hi[3]);
-  if (exact_only || !rp.ok || diff != 0u) return quantize16_exact(w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7], s);
+  // elements whose bracket codes differ: the IEEE quotient, one at a time
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    for (uint32_t m = nonzero_bytes(lo[i] ^ hi[i]); m != 0u; m &= m - 1u) {
+      const int j = (__ffs(m) - 1) >> 3;
+      lo[i] = with_exact_code(lo[i], j, bf16_of_pair(w[2 * i], w[2 * i + 1], j), s);
+    }
+  }
   return make_uint4(lo[0], lo[1], lo[2], lo[3]);
 }
 
@@ -320,12 +353,19 @@ __global__ void __launch_bounds__(256, 4) quant_act_w_kernel(const uint8_t* __re
 // ---------------------------------------------------------------------------
 // Token-axis tiles (128x1) for the weight-gradient GEMM, which contracts over
 // tokens: the group of (mb, k) is channel k over tokens 128*mb..+127 (fewer in
-// a ragged last block).  One 256-thread CTA per 128-token x 128-channel block:
-// thread t owns channels 8*(t%16)..+7 of rows 8*(t/16)..+7, so a warp reads
-// two rows of 256 contiguous bytes per load.  The per-channel amax is reduced
-// over the 16 row groups (a shuffle, then shared memory across the 8 warps);
-// each channel's codes use its own scale, with the same exact division-free
-// filter as the other quantizers.  s is [ceil(M/128), K].
+// a ragged last block).  A 256-thread CTA quantizes one 128-token x
+// 128-channel block at a time: thread t owns channels 8*(t%16)..+7 of tokens
+// 8*(t/16)..+7.  The per-channel amax is reduced over the 16 token groups (a
+// shuffle, then shared memory across the 8 warps); each channel's codes use
+// its own scale, with the same exact division-free filter as the other
+// quantizers.  s is [ceil(M/128), K].
+//
+// The kernel is persistent: a CTA takes blocks at a stride of the grid, and
+// while it quantizes one block the next two blocks' bf16 (32 KB each) are
+// being copied into the other stages of a three-stage shared buffer (16-byte
+// cp.async per thread through the L2), so every CTA keeps loads in flight; a
+// block read straight into registers would leave the memory system idle while
+// its codes are computed.
 // ---------------------------------------------------------------------------
 
 // Codes of fl32(x / s_c) for the 8 bf16 in w (4 words; element i uses column
@@ -346,108 +386,6 @@ __device__ __noinline__ uint2 quantize8_cols_exact(uint32_t w0, uint32_t w1, uin
   }
   return make_uint2(c[0], c[1]);
 }
-
-// kMinBlocks: CTAs per SM the register budget is fitted to (2: 128 registers).
-template <int kMinBlocks = 2>
-__global__ void __launch_bounds__(256, kMinBlocks) quant_act_128x1_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
-                                                              float* __restrict__ s, int64_t M, int64_t K,
-                                                              int64_t num_blocks) {
-  __shared__ float col_max[8][16][8];  // [warp][column group][column]
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int cg = tid & 15, rg = tid >> 4;
-  const int64_t nkc = K >> 7;
-  for (int64_t b = blockIdx.x; b < num_blocks; b += gridDim.x) {
-    const int64_t mb = b / nkc, kc = b % nkc;
-    const int64_t col0 = kc * 128 + cg * 8;
-    const int64_t row0 = mb * 128 + rg * 8;
-    uint4 v[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int64_t row = row0 + r;
-      v[r] = row < M ? ld_nc_v4(x + (row * K + col0) * 2) : make_uint4(0, 0, 0, 0);
-    }
-    // per-column maxima over this thread's 8 rows
-    float m[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) m[c] = 0.0f;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const uint32_t w[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        m[2 * i] = fmaxf(m[2 * i], fabsf(__uint_as_float(w[i] << 16)));
-        m[2 * i + 1] = fmaxf(m[2 * i + 1], fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
-      }
-    }
-    // lanes l and l ^ 16 hold the same columns (two row groups of the warp)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) m[c] = fmaxf(m[c], __shfl_xor_sync(0xFFFFFFFFu, m[c], 16));
-    if (lane < 16) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) col_max[warp][cg][c] = m[c];
-    }
-    __syncthreads();
-    float sc[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float a = col_max[0][cg][c];
-#pragma unroll
-      for (int w = 1; w < 8; ++w) a = fmaxf(a, col_max[w][cg][c]);
-      sc[c] = group_scale(a);
-    }
-    __syncthreads();  // col_max is reused by the next block
-    if (rg == 0) {
-      float* sd = s + mb * K + col0;
-      *reinterpret_cast<float4*>(sd) = make_float4(sc[0], sc[1], sc[2], sc[3]);
-      *reinterpret_cast<float4*>(sd + 4) = make_float4(sc[4], sc[5], sc[6], sc[7]);
-    }
-    // bracketing reciprocals per column, paired as the packed products need them
-    uint64_t lo2[4], hi2[4];
-    bool exact_only = false;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float l0, h0, l1, h1;
-      const bool ok0 = recip_bracket(sc[2 * i], l0, h0), ok1 = recip_bracket(sc[2 * i + 1], l1, h1);
-      asm("mov.b64 %0, {%1, %2};" : "=l"(lo2[i]) : "f"(l0), "f"(l1));
-      asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[i]) : "f"(h0), "f"(h1));
-      exact_only |= sc[2 * i] < kMinFastScale || sc[2 * i + 1] < kMinFastScale || !ok0 || !ok1;
-    }
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int64_t row = row0 + r;
-      if (row >= M) break;
-      const uint32_t w[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
-      uint32_t lo[2], hi[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint64_t x0 = bf16x2_to_f32x2(w[2 * h]), x1 = bf16x2_to_f32x2(w[2 * h + 1]);
-        lo[h] = e4m3x4_from_f32x2(mul_f32x2(x0, lo2[2 * h]), mul_f32x2(x1, lo2[2 * h + 1]));
-        hi[h] = e4m3x4_from_f32x2(mul_f32x2(x0, hi2[2 * h]), mul_f32x2(x1, hi2[2 * h + 1]));
-      }
-      uint2 out = make_uint2(lo[0], lo[1]);
-      if (exact_only || ((lo[0] ^ hi[0]) | (lo[1] ^ hi[1])) != 0u)
-        out = quantize8_cols_exact(w[0], w[1], w[2], w[3], sc[0], sc[1], sc[2], sc[3], sc[4], sc[5], sc[6], sc[7]);
-      *reinterpret_cast<uint2*>(q + row * K + col0) = out;
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Token-axis (128x1) quantization with token-contiguous codes, for the weight
-// gradient dW = dY^T X.  Written as C = A * B^T, that GEMM contracts over
-// tokens: A = dY^T [N, Mp] and B = X^T [K, Mp], each row carrying one scale
-// per 128-token slab.  This kernel quantizes x [M, K] (tokens x channels) in
-// the groups of quant_act_128x1_kernel (same scales s [Mp/128, K], which is
-// the slab-major layout the GEMM stages) and writes the codes transposed,
-// qt [K, Mp] for a padded token count Mp >= M (a multiple of 128); tokens
-// past M get code 0 and whole padding groups scale 1.
-//
-// Per 128x128 block a thread owns 8 tokens x 8 channels, as in the untransposed
-// kernel.  Its 8x8 code bytes are transposed in registers (byte permutes) and
-// written to a shared [channel][token] tile whose 8-byte slots are XOR-
-// swizzled by channel / 8 (two wavefronts per warp store); each channel row
-// then leaves as eight coalesced 16-byte stores.
-// ---------------------------------------------------------------------------
 
 // 4x4 byte transpose: w[i] holds row i (byte j = column j); afterwards w[j]
 // holds column j (byte i = row i).
@@ -475,27 +413,96 @@ __device__ __forceinline__ void transpose8x8_bytes(uint32_t (&lo)[8], uint32_t (
   }
 }
 
-// kMinBlocks: CTAs per SM the register budget is fitted to (3: 80 registers, launched so).
-template <int kMinBlocks = 2>
-__global__ void __launch_bounds__(256, kMinBlocks) quant_act_128x1_t_kernel(const uint8_t* __restrict__ x,
-                                                                uint8_t* __restrict__ qt, float* __restrict__ s,
-                                                                int64_t M, int64_t K, int64_t Mp,
-                                                                int64_t num_blocks) {
-  __shared__ float col_max[8][16][8];            // [warp][column group][column]
-  __shared__ __align__(16) uint8_t tile[128 * 128];  // [channel][token], 8-byte slots swizzled
+// One 128-token x 128-channel block of bf16, as staged in shared memory
+// ([token][channel], 256 bytes per token), and the stages of a CTA: while one
+// is quantized the next two are being filled.
+constexpr int kTokBlockBytes = 128 * 128 * 2;
+constexpr int kTokStages = 3;
+constexpr int kTokSmemBytes = kTokStages * kTokBlockBytes;
+// CTAs per SM the kernel is fitted to: 128 registers, 100 KB of shared memory each.
+constexpr int kTokCtasPerSm = 2;
+
+// kTokenContiguous = false: codes q [M, K], laid out like x.
+//
+// kTokenContiguous = true: the weight gradient dW = dY^T X, written as
+// C = A * B^T, contracts over tokens: A = dY^T [N, Mp] and B = X^T [K, Mp],
+// each row carrying one scale per 128-token slab.  The codes are then written
+// transposed, q = qt [K, Mp] for a padded token count Mp >= M (a multiple of
+// 128); tokens past M get code 0 and whole padding groups scale 1.  The scales
+// s [Mp/128, K] are the slab-major layout the GEMM stages.  A thread's 8x8
+// code bytes are transposed in registers (byte permutes) and written to a
+// [channel][token] tile in the block's spent stage, whose 8-byte slots are
+// XOR-swizzled by channel / 8 (two wavefronts per warp store); each channel
+// row then leaves as eight coalesced 16-byte stores.
+//
+// Blocks are numbered b = mb * (K/128) + kc over Mp/128 token blocks (Mp =
+// 128 * ceil(M/128) for the row-major form).
+template <bool kTokenContiguous>
+__global__ void __launch_bounds__(256, kTokCtasPerSm) quant_act_128x1_kernel(const uint8_t* __restrict__ x,
+                                                                             uint8_t* __restrict__ q,
+                                                                             float* __restrict__ s, int64_t M,
+                                                                             int64_t K, int64_t Mp,
+                                                                             int64_t num_blocks) {
+  extern __shared__ __align__(128) uint8_t stage_buf[];  // [kTokStages][128 tokens][256 bytes]
+  __shared__ float col_max[8][16][8];                    // [warp][column group][column]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cg = tid & 15, rg = tid >> 4;
-  const int64_t nkc = K >> 7;
-  for (int64_t b = blockIdx.x; b < num_blocks; b += gridDim.x) {
-    const int64_t mb = b / nkc, kc = b % nkc;
-    const int64_t col0 = kc * 128 + cg * 8;
-    const int64_t row0 = mb * 128 + rg * 8;
+  // block b = mb * nkc + kc; a CTA's blocks are gridDim.x apart, i.e. step_mb
+  // token blocks and step_kc channel blocks (with a carry)
+  const int nkc = static_cast<int>(K >> 7);
+  const int step_mb = static_cast<int>(gridDim.x) / nkc, step_kc = static_cast<int>(gridDim.x) % nkc;
+  auto advance = [&](int& mb, int& kc) {
+    kc += step_kc;
+    mb += step_mb;
+    if (kc >= nkc) {
+      kc -= nkc;
+      ++mb;
+    }
+  };
+  // Copies of block (mb, kc) into stage st: 16-byte chunk c = tid + 256 i is
+  // token c / 16, channels 8 (c % 16) .. +7, so a warp copies two 256-byte
+  // token rows per instruction.  Tokens past M are zero-filled (nothing is read).
+  auto fetch = [&](int mb, int kc, int st) {
+    const uint32_t dst = smem_u32(stage_buf + st * kTokBlockBytes);
+    const uint8_t* src = x + static_cast<int64_t>(kc) * 256;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int c = tid + 256 * i, row = c >> 4, ch = c & 15;
+      const int64_t grow = static_cast<int64_t>(mb) * 128 + row;
+      const bool in = grow < M;
+      cp_async_16(dst + row * 256 + ch * 16, in ? src + grow * K * 2 + ch * 16 : x, in ? 16u : 0u);
+    }
+  };
+  // the CTA's i-th block b = blockIdx.x + i * gridDim.x lives in stage i % kTokStages;
+  // (fmb, fkc) is the next block to copy, fb its number
+  int fmb = static_cast<int>(blockIdx.x) / nkc, fkc = static_cast<int>(blockIdx.x) % nkc;
+  int64_t fb = blockIdx.x;
+#pragma unroll
+  for (int j = 0; j < kTokStages - 1; ++j) {
+    if (fb < num_blocks) fetch(fmb, fkc, j);
+    cp_async_commit();
+    fb += gridDim.x;
+    advance(fmb, fkc);
+  }
+  int st = 0, mb = static_cast<int>(blockIdx.x) / nkc, kc = static_cast<int>(blockIdx.x) % nkc;
+  for (int64_t b = blockIdx.x; b < num_blocks;
+       b += gridDim.x, advance(mb, kc), st = st + 1 == kTokStages ? 0 : st + 1) {
+    // refill the stage the previous block used (every thread is past it: the
+    // barrier at the end of the previous iteration)
+    if (fb < num_blocks) fetch(fmb, fkc, st == 0 ? kTokStages - 1 : st - 1);
+    cp_async_commit();
+    fb += gridDim.x;
+    advance(fmb, fkc);
+    cp_async_wait<kTokStages - 1>();  // this block's copies have landed; the later blocks' may be in flight
+    __syncthreads();                  // ... every thread's
+    const int64_t col0 = static_cast<int64_t>(kc) * 128 + cg * 8;
+    const int64_t row0 = static_cast<int64_t>(mb) * 128 + rg * 8;
+    uint8_t* buf = stage_buf + st * kTokBlockBytes;
+    // this thread's 8 tokens x 8 channels (a warp reads two 256-byte rows per load)
     uint4 v[8];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int64_t row = row0 + r;
-      v[r] = row < M ? ld_nc_v4(x + (row * K + col0) * 2) : make_uint4(0, 0, 0, 0);
-    }
+    for (int r = 0; r < 8; ++r) v[r] = *reinterpret_cast<const uint4*>(buf + (rg * 8 + r) * 256 + cg * 16);
+    // per-channel maxima over this thread's 8 tokens
     float m[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) m[c] = 0.0f;
@@ -508,13 +515,14 @@ __global__ void __launch_bounds__(256, kMinBlocks) quant_act_128x1_t_kernel(cons
         m[2 * i + 1] = fmaxf(m[2 * i + 1], fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
       }
     }
+    // lanes l and l ^ 16 hold the same channels (two token groups of the warp)
 #pragma unroll
     for (int c = 0; c < 8; ++c) m[c] = fmaxf(m[c], __shfl_xor_sync(0xFFFFFFFFu, m[c], 16));
     if (lane < 16) {
 #pragma unroll
       for (int c = 0; c < 8; ++c) col_max[warp][cg][c] = m[c];
     }
-    __syncthreads();
+    __syncthreads();  // col_max is complete, and the stage has been read by every thread
     float sc[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -528,6 +536,7 @@ __global__ void __launch_bounds__(256, kMinBlocks) quant_act_128x1_t_kernel(cons
       *reinterpret_cast<float4*>(sd) = make_float4(sc[0], sc[1], sc[2], sc[3]);
       *reinterpret_cast<float4*>(sd + 4) = make_float4(sc[4], sc[5], sc[6], sc[7]);
     }
+    // bracketing reciprocals per channel, paired as the packed products need them
     uint64_t lo2[4], hi2[4];
     bool exact_only = false;
 #pragma unroll
@@ -538,7 +547,7 @@ __global__ void __launch_bounds__(256, kMinBlocks) quant_act_128x1_t_kernel(cons
       asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[i]) : "f"(h0), "f"(h1));
       exact_only |= sc[2 * i] < kMinFastScale || sc[2 * i + 1] < kMinFastScale || !ok0 || !ok1;
     }
-    // codes of the 8 tokens (zero rows past M give code 0)
+    // codes of the 8 tokens (zero tokens past M give code 0)
     uint32_t clo[8], chi[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
@@ -550,31 +559,53 @@ __global__ void __launch_bounds__(256, kMinBlocks) quant_act_128x1_t_kernel(cons
         lo[h] = e4m3x4_from_f32x2(mul_f32x2(x0, lo2[2 * h]), mul_f32x2(x1, lo2[2 * h + 1]));
         hi[h] = e4m3x4_from_f32x2(mul_f32x2(x0, hi2[2 * h]), mul_f32x2(x1, hi2[2 * h + 1]));
       }
-      uint2 out = make_uint2(lo[0], lo[1]);
-      if (exact_only || ((lo[0] ^ hi[0]) | (lo[1] ^ hi[1])) != 0u)
-        out = quantize8_cols_exact(w[0], w[1], w[2], w[3], sc[0], sc[1], sc[2], sc[3], sc[4], sc[5], sc[6], sc[7]);
-      clo[r] = out.x;
-      chi[r] = out.y;
-    }
-    transpose8x8_bytes(clo, chi);  // now channel c: tokens 0-3 in clo[c], 4-7 in chi[c]
-    // channel row cg*8 + c, logical 8-byte slot rg, physical slot rg ^ cg
+      if (exact_only) {
+        const uint2 out =
+            quantize8_cols_exact(w[0], w[1], w[2], w[3], sc[0], sc[1], sc[2], sc[3], sc[4], sc[5], sc[6], sc[7]);
+        lo[0] = out.x;
+        lo[1] = out.y;
+      } else {
+        // elements whose bracket codes differ: the IEEE quotient, one at a time
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-      *reinterpret_cast<uint2*>(tile + (cg * 8 + c) * 128 + ((rg ^ cg) << 3)) = make_uint2(clo[c], chi[c]);
-    __syncthreads();
-    uint8_t* dst = qt + (kc * 128) * Mp + mb * 128;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int c = tid + 256 * i, row = c >> 3, ch = c & 7;
-      const int swz = row >> 3;  // the row's column group, 0..15
-      // logical slots 2ch, 2ch+1 sit in physical 16-byte chunk ch ^ (swz / 2),
-      // their halves swapped when swz is odd
-      uint4 o = *reinterpret_cast<const uint4*>(tile + row * 128 + ((ch ^ (swz >> 1)) << 4));
-      if (swz & 1) o = make_uint4(o.z, o.w, o.x, o.y);
-      *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(row) * Mp + ch * 16) = o;
+        for (int h = 0; h < 2; ++h) {
+          for (uint32_t mk = nonzero_bytes(lo[h] ^ hi[h]); mk != 0u; mk &= mk - 1u) {
+            const int j = (__ffs(mk) - 1) >> 3;
+            const float sj = j == 0 ? sc[4 * h] : j == 1 ? sc[4 * h + 1] : j == 2 ? sc[4 * h + 2] : sc[4 * h + 3];
+            lo[h] = with_exact_code(lo[h], j, bf16_of_pair(w[2 * h], w[2 * h + 1], j), sj);
+          }
+        }
+      }
+      clo[r] = lo[0];
+      chi[r] = lo[1];
     }
-    __syncthreads();  // col_max and the tile are reused by the next block
+    if constexpr (kTokenContiguous) {
+      transpose8x8_bytes(clo, chi);  // now channel c: tokens 0-3 in clo[c], 4-7 in chi[c]
+      // channel row cg*8 + c of the tile, logical 8-byte slot rg, physical slot rg ^ cg
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint2*>(buf + (cg * 8 + c) * 128 + ((rg ^ cg) << 3)) = make_uint2(clo[c], chi[c]);
+      __syncthreads();
+      uint8_t* dst = q + (static_cast<int64_t>(kc) * 128) * Mp + static_cast<int64_t>(mb) * 128;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = tid + 256 * i, row = c >> 3, ch = c & 7;
+        const int swz = row >> 3;  // the row's channel group, 0..15
+        // logical slots 2ch, 2ch+1 sit in physical 16-byte chunk ch ^ (swz / 2),
+        // their halves swapped when swz is odd
+        uint4 o = *reinterpret_cast<const uint4*>(buf + row * 128 + ((ch ^ (swz >> 1)) << 4));
+        if (swz & 1) o = make_uint4(o.z, o.w, o.x, o.y);
+        *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(row) * Mp + ch * 16) = o;
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int64_t row = row0 + r;
+        if (row < M) *reinterpret_cast<uint2*>(q + row * K + col0) = make_uint2(clo[r], chi[r]);
+      }
+    }
+    __syncthreads();  // col_max, and this stage (refilled by the next iteration's copies), are reused
   }
+  cp_async_wait<0>();  // only empty groups can be pending here
 }
 
 // ---------------------------------------------------------------------------
@@ -645,12 +676,15 @@ __global__ void __launch_bounds__(256) transpose_w_128x128_kernel(const uint8_t*
 // configurations' GEMM1 width, twice GEMM2's depth, implies it.)
 //
 // h is the correctly rounded bf16 of the expression.  The FP32 evaluation
-// (expf within 2 ulp, three rounded operations: relative error below 2^-21)
-// is bracketed by h (1 -+ 2^-20); when both ends round to the same bf16, that
-// is the result (rounding is monotone).  Otherwise -- a value within ~2^-20 of
-// a bf16 rounding midpoint, or outside the range where the bound holds -- the
+// (expf within 2 ulp, the quotient by div.full.f32 within 2 ulp, one rounded
+// add and one rounded multiply: relative error below 2.5 * 2^-22) is
+// bracketed by h (1 -+ 2^-20); when both ends round to the same bf16, that is
+// the result (rounding is monotone).  Otherwise -- a value within ~2^-20 of a
+// bf16 rounding midpoint, or outside the range where the bound holds -- the
 // expression is evaluated in double and rounded to bf16 through round-to-odd
-// FP32 (16 spare bits, so the two steps round once).
+// FP32 (16 spare bits, so the two steps round once).  The FP32 evaluation and
+// the bracket are branch-free; the elements the bracket leaves open (about one
+// in 2^11) are redone afterwards.
 // ---------------------------------------------------------------------------
 __device__ __noinline__ uint32_t swiglu_bf16_exact(float g, float u) {
   const double hd = static_cast<double>(g) / (1.0 + exp(-static_cast<double>(g))) * static_cast<double>(u);
@@ -659,25 +693,61 @@ __device__ __noinline__ uint32_t swiglu_bf16_exact(float g, float u) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
-__device__ __forceinline__ uint32_t swiglu_bf16(float g, float u) {
+// a / b within 2 ulp for all finite a, b (PTX div.full.f32): no branch.
+__device__ __forceinline__ float div_full(float a, float b) {
+  float r;
+  asm("div.full.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// Two floats rounded to nearest-even bf16, packed (lo in the low half).
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// FP32 g / (1 + exp(-g)) * u; `ok` when exp did not overflow and |h| lies in
+// [2^-100, 2^120], where the relative error bound holds.
+__device__ __forceinline__ float swiglu_f32(float g, float u, bool& ok) {
   const float e = expf(-g);
-  const float h = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, e)), u);
+  const float h = __fmul_rn(div_full(g, __fadd_rn(1.0f, e)), u);
   const float a = fabsf(h);
-  if (isfinite(e) && a >= 0x1p-100f && a <= 0x1p+120f) {
-    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(h, 1.0f - 0x1p-20f)));
-    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(h, 1.0f + 0x1p-20f)));
-    if (lo == hi) return lo;
-  }
-  return swiglu_bf16_exact(g, u);
+  ok = e <= 0x1.fffffep+127f && a >= 0x1p-100f && a <= 0x1p+120f;
+  return h;
 }
 
 // Eight words of bf16 pairs (gate) and (up) -> eight words of bf16 pairs of h.
-__device__ __forceinline__ void swiglu16(const uint32_t (&gw)[8], const uint32_t (&uw)[8], uint32_t (&hw)[8]) {
+// gp, up: where gw and uw were loaded from; the rare redo path reads its
+// word there again rather than keeping all sixteen words live.
+__device__ __forceinline__ void swiglu16(const uint32_t (&gw)[8], const uint32_t (&uw)[8], uint32_t (&hw)[8],
+                                         const uint8_t* gp, const uint8_t* up) {
+  uint32_t redo = 0u;  // bit 2i + j: the half j of word i is left open by its bracket
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t h0 = swiglu_bf16(__uint_as_float(gw[i] << 16), __uint_as_float(uw[i] << 16));
-    const uint32_t h1 = swiglu_bf16(__uint_as_float(gw[i] & 0xFFFF0000u), __uint_as_float(uw[i] & 0xFFFF0000u));
-    hw[i] = h0 | (h1 << 16);
+    bool ok0, ok1;
+    const float h0 = swiglu_f32(__uint_as_float(gw[i] << 16), __uint_as_float(uw[i] << 16), ok0);
+    const float h1 = swiglu_f32(__uint_as_float(gw[i] & 0xFFFF0000u), __uint_as_float(uw[i] & 0xFFFF0000u), ok1);
+    const uint32_t lo = bf16x2_rn(__fmul_rn(h0, 1.0f - 0x1p-20f), __fmul_rn(h1, 1.0f - 0x1p-20f));
+    const uint32_t hi = bf16x2_rn(__fmul_rn(h0, 1.0f + 0x1p-20f), __fmul_rn(h1, 1.0f + 0x1p-20f));
+    hw[i] = lo;
+    const uint32_t d = lo ^ hi;
+    redo |= static_cast<uint32_t>(!ok0 || (d & 0xFFFFu) != 0u) << (2 * i);
+    redo |= static_cast<uint32_t>(!ok1 || (d >> 16) != 0u) << (2 * i + 1);
+  }
+  for (; redo != 0u; redo &= redo - 1u) {
+    const int b = __ffs(redo) - 1, i = b >> 1;
+    const uint32_t g = __ldg(reinterpret_cast<const uint32_t*>(gp) + i);
+    const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(up) + i);
+    if (b & 1) {
+      const uint32_t x = swiglu_bf16_exact(__uint_as_float(g & 0xFFFF0000u), __uint_as_float(u & 0xFFFF0000u));
+#pragma unroll
+      for (int k = 0; k < 8; ++k) hw[k] = i == k ? (hw[k] & 0xFFFFu) | (x << 16) : hw[k];
+    } else {
+      const uint32_t x = swiglu_bf16_exact(__uint_as_float(g << 16), __uint_as_float(u << 16));
+#pragma unroll
+      for (int k = 0; k < 8; ++k) hw[k] = i == k ? (hw[k] & 0xFFFF0000u) | x : hw[k];
+    }
   }
 }
 
@@ -710,7 +780,7 @@ __global__ void __launch_bounds__(256, 5) swiglu_quant_1x128_kernel(const uint8_
       const uint8_t* src = c1 + ((row * 2 * inter) + kb * 128 + sub * 16) * 2;
       ld_nc_v8(src, gw);
       ld_nc_v8(src + inter * 2, uw);
-      swiglu16(gw, uw, hw);
+      swiglu16(gw, uw, hw, src, src + inter * 2);
     } else {
       zero8(hw);
     }

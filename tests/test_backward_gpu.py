@@ -35,7 +35,9 @@ def _bits(rng, shape, scale=1.0, outliers=0, chan=False):
     return wl.bf16_bits(x)
 
 
-@pytest.mark.parametrize("M,K", [(128, 128), (256, 384), (200, 256), (1, 128), (1000, 640)])
+# (3000, 7168): 24 x 56 = 1344 blocks, about 4.5 per CTA of the persistent
+# grid (2 per SM), so every CTA cycles through all three shared stages
+@pytest.mark.parametrize("M,K", [(128, 128), (256, 384), (200, 256), (1, 128), (1000, 640), (3000, 7168)])
 def test_token_axis_quant_matches_oracle(dev, M, K):
     rng = np.random.default_rng(M * 7 + K)
     x = _bits(rng, (M, K), outliers=max(1, M * K // 5000), chan=True)
@@ -49,7 +51,8 @@ def test_token_axis_quant_matches_oracle(dev, M, K):
     assert np.array_equal(bytes_of(q).reshape(M, K), oq)
 
 
-def test_token_axis_quant_every_bf16_amax(dev):
+@pytest.mark.parametrize("token_contiguous", [False, True])
+def test_token_axis_quant_every_bf16_amax(dev, token_contiguous):
     """Every 16th finite non-negative bf16 value as the amax of one group."""
     amax_bits = np.arange(0, 0x7F80, 16, dtype=np.uint32)
     a = (amax_bits << 16).view(np.float32)
@@ -61,11 +64,16 @@ def test_token_axis_quant_every_bf16_amax(dev):
     xb[7, :] = amax_bits.astype(np.uint16)        # the amax of each channel's group
     K = (g + TILE - 1) // TILE * TILE
     xb = np.pad(xb, ((0, 0), (0, K - g)))
-    q, s = fq.fp8_quant_act_128x1(to_torch_bf16(xb, dev))
-    torch.cuda.synchronize(dev)
     oq, os_ = oracle.quant_act_128x1(xb)
+    if token_contiguous:
+        qt, s = fq.fp8_quant_act_128x1_t(to_torch_bf16(xb, dev), Mp=TILE)
+        torch.cuda.synchronize(dev)
+        assert np.array_equal(bytes_of(qt).reshape(K, TILE), np.ascontiguousarray(oq.T))
+    else:
+        q, s = fq.fp8_quant_act_128x1(to_torch_bf16(xb, dev))
+        torch.cuda.synchronize(dev)
+        assert np.array_equal(bytes_of(q).reshape(xb.shape), oq)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
-    assert np.array_equal(bytes_of(q).reshape(xb.shape), oq)
 
 
 @pytest.mark.parametrize("shape", [(128, 128), (256, 384), (3, 128, 256)])
@@ -103,7 +111,7 @@ def _pad_tokens(x, Mp):
 
 
 @pytest.mark.parametrize("M,K,pad", [(128, 128, 128), (256, 384, 512), (200, 256, 128), (1, 128, 512),
-                                     (1000, 640, 128), (1000, 640, 512)])
+                                     (1000, 640, 128), (1000, 640, 512), (3000, 7168, 512)])
 def test_token_contiguous_quant_matches_oracle(dev, M, K, pad):
     """Token-axis groups with the codes written token-contiguous: qt[k, m] is
     the code of x[m, k]; padding tokens (m >= M) get code 0 and groups made

@@ -43,8 +43,8 @@ def test_act_1x128_covers_every_element_once(M, K, grid):
 
 
 def act_128x1_map(M, K, grid):
-    """quant_act_128x1_kernel: one 128x128 block per CTA step; thread t owns
-    channels 8*(t%16)..+7 of rows 8*(t/16)..+7; rows past M are skipped."""
+    """quant_act_128x1_kernel<false>: one 128x128 block per CTA step; thread t
+    owns channels 8*(t%16)..+7 of rows 8*(t/16)..+7; rows past M are skipped."""
     nkc, nmb = K // TILE, -(-M // TILE)
     blocks = nmb * nkc
     written = np.zeros((M, K), dtype=np.int32)
@@ -149,9 +149,9 @@ def test_transpose_warp_stores_are_full_rows():
 
 
 def test_launch_caps_leave_no_work_behind():
-    """The launchers cap the grid (SMs x 10, x 16, x 64); the grid-stride loops
-    above cover any count of blocks with any positive grid."""
-    for blocks, cap in [(10, 1480), (5000, 1480), (1, 2368), (9999, 2368)]:
+    """The launchers cap the grid (SMs x 2, x 10, x 16, x 64); the grid-stride
+    loops above cover any count of blocks with any positive grid."""
+    for blocks, cap in [(10, 1480), (5000, 1480), (1, 2368), (9999, 2368), (1792, 296), (5, 296)]:
         grid = min(blocks, cap)
         covered = sum(len(range(bx, blocks, grid)) for bx in range(grid))
         assert covered == blocks
@@ -193,9 +193,9 @@ def test_byte_transpose_8x8():
 
 
 def act_128x1_t_map(M, K, grid, Mp=None):
-    """quant_act_128x1_t_kernel: per 128x128 block, thread (cg = t % 16,
-    rg = t / 16) writes channel rows cg*8+c of the shared tile at physical
-    8-byte slot rg ^ cg; the store loop reads row c >> 3, 16-byte chunk
+    """quant_act_128x1_kernel<true>: per 128x128 block, thread (cg = t % 16,
+    rg = t / 16) writes channel rows cg*8+c of the shared tile (the block's
+    spent stage) at physical 8-byte slot rg ^ cg; the store loop reads row c >> 3, 16-byte chunk
     (c & 7) ^ (row >> 4), swapping halves when (row >> 3) is odd, and writes
     qt[kc*128 + row, mb*128 + 16*(c & 7) ...].  Returns the transposed codes
     of a matrix of distinct token/channel tags and the write counts."""
@@ -255,3 +255,143 @@ def test_act_128x1_t_shared_store_conflicts():
             slots = [(((t & 15) * 8 + c) * 128 + (((t >> 4) ^ (t & 15)) << 3)) % 128 // 8
                      for t in range(32 * w, 32 * w + 32)]
             assert sorted(slots) == sorted(list(range(16)) * 2)
+
+
+# ---------------------------------------------------------------- token-axis staging
+TOK_STAGES = 3
+TOK_BLOCK_BYTES = 128 * 256
+
+
+def token_axis_fetch_chunks():
+    """The copy map of one block: 16-byte chunk c = t + 256 i (t < 256,
+    i < 8) is token c >> 4, channels 8 (c & 15) .. +7, at shared byte
+    (c >> 4) * 256 + (c & 15) * 16 of the stage."""
+    for t in range(256):
+        for i in range(8):
+            c = t + 256 * i
+            row, ch = c >> 4, c & 15
+            yield t, row, ch, row * 256 + ch * 16
+
+
+def test_token_axis_copies_fill_each_stage_once_in_bounds():
+    seen = np.zeros(TOK_BLOCK_BYTES, dtype=np.int32)
+    for _, row, ch, off in token_axis_fetch_chunks():
+        assert 0 <= off and off + 16 <= TOK_BLOCK_BYTES
+        assert off == row * 256 + ch * 16 and row < 128 and ch < 16
+        seen[off:off + 16] += 1
+    assert np.all(seen == 1)
+    # a warp's copy instruction (fixed i) covers two whole 256-byte token rows
+    for w in range(8):
+        for i in range(8):
+            rows = {(t + 256 * i) >> 4 for t in range(32 * w, 32 * w + 32)}
+            assert len(rows) == 2
+
+
+def test_token_axis_register_reads_match_the_staged_layout():
+    """Thread (cg = t % 16, rg = t / 16) reads its 8 tokens x 8 channels at
+    stage byte (rg*8 + r) * 256 + cg * 16: the chunk the copy map put there."""
+    where = {}
+    for _, row, ch, off in token_axis_fetch_chunks():
+        where[off] = (row, ch * 8)
+    for t in range(256):
+        cg, rg = t & 15, t >> 4
+        for r in range(8):
+            assert where[(rg * 8 + r) * 256 + cg * 16] == (rg * 8 + r, cg * 8)
+
+
+def test_token_axis_copy_sources_stay_in_bounds():
+    """Tokens past M are zero-filled: no byte is read for them; the other
+    copies read inside x [M, K]."""
+    for M, K in [(1, 128), (200, 256), (129, 384)]:
+        nkc, nmb = K // 128, -(-M // 128)
+        for b in range(nmb * nkc):
+            mb, kc = divmod(b, nkc)
+            for _, row, ch, _ in token_axis_fetch_chunks():
+                grow = mb * 128 + row
+                if grow < M:
+                    src = (grow * K + kc * 128 + ch * 8) * 2
+                    assert 0 <= src and src + 16 <= M * K * 2
+
+
+def token_axis_pipeline(blocks, grid):
+    """Replays the kernel's stage bookkeeping per CTA: the prologue fills
+    stages 0 .. S-2 with the CTA's first blocks; iteration i (block
+    blockIdx + i * grid, stage st = i % S) refills the stage of iteration
+    i - 1 with block i + S - 1, commits one group (possibly empty) and waits
+    until at most S - 1 groups are pending.  Checks that a refill only hits a
+    stage whose block every thread has finished with, that the block read is
+    the one copied into the stage, and that its copy group is complete."""
+    order = []
+    for bx in range(min(blocks, grid)):
+        stage = [None] * TOK_STAGES        # block held (or being filled) per stage
+        groups = []                         # committed groups, in order: block or None
+        for j in range(TOK_STAGES - 1):
+            bj = bx + j * grid
+            if bj < blocks:
+                stage[j] = bj
+            groups.append(bj if bj < blocks else None)
+        st, i, b = 0, 0, bx
+        done = set()
+        while b < blocks:
+            bn = b + (TOK_STAGES - 1) * grid
+            refill = TOK_STAGES - 1 if st == 0 else st - 1
+            if bn < blocks:
+                assert stage[refill] is None or stage[refill] in done
+                stage[refill] = bn
+            groups.append(bn if bn < blocks else None)
+            complete = groups[:len(groups) - (TOK_STAGES - 1)]   # wait_group(S - 1)
+            assert b in complete
+            assert stage[st] == b
+            order.append(b)
+            done.add(b)
+            b += grid
+            i += 1
+            st = 0 if st + 1 == TOK_STAGES else st + 1
+    return order
+
+
+@pytest.mark.parametrize("blocks,grid", [(1, 296), (5, 296), (296, 296), (297, 296), (1792, 296), (40, 3),
+                                         (7, 2), (3, 1)])
+def test_token_axis_pipeline_processes_every_block_once(blocks, grid):
+    order = token_axis_pipeline(blocks, grid)
+    assert sorted(order) == list(range(blocks))
+
+
+def test_token_axis_shared_memory_fits_the_ctas_per_sm():
+    """Three 32 KB stages plus the 4 KB channel-maxima array per CTA, two CTAs
+    per SM, within the 228 KB an SM offers (1 KB reserved per CTA)."""
+    per_cta = TOK_STAGES * TOK_BLOCK_BYTES + 8 * 16 * 8 * 4 + 1024
+    assert 2 * per_cta <= 228 * 1024
+    assert TOK_STAGES * TOK_BLOCK_BYTES <= 227 * 1024
+
+
+# ---------------------------------------------------------------- per-element exact codes
+def nonzero_bytes(d):
+    """Restates the quantizers' nonzero_bytes: bit 8j + 7 set when byte j of d is nonzero."""
+    return (((d & 0x7F7F7F7F) + 0x7F7F7F7F) | d) & 0x80808080
+
+
+def test_nonzero_bytes_marks_exactly_the_nonzero_bytes():
+    rng = np.random.default_rng(3)
+    words = [0, 0xFFFFFFFF, 0x80808080, 0x01010101, 0x7F7F7F7F, 0x00800001]
+    words += [int(v) for v in rng.integers(0, 2 ** 32, 2000, dtype=np.uint64)]
+    # every byte value in every position, the other bytes zero
+    words += [b << (8 * j) for j in range(4) for b in range(256)]
+    for d in words:
+        want = sum(0x80 << (8 * j) for j in range(4) if (d >> (8 * j)) & 0xFF)
+        assert nonzero_bytes(d) == want, hex(d)
+
+
+def test_code_byte_names_its_source_element():
+    """Code word i of a lane's 16 codes holds elements 4i .. 4i+3: byte j is the
+    bf16 at word 2i + j/2, half j%2 (low half first), the order in which the
+    packed products are converted.  bf16_of_pair must pick that element."""
+    bf16 = np.arange(16, dtype=np.uint32) + 0x3F80      # distinct bf16 patterns, element e at index e
+    w = [int(bf16[2 * k]) | (int(bf16[2 * k + 1]) << 16) for k in range(8)]
+    for i in range(4):
+        # conversion order: pairs (w[2i] low, high), (w[2i+1] low, high) -> bytes 0..3
+        converted = [w[2 * i] & 0xFFFF, w[2 * i] >> 16, w[2 * i + 1] & 0xFFFF, w[2 * i + 1] >> 16]
+        for j in range(4):
+            word = w[2 * i + 1] if j & 2 else w[2 * i]
+            picked = (word >> 16) if j & 1 else (word & 0xFFFF)
+            assert picked == converted[j] == int(bf16[4 * i + j])

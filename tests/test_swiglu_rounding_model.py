@@ -3,11 +3,12 @@
 The fused SwiGLU + requantization kernel must produce h = the correctly
 rounded bf16 of g / (1 + exp(-g)) * u.  It evaluates the expression in FP32,
 brackets the result by (1 -+ 2^-20) -- wider than the evaluation's error
-bound, about 1.75 * 2^-22 with an exp within 2 ulp -- and keeps the bf16 both
-ends round to; otherwise it evaluates in double and rounds to bf16 through
-round-to-odd FP32.  These tests restate both steps with numpy (FP32 exp as a
-stand-in for the device's, which has the same 2-ulp bound) and check them
-against exact rounding of the real value.
+bound, below 2.5 * 2^-22 with the exp and the quotient each within 2 ulp
+(expf; div.full.f32) -- and keeps the bf16 both ends round to; otherwise it
+evaluates in double and rounds to bf16 through round-to-odd FP32.  These
+tests restate both steps with numpy, with the exp and the quotient each moved
+by a random whole number of ulps in [-2, 2] (the device's worst cases lie in
+that range), and check them against exact rounding of the real value.
 """
 import math
 from fractions import Fraction
@@ -49,12 +50,28 @@ def near_midpoint(v: float, rel: float = 1e-12) -> bool:
     return min(abs(abs(v) - (abs(lo) + half_ulp)), abs(abs(v) - (abs(lo) - half_ulp))) <= rel * abs(v)
 
 
-def fast_path(g: np.ndarray, u: np.ndarray):
-    """FP32 evaluation and the bracket test; returns (bf16 bits, decided mask)."""
+def ulp_shift(x: np.ndarray, k: np.ndarray) -> np.ndarray:
+    """x moved by k (|k| <= 2) units in the last place, binary32."""
+    x = x.astype(np.float32).copy()
+    with np.errstate(over="ignore", invalid="ignore"):
+        for step in (1, 2):
+            up, dn = k >= step, k <= -step
+            x[up] = np.nextafter(x[up], np.float32(np.inf), dtype=np.float32)
+            x[dn] = np.nextafter(x[dn], np.float32(-np.inf), dtype=np.float32)
+    return x
+
+
+def fast_path(g: np.ndarray, u: np.ndarray, rng=None):
+    """FP32 evaluation and the bracket test; returns (bf16 bits, decided mask).
+    With rng, the exp and the quotient are each moved by up to 2 ulp."""
     with np.errstate(over="ignore", under="ignore", invalid="ignore", divide="ignore"):
         e = np.exp(-g).astype(np.float32)
-        h = (g / (np.float32(1.0) + e)).astype(np.float32) * u
-        h = h.astype(np.float32)
+        if rng is not None:
+            e = ulp_shift(e, rng.integers(-2, 3, e.size))
+        q = (g / (np.float32(1.0) + e)).astype(np.float32)
+        if rng is not None:
+            q = ulp_shift(q, rng.integers(-2, 3, q.size))
+        h = (q * u).astype(np.float32)
         lo = (h * np.float32(1.0 - 2.0 ** -20)).astype(np.float32)
         hi = (h * np.float32(1.0 + 2.0 ** -20)).astype(np.float32)
     a = np.abs(h)
@@ -69,7 +86,7 @@ def test_fast_path_is_correctly_rounded():
     # GEMM1 outputs: gates of a few units, wide range of up values, some far gates
     g = bf16_to_f32(bf16_bits((rng.standard_normal(n) * np.exp(rng.uniform(-6, 3, n))).astype(np.float32)))
     u = bf16_to_f32(bf16_bits((rng.standard_normal(n) * np.exp(rng.uniform(-6, 5, n))).astype(np.float32)))
-    bits, decided = fast_path(g, u)
+    bits, decided = fast_path(g, u, rng=np.random.default_rng(7))
     idx = np.flatnonzero(decided)
     assert decided.mean() > 0.998          # the double path is rare
     for i in idx[:: max(1, idx.size // 20000)]:
