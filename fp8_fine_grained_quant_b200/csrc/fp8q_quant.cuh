@@ -444,7 +444,12 @@ __global__ void __launch_bounds__(256, kTokCtasPerSm) quant_act_128x1_kernel(con
                                                                              int64_t K, int64_t Mp,
                                                                              int64_t num_blocks) {
   extern __shared__ __align__(128) uint8_t stage_buf[];  // [kTokStages][128 tokens][256 bytes]
-  __shared__ float col_max[8][16][8];                    // [warp][column group][column]
+  __shared__ __align__(16) uint32_t col_max[8][16][4];   // [warp][channel group][word]: bf16 maxima, packed
+  // per channel of the block: scale, bracketing reciprocals, whether its codes take the division path
+  __shared__ __align__(16) float ch_scale[128];
+  __shared__ __align__(16) float ch_rlo[128];
+  __shared__ __align__(16) float ch_rhi[128];
+  __shared__ __align__(8) uint8_t ch_exact[128];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cg = tid & 15, rg = tid >> 4;
   // block b = mb * nkc + kc; a CTA's blocks are gridDim.x apart, i.e. step_mb
@@ -502,51 +507,56 @@ __global__ void __launch_bounds__(256, kTokCtasPerSm) quant_act_128x1_kernel(con
     uint4 v[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) v[r] = *reinterpret_cast<const uint4*>(buf + (rg * 8 + r) * 256 + cg * 16);
-    // per-channel maxima over this thread's 8 tokens
-    float m[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) m[c] = 0.0f;
+    // per-channel maxima of |x| over this thread's 8 tokens, as packed bf16 pairs
+    // (word i: channels 2i and 2i + 1; a maximum of bf16 values is exact)
+    uint32_t m[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      const uint32_t w[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        m[2 * i] = fmaxf(m[2 * i], fabsf(__uint_as_float(w[i] << 16)));
-        m[2 * i + 1] = fmaxf(m[2 * i + 1], fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
-      }
+      m[0] = max_bf16x2(m[0], v[r].x & 0x7FFF7FFFu);
+      m[1] = max_bf16x2(m[1], v[r].y & 0x7FFF7FFFu);
+      m[2] = max_bf16x2(m[2], v[r].z & 0x7FFF7FFFu);
+      m[3] = max_bf16x2(m[3], v[r].w & 0x7FFF7FFFu);
     }
     // lanes l and l ^ 16 hold the same channels (two token groups of the warp)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) m[c] = fmaxf(m[c], __shfl_xor_sync(0xFFFFFFFFu, m[c], 16));
-    if (lane < 16) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) col_max[warp][cg][c] = m[c];
-    }
+    for (int i = 0; i < 4; ++i) m[i] = max_bf16x2(m[i], __shfl_xor_sync(0xFFFFFFFFu, m[i], 16));
+    if (lane < 16) *reinterpret_cast<uint4*>(&col_max[warp][cg][0]) = make_uint4(m[0], m[1], m[2], m[3]);
     __syncthreads();  // col_max is complete, and the stage has been read by every thread
-    float sc[8];
+    // one thread per channel: its amax over the 8 warps, scale and bracket, once for the block
+    if (tid < 128) {
+      uint32_t a = 0u;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float a = col_max[0][cg][c];
-#pragma unroll
-      for (int w = 1; w < 8; ++w) a = fmaxf(a, col_max[w][cg][c]);
-      sc[c] = group_scale(a);
+      for (int w = 0; w < 8; ++w) a = max_bf16x2(a, col_max[w][tid >> 3][(tid & 7) >> 1]);
+      const float amax = __uint_as_float((tid & 1) ? (a & 0xFFFF0000u) : (a << 16));
+      const float sc = group_scale(amax);
+      float lo, hi;
+      const bool ok = recip_bracket(sc, lo, hi);
+      ch_scale[tid] = sc;
+      ch_rlo[tid] = lo;
+      ch_rhi[tid] = hi;
+      ch_exact[tid] = static_cast<uint8_t>(sc < kMinFastScale || !ok);
+      s[mb * K + static_cast<int64_t>(kc) * 128 + tid] = sc;
     }
-    if (rg == 0) {
-      float* sd = s + mb * K + col0;
-      *reinterpret_cast<float4*>(sd) = make_float4(sc[0], sc[1], sc[2], sc[3]);
-      *reinterpret_cast<float4*>(sd + 4) = make_float4(sc[4], sc[5], sc[6], sc[7]);
-    }
-    // bracketing reciprocals per channel, paired as the packed products need them
+    __syncthreads();
+    // this thread's 8 channels' bracketing reciprocals, paired as the packed products need them
     uint64_t lo2[4], hi2[4];
-    bool exact_only = false;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float l0, h0, l1, h1;
-      const bool ok0 = recip_bracket(sc[2 * i], l0, h0), ok1 = recip_bracket(sc[2 * i + 1], l1, h1);
-      asm("mov.b64 %0, {%1, %2};" : "=l"(lo2[i]) : "f"(l0), "f"(l1));
-      asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[i]) : "f"(h0), "f"(h1));
-      exact_only |= sc[2 * i] < kMinFastScale || sc[2 * i + 1] < kMinFastScale || !ok0 || !ok1;
+    {
+      const float4 l0 = *reinterpret_cast<const float4*>(&ch_rlo[cg * 8]);
+      const float4 l1 = *reinterpret_cast<const float4*>(&ch_rlo[cg * 8 + 4]);
+      const float4 h0 = *reinterpret_cast<const float4*>(&ch_rhi[cg * 8]);
+      const float4 h1 = *reinterpret_cast<const float4*>(&ch_rhi[cg * 8 + 4]);
+      asm("mov.b64 %0, {%1, %2};" : "=l"(lo2[0]) : "f"(l0.x), "f"(l0.y));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(lo2[1]) : "f"(l0.z), "f"(l0.w));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(lo2[2]) : "f"(l1.x), "f"(l1.y));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(lo2[3]) : "f"(l1.z), "f"(l1.w));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[0]) : "f"(h0.x), "f"(h0.y));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[1]) : "f"(h0.z), "f"(h0.w));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[2]) : "f"(h1.x), "f"(h1.y));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(hi2[3]) : "f"(h1.z), "f"(h1.w));
     }
+    const uint2 ex = *reinterpret_cast<const uint2*>(&ch_exact[cg * 8]);
+    const bool exact_only = (ex.x | ex.y) != 0u;
+    const float* my_scale = &ch_scale[cg * 8];
     // codes of the 8 tokens (zero tokens past M give code 0)
     uint32_t clo[8], chi[8];
 #pragma unroll
@@ -560,8 +570,8 @@ __global__ void __launch_bounds__(256, kTokCtasPerSm) quant_act_128x1_kernel(con
         hi[h] = e4m3x4_from_f32x2(mul_f32x2(x0, hi2[2 * h]), mul_f32x2(x1, hi2[2 * h + 1]));
       }
       if (exact_only) {
-        const uint2 out =
-            quantize8_cols_exact(w[0], w[1], w[2], w[3], sc[0], sc[1], sc[2], sc[3], sc[4], sc[5], sc[6], sc[7]);
+        const uint2 out = quantize8_cols_exact(w[0], w[1], w[2], w[3], my_scale[0], my_scale[1], my_scale[2],
+                                               my_scale[3], my_scale[4], my_scale[5], my_scale[6], my_scale[7]);
         lo[0] = out.x;
         lo[1] = out.y;
       } else {
@@ -570,8 +580,7 @@ __global__ void __launch_bounds__(256, kTokCtasPerSm) quant_act_128x1_kernel(con
         for (int h = 0; h < 2; ++h) {
           for (uint32_t mk = nonzero_bytes(lo[h] ^ hi[h]); mk != 0u; mk &= mk - 1u) {
             const int j = (__ffs(mk) - 1) >> 3;
-            const float sj = j == 0 ? sc[4 * h] : j == 1 ? sc[4 * h + 1] : j == 2 ? sc[4 * h + 2] : sc[4 * h + 3];
-            lo[h] = with_exact_code(lo[h], j, bf16_of_pair(w[2 * h], w[2 * h + 1], j), sj);
+            lo[h] = with_exact_code(lo[h], j, bf16_of_pair(w[2 * h], w[2 * h + 1], j), my_scale[4 * h + j]);
           }
         }
       }

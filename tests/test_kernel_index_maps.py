@@ -395,3 +395,16 @@ def test_code_byte_names_its_source_element():
             word = w[2 * i + 1] if j & 2 else w[2 * i]
             picked = (word >> 16) if j & 1 else (word & 0xFFFF)
             assert picked == converted[j] == int(bf16[4 * i + j])
+
+
+def test_token_axis_channel_maxima_reach_their_channel_thread():
+    """Thread (cg, lane < 16) stores its packed maxima word i (channels
+    8 cg + 2i, low half, and 8 cg + 2i + 1, high half) at col_max[warp][cg][i];
+    channel thread t < 128 reads word (t & 7) >> 1 of [warp][t >> 3], half t & 1."""
+    stored = {}
+    for cg in range(16):
+        for i in range(4):
+            stored[(cg, i, 0)] = 8 * cg + 2 * i
+            stored[(cg, i, 1)] = 8 * cg + 2 * i + 1
+    for t in range(128):
+        assert stored[(t >> 3, (t & 7) >> 1, t & 1)] == t
