@@ -131,3 +131,21 @@ def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(tmp_path, monk
     assert bench.traffic_for("gemm_blockscaled", "dense_fprop") == 123
     assert bench.traffic_for("quant_act_w", "dense_fprop") is None      # taken on other sources
     assert bench.traffic_for("gemm_blockscaled", "long_k") is None       # never taken
+
+
+def test_profile_sizes_shrink_the_workloads_they_name(monkeypatch):
+    """--profile-size keeps each named workload's layout with fewer rows or
+    experts (captures that take many passes stay small); the chained MoE decode
+    takes the masked layout with 8 experts.  The generators are stubbed: only
+    the arguments make_workload passes are checked."""
+    calls = []
+    monkeypatch.setattr(wl, "moe_masked", lambda **kw: calls.append(("moe_masked", kw)) or "masked")
+    monkeypatch.setitem(wl.CONFIGS, "dense_fprop", lambda **kw: calls.append(("dense_fprop", kw)) or "dense")
+    monkeypatch.setattr(bench, "PROFILE_SIZE", True)
+    assert bench.make_workload("moe_masked_chain") == "masked"
+    assert bench.make_workload("dense_fprop") == "dense"
+    assert calls == [("moe_masked", {"device": None, "E": 8}), ("dense_fprop", {"M": 2048})]
+    monkeypatch.setattr(bench, "PROFILE_SIZE", False)
+    calls.clear()
+    assert bench.make_workload("moe_masked_chain") == "masked"
+    assert calls == [("moe_masked", {"shard": 0, "device": None})]
